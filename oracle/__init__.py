@@ -1,0 +1,105 @@
+"""Oracle for the attention forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  The product path (``tiled_attention_15_b200``)
+never imports it, and it never imports the product path.
+
+``attention(q, k, v, scale, causal, rows=None)`` is the plain three-pass
+definition of attention in double precision (S = scale*Q K^T, row softmax,
+times V), written in C (``attn_oracle.c``) and run on the host cores with
+OpenMP.  Source of the definition: the "standard attention" steps on the
+mooersco.com page (section "标准 Attention 的瓶颈在哪") and section 二 of the
+gitcode.csdn.net page; the scale 1/sqrt(head_dim) from the Scale step of the
+hwcomputing.csdn.net page's fused-kernel listing.  Every function of this
+package is pinned by ``tests/test_oracle.py`` against values fixed by the pages
+and by mathematics (see that file's header); nothing here is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``attn_oracle.c`` with gcc (-O2 -fopenmp, no fast-math) into liboracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        lib.oracle_attention.restype = ctypes.c_int
+        lib.oracle_attention.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
+            ctypes.c_int]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _as_f32(x) -> np.ndarray:
+    """Widen a (rounded fp16/bf16) tensor or array to a contiguous float32 numpy array (exact)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu").float().numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def attention(q, k, v, scale: float, causal: bool, rows: Optional[np.ndarray] = None,
+              nthreads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Reference attention in float64.
+
+    q: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] (torch tensors or numpy arrays).
+    rows: optional sorted int64 array of query positions; only those rows are
+    computed (then the result has R = len(rows) rows per head).
+    Returns (O [B, Hq, R, D] float64, LSE [B, Hq, R] float64).
+    """
+    lib = _load()
+    qf, kf, vf = _as_f32(q), _as_f32(k), _as_f32(v)
+    B, Hq, Nq, D = qf.shape
+    Bk, Hkv, Nk, Dk = kf.shape
+    if (Bk, Dk) != (B, D) or vf.shape != kf.shape:
+        raise ValueError("shape mismatch between q, k, v")
+    if rows is not None:
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        if rows.ndim != 1 or rows.size == 0 or rows.min() < 0 or rows.max() >= Nq:
+            raise ValueError("rows must be a non-empty 1-D array of positions in [0, Nq)")
+        qf = np.ascontiguousarray(qf[:, :, rows, :])
+        R = int(rows.shape[0])
+        pos_ptr = rows.ctypes.data
+    else:
+        R = Nq
+        pos_ptr = None
+    o = np.empty((B, Hq, R, D), dtype=np.float64)
+    lse = np.empty((B, Hq, R), dtype=np.float64)
+    rc = lib.oracle_attention(qf.ctypes.data, pos_ptr, R, kf.ctypes.data, vf.ctypes.data,
+                              o.ctypes.data, lse.ctypes.data, B, Hq, Hkv, Nq, Nk, D,
+                              float(scale), int(bool(causal)), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_attention rejected its arguments (code {rc})")
+    return o, lse
