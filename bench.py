@@ -1,0 +1,381 @@
+"""Benchmark of the fused attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one pass of the whole hot path over one batch of the LLaMA-7B
+attention-layer workload (B=2, Hq=Hkv=32, N=2048, D=128, fp16,
+scale=1/sqrt(128)): the non-causal forward pass and the causal forward pass,
+both through the library's C ABI.  Inputs are synthetic (seeded N(0,1),
+rounded to fp16) and resident in HBM when timing starts; L2 is flushed
+(256 MiB write) between steps because the inputs (~100 MB) fit in L2.
+
+metric: attention forward TFLOP/s with FLOPs = 4*B*Hq*Nq*Nk*D (halved for the
+causal pass).  Prints one JSON line on rank 0.  For N > 1 (torchrun) every rank
+runs an independent copy of the workload (weak scaling, no data-path
+collective); time is the max over ranks.
+
+--impl reference times the CPU oracle (plain three-pass fp64 attention) on the
+host cores on bounded row samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd TFLOP/s (4·B·Hq·Nq·Nk·D, ½ if causal) and % of B200 dense FP16 peak"
+SPEC_PEAK_TFLOPS = 2250.0
+FALLBACK_PEAK_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gate", action="store_true", help="skip the N=4096/8192 gate configs")
+    return ap.parse_args()
+
+
+def workloads():
+    from fa_inputs import llama7b
+    return [llama7b(False), llama7b(True)]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return FALLBACK_PEAK_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tiled_attention_15_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel."""
+    p = os.path.join(ROOT, "profiles", "fa_fwd_d128_llama7b_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if "=" in line and not line.startswith("#"):
+                a, b = line.split("=", 1)
+                kv[a.strip()] = b.strip()
+    if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """NVML samples of SM clock and clock-event reasons while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.ok = False
+        self.samples, self.reasons = [], set()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def oracle_sample(ws, rows_per_head: int, seed: int, qkv=None):
+    """Run the oracle on a seeded sample of query rows of every head; returns (flops, seconds)."""
+    import numpy as np
+    import oracle
+    from fa_inputs import make_qkv, sample_rows
+    flops, secs = 0.0, 0.0
+    for w in ws:
+        q, k, v = qkv if qkv is not None else make_qkv(w)
+        rows = sample_rows(w.Nq, rows_per_head, seed)
+        vis = np.minimum(rows + 1, w.Nk) if w.causal else np.full(len(rows), w.Nk)
+        flops += 4.0 * w.D * float(vis.sum()) * w.B * w.Hq
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, w.softmax_scale, w.causal, rows=rows)
+        secs += time.perf_counter() - t0
+    return flops, secs
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    from fa_inputs import make_qkv
+    ws = workloads()
+    qkv = make_qkv(ws[0])  # both passes use the same seed-0 draws
+    rows = 32
+    for i in range(args.warmup):
+        oracle_sample(ws, rows, 1000 + i, qkv)
+    flops = secs = 0.0
+    for i in range(args.steps):
+        f, s = oracle_sample(ws, rows, i, qkv)
+        flops += f
+        secs += s
+    tflops = flops / secs / 1e12
+    cores = oracle.max_threads()
+    sample = (f"{rows} seeded query rows per (b, head) of each pass (non-causal, causal) per step; "
+              f"{args.steps} steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), rounded to fp16)",
+        "config": {"workload": "llama7b-attn B2 Hq32 Hkv32 N2048 D128 fp16, non-causal + causal",
+                   "B": 2, "Hq": 32, "Hkv": 32, "N": 2048, "D": 128},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- CUDA arm
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import tiled_attention_15_b200 as fa
+    from fa_inputs import make_qkv
+
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    ws = workloads()
+    inputs = []
+    for w in ws:
+        q, k, v = make_qkv(w)
+        inputs.append((w, q, k, v))
+    # the non-causal and causal passes share the same Q, K, V draws (seed 0)
+    q, k, v = (x.to(dev) for x in inputs[0][1:])
+    outs = [(torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev))
+            for _ in ws]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    def step():
+        for w, (o, lse) in zip(ws, outs):
+            fa.fa_fwd(q, k, v, o=o, lse=lse, scale=w.softmax_scale, causal=w.causal, stream=sptr)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert fa.device_status(reset=True) == 0
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ws) + 1)] for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.zero_()
+            e = ev[i]
+            e[0].record(stream)
+            for j, (w, (o, lse)) in enumerate(zip(ws, outs)):
+                fa.fa_fwd(q, k, v, o=o, lse=lse, scale=w.softmax_scale, causal=w.causal,
+                          stream=sptr)
+                e[j + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    per_launch = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)] for j in range(len(ws))]
+    step_ms = [sum(per_launch[j][i] for j in range(len(ws))) for i in range(K)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    assert fa.device_status(reset=True) == 0
+    flops_step = sum(w.flops() for w in ws)
+    value = world * flops_step * K / (total_ms * 1e-3) / 1e12
+
+    # ---- end to end: pinned host inputs -> device -> both passes -> O and LSE back to host
+    hq, hk, hv = (x.pin_memory() for x in inputs[0][1:])
+    ho = [(torch.empty(q.shape, dtype=q.dtype, pin_memory=True),
+           torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)) for _ in ws]
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in ho)
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    E = max(10, K // 20)
+
+    def e2e_step():
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        for w, (o, lse), (h_o, h_l) in zip(ws, outs, ho):
+            fa.fa_fwd(qd, kd, vd, o=o, lse=lse, scale=w.softmax_scale, causal=w.causal, stream=sptr)
+            h_o.copy_(o, non_blocking=True)
+            h_l.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops_step * E / (e2e_ms * 1e-3) / 1e12
+
+    # ---- gate configs (N = 4096 / 8192, D = 128), a few launches each, L2 flushed
+    gate = {}
+    if not args.no_gate:
+        from fa_inputs import seq_sweep
+        for n in (4096, 8192):
+            w0 = seq_sweep(n, False)
+            gq, gk, gv = (x.to(dev) for x in make_qkv(w0))
+            go, gl = torch.empty_like(gq), torch.empty(gq.shape[:3], dtype=torch.float32, device=dev)
+            for causal in (False, True):
+                w = seq_sweep(n, causal)
+                ts = []
+                for i in range(13):
+                    flush.zero_()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    fa.fa_fwd(gq, gk, gv, o=go, lse=gl, scale=w.softmax_scale, causal=causal,
+                              stream=sptr)
+                    b.record(stream)
+                    torch.cuda.synchronize()
+                    if i >= 3:
+                        ts.append(a.elapsed_time(b))
+                ms = statistics.median(ts)
+                gate[f"N{n}_{'causal' if causal else 'noncausal'}"] = {
+                    "ms": round(ms, 4), "tflops": round(w.flops() / (ms * 1e-3) / 1e12, 1)}
+            del gq, gk, gv, go, gl
+        assert fa.device_status(reset=True) == 0
+
+    peak, peak_sus, peak_kind = peaks()
+    launch_ms = total_ms / world / (K * len(ws)) if world > 1 else total_ms / (K * len(ws))
+    achieved = (flops_step / len(ws)) / (launch_ms * 1e-3) / 1e12
+    traffic = recorded_traffic()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+        "data": "synthetic (seeded N(0,1), rounded to fp16; scale 1/sqrt(128))",
+        "config": {"workload": "llama7b-attn B2 Hq32 Hkv32 N2048 D128 fp16, non-causal + causal",
+                   "B": 2, "Hq": 32, "Hkv": 32, "N": 2048, "D": 128,
+                   "passes_per_step": ["non-causal", "causal"],
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+        "pct_of_peak": {"measured_burst": round(100 * value / world / peak, 1),
+                        "measured_sustained": round(100 * value / world / peak_sus, 1),
+                        "spec_2250": round(100 * value / world / SPEC_PEAK_TFLOPS, 1),
+                        "peak_source": peak_kind},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic,
+                     "kernel": "fa::fa_fwd_kernel<128, 2, false> (fp16, D=128)",
+                     "peak_note": f"{peak_kind} bf16 dense burst (fp16:bf16 nominal ratio 1:1)"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * len(ws),
+        "clocks": clk.summary(),
+        "gate_d128": gate,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        f, s = oracle_sample(ws, 512, 0, tuple(x for x in inputs[0][1:]))
+        line["cpu_baseline"] = {
+            "value": f / s / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": "512 seeded query rows per (b, head) of each pass (non-causal, causal); "
+                      f"{f / 1e9:.1f} GFLOP in {s:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

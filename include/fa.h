@@ -1,0 +1,114 @@
+/*
+ * fa.h -- C ABI of the fused, tiled attention forward pass for NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources: "FlashAttention 算子" article on mooersco.com, sections
+ * "标准 Attention 的瓶颈在哪" and "昇腾NPU上的分块策略"):
+ *
+ *     O = softmax(scale * Q K^T  [with causal mask]) V
+ *
+ * computed block by block with an online softmax (running row maximum and row
+ * sum, partial output rescaled when the maximum moves), so that the Nq x Nk
+ * score and probability matrices never reach device memory.  The tensors are
+ * the [batch, heads, sequence, head_dim] fp16 tensors of the PyTorch call on
+ * that page ("通过 PyTorch 调用 FlashAttention"); head_dim is 64, 128 or 256
+ * as that section lists; causal masking is its is_causal flag; grouped-query
+ * and multi-query heads (Hkv < Hq) are those of section 六 of the
+ * gitcode.csdn.net article.
+ *
+ * Conventions shared by every entry point below
+ * ---------------------------------------------
+ * Layout     q, o: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D]; all contiguous
+ *            (row-major, D fastest), all of one 16-bit dtype.  lse: float32
+ *            [B, Hq, Nq], contiguous.
+ * Memory     q, k, v, o and lse are DEVICE pointers on the current CUDA device.
+ *            Each of q, k, v, o must be 16-byte aligned (tensor-memory-access
+ *            descriptors require it); lse must be 4-byte aligned.  The caller
+ *            owns every buffer; the library allocates no device memory and
+ *            keeps no per-call state.  o and lse must not overlap q, k or v.
+ * Heads      Hq must be a multiple of Hkv; query head h reads key/value head
+ *            h / (Hq / Hkv) (contiguous groups).
+ * Causal     causal != 0 keeps key j for query i iff j <= i (top-left
+ *            alignment, as PyTorch's scaled_dot_product_attention(is_causal=True)).
+ * Scale      any finite float, applied to the scores before the softmax; the
+ *            pages use 1/sqrt(D).  scale = 0 gives the plain average of V.
+ * LSE        lse[b,h,i] = ln sum_j exp(scale * q_i . k_j) over the visible keys
+ *            (natural log, scale included).  lse may be NULL: then it is not
+ *            written.
+ * Stream     `stream` is a cudaStream_t (NULL = legacy default stream).  The
+ *            call only enqueues work and returns; results are ready when the
+ *            stream reaches that point.
+ * Errors     every entry point returns FA_OK (0) or one of the fa_status codes
+ *            below.  Argument errors are detected on the host before anything
+ *            is enqueued; nothing is launched then.  Faults inside the kernel
+ *            are not reported by the return value: a kernel wait that exceeds
+ *            its time limit records FA_ERR_DEVICE_TIMEOUT in a device status
+ *            word that fa_device_status() reads.
+ * Threads    the entry points are thread-safe; per-device set-up (function
+ *            attributes, driver entry point) happens once, on first use.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum fa_dtype { FA_FP16 = 0, FA_BF16 = 1 };
+
+enum fa_status {
+  FA_OK = 0,
+  FA_ERR_NULL_POINTER = 1,         /* q, k, v or o is NULL                        */
+  FA_ERR_MISALIGNED = 2,           /* q, k, v, o not 16-byte aligned; lse not 4    */
+  FA_ERR_BAD_SHAPE = 3,            /* B, Hq, Hkv, Nq or Nk < 1, or sizes overflow  */
+  FA_ERR_BAD_GROUPING = 4,         /* Hq % Hkv != 0                               */
+  FA_ERR_UNSUPPORTED_HEAD_DIM = 5, /* D not in {64, 128, 256}                      */
+  FA_ERR_BAD_SCALE = 6,            /* scale is NaN or infinite                     */
+  FA_ERR_BAD_DTYPE = 7,            /* dtype not FA_FP16 or FA_BF16                 */
+  FA_ERR_NO_DEVICE = 8,            /* no current CUDA device, or it is not sm_100  */
+  FA_ERR_LAUNCH = 9,               /* the CUDA runtime refused the launch          */
+  FA_ERR_DRIVER = 10,              /* tensor-map encoding via the driver failed    */
+  FA_ERR_DEVICE_TIMEOUT = 11,      /* (device status) a kernel wait hit its limit  */
+  FA_ERR_OVERLAP = 12              /* o or lse overlaps q, k or v                  */
+};
+
+/*
+ * Fused attention forward (the operation above).
+ *   q, k, v   device inputs (see Layout); read only.
+ *   o         device output [B, Hq, Nq, D], same dtype as the inputs, rounded to
+ *             nearest even from the fp32 result.
+ *   lse       device output [B, Hq, Nq] float32, or NULL.
+ *   B         batch size;  Hq, Hkv  query and key/value heads;
+ *   Nq, Nk    query and key sequence lengths (any value >= 1; tails are masked);
+ *   D         head_dim, one of 64, 128, 256;
+ *   scale     score scale;  causal  0 or 1;
+ *   stream    cudaStream_t to enqueue on;
+ *   dtype     FA_FP16 or FA_BF16.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream, int dtype);
+
+/* fa_fwd with the dtype fixed (the fourteen-argument form). */
+int fa_fwd_fp16(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream);
+int fa_fwd_bf16(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream);
+
+/* Human-readable text for a status code (static storage; never NULL). */
+const char *fa_status_string(int status);
+
+/*
+ * Device status word of the current device: FA_OK, or FA_ERR_DEVICE_TIMEOUT if
+ * a kernel of this library gave up on a wait since the last reset.  Synchronises
+ * the device.  reset != 0 clears the word after reading it.  Returns a negative
+ * value if the word cannot be read (no device).
+ */
+int fa_device_status(int reset);
+
+/* Number of work tiles (CTAs' units of work) one fa_fwd call would schedule;
+ * 0 for invalid arguments.  Host only; used to count launches and to size tests. */
+long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FA_H_ */

@@ -1,0 +1,89 @@
+"""C-ABI tests that need no GPU: the library loads, exports every function
+include/fa.h declares, and rejects bad arguments on the host before any CUDA
+work (fake, never-dereferenced pointer values are enough for that)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import tiled_attention_15_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_attention_15_b200.csrc import build
+    build.build()
+    return fa.load_library()
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_binding_names():
+    assert sorted(fa.EXPORTED) == _declared()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (fa_[a-z0-9_]+)$", out, flags=re.M))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    for code in range(0, 13):
+        s = fa.status_string(code)
+        assert s and s != "unknown status", code
+    assert fa.status_string(99) == "unknown status"
+
+
+def test_num_tiles(lib):
+    # 256 query rows per work tile for D <= 128, 128 for D = 256
+    assert fa.num_tiles(2, 32, 2048, 128) == 2 * 32 * 8
+    assert fa.num_tiles(1, 1, 257, 64) == 2
+    assert fa.num_tiles(1, 2, 129, 256) == 4
+    assert fa.num_tiles(1, 1, 1, 96) == 0
+
+
+A = 1 << 20  # fake 16-byte-aligned addresses, far apart; never dereferenced
+GOOD = dict(q=1 * A, k=2 * A, v=3 * A, o=4 * A, lse=5 * A, B=1, Hq=4, Hkv=2, Nq=64, Nk=64, D=128,
+            scale=0.125, causal=0, stream=0, dtype=fa.FA_FP16)
+
+
+def _call(**kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_raw(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                         a["Nq"], a["Nk"], a["D"], a["scale"], a["causal"], a["stream"], a["dtype"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=2), 7),
+    (dict(D=96), 5), (dict(D=32), 5), (dict(D=0), 5),
+    (dict(B=0), 3), (dict(Hq=0), 3), (dict(Hkv=0), 3), (dict(Nq=0), 3), (dict(Nk=-1), 3),
+    (dict(Hq=6, Hkv=4), 4),
+    (dict(scale=float("nan")), 6), (dict(scale=float("inf")), 6),
+    (dict(q=0), 1), (dict(o=0), 1),
+    (dict(k=2 * A + 8), 2), (dict(lse=5 * A + 2), 2),
+    (dict(o=1 * A + 64), 12), (dict(lse=3 * A + 32), 12),
+])
+def test_host_argument_checks(lib, kw, code):
+    assert _call(**kw) == code
+
+
+def test_valid_arguments_reach_the_device_check(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-only check")
+    assert _call() == 8  # FA_ERR_NO_DEVICE without a GPU
+    assert _call(lse=0) == 8  # lse may be NULL

@@ -1,0 +1,151 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small and ragged shapes are compared on every output element; the workloads
+the pages measure on (LLaMA-7B layer, sequence sweep, GQA/MQA and head-dim
+sweep, 128K context) are compared on seeded samples of query rows (every head,
+rows 0 and N-1 always included), plus properties that hold at any size.
+
+Tolerances (max abs difference against the fp64 oracle): fp16 inputs O 4e-3
+and LSE 1e-3; bf16 inputs O 1.6e-2 and LSE 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tiled_attention_15_b200 as fa
+from fa_inputs import TINY, LONG, Workload, gqa, llama7b, make_qkv, sample_rows, seq_sweep
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp16": (4e-3, 1e-3), "bf16": (1.6e-2, 1e-3)}
+
+
+def run_cuda(w: Workload, dev, q=None, k=None, v=None):
+    if q is None:
+        q, k, v = make_qkv(w)
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    o, lse = fa.fa_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal)
+    torch.cuda.synchronize()
+    assert fa.device_status(reset=True) == 0
+    return (q, k, v), o, lse
+
+
+def compare(w: Workload, dev, rows=None):
+    (q, k, v), o, lse = run_cuda(w, dev)
+    ref_o, ref_l = oracle.attention(q, k, v, w.softmax_scale, w.causal, rows=rows)
+    got_o = o.float().cpu().numpy().astype(np.float64)
+    got_l = lse.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got_o, got_l = got_o[:, :, rows], got_l[:, :, rows]
+    assert np.isfinite(got_o).all() and np.isfinite(got_l).all()
+    to, tl = TOL[w.dtype]
+    do = np.abs(got_o - ref_o).max()
+    dl = np.abs(got_l - ref_l).max()
+    assert do <= to, f"{w.name}: max|dO| = {do:.3e} > {to}"
+    assert dl <= tl, f"{w.name}: max|dLSE| = {dl:.3e} > {tl}"
+    return o, lse, (q, k, v), do, dl
+
+
+# ------------------------------------------------------------ every element
+def test_tiny_config(cuda_dev):
+    compare(TINY, cuda_dev)
+
+
+EDGE = []
+for D in (64, 128, 256):
+    for nq, nk in ((1, 1), (17, 17), (127, 127), (129, 129), (255, 300), (300, 255), (513, 513),
+                   (1, 700), (700, 1)):
+        for causal in (False, True):
+            EDGE.append(Workload(f"edge D{D} {nq}x{nk} {'c' if causal else 'nc'}", 1, 2, 1, nq, nk,
+                                 D, "fp16", causal, seed=nq + nk + D))
+
+
+@pytest.mark.parametrize("w", EDGE, ids=lambda w: w.name)
+def test_ragged_shapes(cuda_dev, w):
+    compare(w, cuda_dev)
+
+
+MIXED = [
+    Workload("bf16 D128 GQA4 B2", 2, 8, 2, 384, 384, 128, "bf16", True, seed=11),
+    Workload("bf16 D64 MQA", 1, 4, 1, 640, 640, 64, "bf16", False, seed=12),
+    Workload("bf16 D256 GQA", 1, 4, 2, 520, 520, 256, "bf16", True, seed=13),
+    Workload("fp16 D128 peaky", 1, 2, 2, 1024, 1024, 128, "fp16", False, seed=14, q_mult=4.0),
+    Workload("fp16 D256 peaky causal", 1, 2, 1, 700, 700, 256, "fp16", True, seed=15, q_mult=4.0),
+    Workload("bf16 D128 outliers", 1, 2, 1, 1000, 1000, 128, "bf16", True, seed=16,
+             outlier_frac=0.01),
+    Workload("fp16 D64 many tiles", 3, 5, 5, 1100, 900, 64, "fp16", True, seed=17),
+]
+
+
+@pytest.mark.parametrize("w", MIXED, ids=lambda w: w.name)
+def test_mixed(cuda_dev, w):
+    compare(w, cuda_dev)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.5])
+def test_scale_values(cuda_dev, scale):
+    w = Workload("scale", 1, 2, 2, 300, 300, 128, "fp16", True, seed=3, scale=scale)
+    o, lse, (q, k, v), _, _ = compare(w, cuda_dev)
+    if scale == 0.0:  # uniform average over the visible prefix
+        n = torch.arange(1, 301, dtype=torch.float64)
+        np.testing.assert_allclose(lse.cpu().double().numpy(), np.log(n.numpy())[None, None].repeat(2, 1),
+                                   atol=1e-5)
+
+
+def test_deterministic_and_lse_optional(cuda_dev):
+    w = Workload("det", 1, 4, 2, 777, 777, 128, "bf16", True, seed=5)
+    (q, k, v), o1, l1 = run_cuda(w, cuda_dev)
+    qd, kd, vd = (x.to(cuda_dev) for x in (q, k, v))
+    o2, l2 = fa.fa_fwd(qd, kd, vd, scale=w.softmax_scale, causal=True)
+    o3, none = fa.fa_fwd(qd, kd, vd, scale=w.softmax_scale, causal=True, return_lse=False)
+    torch.cuda.synchronize()
+    assert none is None
+    assert torch.equal(o1, o2) and torch.equal(l1, l2) and torch.equal(o1, o3)
+
+
+def test_side_stream(cuda_dev):
+    w = Workload("stream", 1, 2, 2, 512, 512, 64, "fp16", False, seed=6)
+    q, k, v = (x.to(cuda_dev) for x in make_qkv(w))
+    ref, _ = fa.fa_fwd(q, k, v, causal=False)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o, _ = fa.fa_fwd(q, k, v, causal=False)
+    s.synchronize()
+    assert torch.equal(o, ref)
+
+
+# ------------------------------------------------------------ full-size workloads (sampled rows)
+def _full(w, n_rows, cuda_dev):
+    rows = sample_rows(w.Nq, n_rows, w.seed)
+    o, lse, (q, k, v), do, dl = compare(w, cuda_dev, rows=rows)
+    # properties at every row: O is a convex combination of V rows, LSE is finite
+    vmax = v.float().abs().amax(dim=(2, 3)).to(cuda_dev)
+    g = w.Hq // w.Hkv
+    bound = vmax.repeat_interleave(g, dim=1)[..., None, None]
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    assert bool((o.float().abs() <= bound * (1 + 1e-2) + 1e-2).all())
+    return do, dl
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("peaky", [False, True])
+def test_llama7b_layer(cuda_dev, causal, peaky):
+    _full(llama7b(causal, peaky), 64, cuda_dev)
+
+
+@pytest.mark.parametrize("n", [512, 2048, 4096, 8192])
+@pytest.mark.parametrize("causal", [False, True])
+def test_sequence_sweep(cuda_dev, n, causal):
+    _full(seq_sweep(n, causal), 48, cuda_dev)
+
+
+@pytest.mark.parametrize("hkv,d", [(8, 128), (1, 128), (8, 64), (8, 256)])
+def test_gqa_headdim(cuda_dev, hkv, d):
+    _full(gqa(hkv, d), 16, cuda_dev)
+
+
+def test_long_context_128k(cuda_dev):
+    _full(LONG, 256, cuda_dev)

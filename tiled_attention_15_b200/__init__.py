@@ -1,0 +1,127 @@
+"""Python binding of the B200 fused attention forward library (``libfa.so``).
+
+Argument marshalling only: every step of the attention forward pass runs in the
+CUDA kernels behind the C ABI declared in ``include/fa.h``.  PyTorch supplies
+device memory and the current stream.  There is no fallback: if the library is
+missing, importing the functions raises.
+
+    from tiled_attention_15_b200 import fa_fwd
+    o, lse = fa_fwd(q, k, v, causal=True)          # q,k,v: cuda fp16/bf16 [B,H,N,D]
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_FP16, FA_BF16 = 0, 1
+FA_OK = 0
+FA_ERR_DEVICE_TIMEOUT = 11
+
+# Every symbol include/fa.h declares (checked by the tests).
+EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_status_string", "fa_device_status",
+            "fa_fwd_num_tiles")
+
+
+class FaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: status {code} ({status_string(code)})")
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libfa.so (built by ``python -m tiled_attention_15_b200.csrc.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                           "(run python -m tiled_attention_15_b200.csrc.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fwd_args = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
+    lib.fa_fwd.argtypes = fwd_args + [i]
+    lib.fa_fwd.restype = i
+    for name in ("fa_fwd_fp16", "fa_fwd_bf16"):
+        getattr(lib, name).argtypes = fwd_args
+        getattr(lib, name).restype = i
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_device_status.argtypes = [i]
+    lib.fa_device_status.restype = i
+    lib.fa_fwd_num_tiles.argtypes = [i, i, i, i]
+    lib.fa_fwd_num_tiles.restype = ctypes.c_longlong
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().fa_status_string(int(code)).decode()
+
+
+def device_status(reset: bool = False) -> int:
+    """FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel gave up on a wait (synchronises the device)."""
+    return int(load_library().fa_device_status(1 if reset else 0))
+
+
+def num_tiles(B: int, Hq: int, Nq: int, D: int) -> int:
+    return int(load_library().fa_fwd_num_tiles(B, Hq, Nq, D))
+
+
+def fa_fwd_raw(q: int, k: int, v: int, o: int, lse: Optional[int], B: int, Hq: int, Hkv: int,
+               Nq: int, Nk: int, D: int, scale: float, causal: bool, stream: int,
+               dtype: int) -> int:
+    """The C entry point with plain integers for pointers; returns the status code."""
+    return int(load_library().fa_fwd(q, k, v, o, lse or None, B, Hq, Hkv, Nq, Nk, D,
+                                     ctypes.c_float(scale), 1 if causal else 0, stream or None,
+                                     dtype))
+
+
+def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False,
+           return_lse: bool = True, stream=None) -> Tuple[object, Optional[object]]:
+    """Fused attention forward on the current CUDA stream.
+
+    q: [B, Hq, Nq, D], k/v: [B, Hkv, Nk, D] contiguous CUDA tensors, fp16 or bf16.
+    o: optional output like q; lse: optional float32 [B, Hq, Nq] output.
+    scale defaults to 1/sqrt(D).  Returns (o, lse or None).
+    """
+    import torch
+
+    lib = load_library()
+    if q.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("q, k, v must be float16 or bfloat16")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("expected q [B,Hq,Nq,D] and k, v [B,Hkv,Nk,D]")
+    B, Hq, Nq, D = q.shape
+    Bk, Hkv, Nk, Dk = k.shape
+    if (Bk, Dk) != (B, D):
+        raise ValueError("batch and head_dim of q and k differ")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if o is None:
+        o = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    elif hasattr(stream, "cuda_stream"):
+        stream = stream.cuda_stream
+    dtype = FA_BF16 if q.dtype == torch.bfloat16 else FA_FP16
+    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                    lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, D,
+                    ctypes.c_float(scale), 1 if causal else 0, stream or None, dtype)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd")
+    return o, lse

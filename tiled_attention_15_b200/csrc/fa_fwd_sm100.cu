@@ -1,0 +1,783 @@
+// fa_fwd_sm100.cu -- fused, tiled attention forward pass (FlashAttention) for B200 / sm_100a.
+//
+// What is computed (mooersco.com article "昇腾CANN ops-transformer 仓的 FlashAttention
+// 算子", section "昇腾NPU上的分块策略", steps 1-5): for every query row block and
+// every key/value column block, S = Q K^T on the matrix unit, an online-softmax
+// update of the running row maximum m and row sum l on the vector unit, and
+// O += P V back on the matrix unit, with S and P kept on chip.  The B200 mapping:
+//
+//   * one persistent CTA per SM walks a list of work tiles; a work tile is
+//     NQ = 2 query tiles of 128 rows (NQ = 1 for head_dim 256) of one
+//     (batch, head);
+//   * warp 9 (one thread) streams Q once per tile and K_j / V_j blocks of 128
+//     keys through an NST-stage shared-memory ring with TMA (the page's double
+//     buffering, deeper);
+//   * warp 8 (one thread) issues tcgen05.mma: S_q = Q_q K_j^T into tensor memory
+//     (fp32), then O_q += P_q V_j with P read from tensor memory, where the
+//     softmax wrote it over S_q as 16-bit values;
+//   * warps 0-3 and 4-7 are two softmax warpgroups, one per query tile, one row
+//     per thread: row max, exp2 with the scale folded in, row sum, P back to
+//     tensor memory; the partial O in tensor memory is rescaled only when the
+//     row maximum grew by more than 2^8 since the last rescale (exact: any
+//     common stabiliser gives the same softmax), and 1/l is applied once, in
+//     the epilogue, which also writes the natural-log row LSE;
+//   * causal attention skips key blocks above the diagonal and masks only the
+//     blocks that straddle it (or the key tail);
+//   * with NQ = 2 the two query tiles ping-pong: the tensor core works on one
+//     tile's S or PV while the other tile's softmax runs.
+//
+// Tensor memory (512 columns x 128 lanes x 32 bit): S_0 at column 0, S_1 at
+// 128 (for NQ = 1 these are two S buffers of the single tile, used for
+// alternate key blocks), O_q at 256 + q*D.
+//
+// Every wait on an mbarrier is bounded (kWaitLimitNs); a wait that runs out
+// records FA_ERR_DEVICE_TIMEOUT in a device status word, makes the whole CTA
+// leave its loops, waits (bounded) for its own TMA loads in flight, frees its
+// tensor memory and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+__device__ unsigned int g_status = 0;
+
+constexpr int kBM = 128;  // query rows per query tile (MMA M)
+constexpr int kBN = 128;  // keys per key/value block (MMA N of S, K of PV)
+constexpr int kThreads = 384;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
+constexpr float kRescaleThreshold = 8.0f;         // log2 units: P <= 2^8 between rescales
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D, int NQ>
+struct Geometry {
+  static constexpr int DCH = D / 64;  // 128-byte (64-element) column chunks per row
+  static constexpr int Q_BYTES = kBM * D * 2;
+  static constexpr int KV_BYTES = kBN * D * 2;
+  static constexpr int CHUNK_Q = kBM * 128;   // one 64-column chunk of a Q tile
+  static constexpr int CHUNK_KV = kBN * 128;  // one 64-column chunk of a K/V block
+  static constexpr int NST = D == 64 ? 8 : (D == 128 ? 4 : 2);
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = NQ * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NST * KV_BYTES;
+  // mbarrier indices
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = 2 + NST,
+                       B_SFULL = 2 + 2 * NST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
+                       B_OEMPTY = B_OFULL + 2, B_PVDONE = B_OEMPTY + 2, NBAR = B_PVDONE + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (u32)
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(NQ == 2 ? (256 + 2 * D <= 512) : (256 + D <= 512), "tensor memory budget");
+};
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, Nq, Nk, group;
+  int causal;
+  float c;          // scale * log2(e)
+  int qt_per_head;  // work tiles per (batch, head)
+  int n_tiles;
+  int nkb;  // key blocks: ceil(Nk / kBN)
+};
+
+struct Tile {
+  int bh;     // b * Hq + hq
+  int row0;   // first query row of the work tile
+  int kvz;    // b * Hkv + kv head
+  int nblk[2];
+  int nb;
+};
+
+template <int NQ>
+__device__ __forceinline__ Tile get_tile(const FwdParams& p, int t) {
+  Tile T;
+  const int BH = p.B * p.Hq;
+  int qt;
+  if (p.causal) {  // heaviest (last) query tiles first
+    qt = p.qt_per_head - 1 - t / BH;
+    T.bh = t % BH;
+  } else {  // tiles of one head adjacent: K/V of a head stay hot in L2
+    T.bh = t / p.qt_per_head;
+    qt = t % p.qt_per_head;
+  }
+  T.row0 = qt * NQ * kBM;
+  const int b = T.bh / p.Hq, hq = T.bh % p.Hq;
+  T.kvz = b * p.Hkv + hq / p.group;
+  T.nb = 0;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int rf = T.row0 + q * kBM;
+    int n = 0;
+    if (q < NQ && rf < p.Nq) {
+      n = p.nkb;
+      if (p.causal) {
+        const int rl = min(rf + kBM - 1, p.Nq - 1);
+        n = min(p.nkb, rl / kBN + 1);
+      }
+    }
+    T.nblk[q] = n;
+    T.nb = max(T.nb, n);
+  }
+  return T;
+}
+
+// Work tiles of this CTA, in a zig-zag over rounds of gridDim.x tiles so that
+// heavy-first causal lists spread evenly.
+struct TileIter {
+  int r, cta, G, n;
+  __device__ TileIter(int n_tiles) : r(-1), cta(blockIdx.x), G(gridDim.x), n(n_tiles) {}
+  __device__ bool next(int& t) {
+    while (true) {
+      ++r;
+      if (r * G >= n) return false;
+      const int pos = (r & 1) ? (G - 1 - cta) : cta;
+      t = r * G + pos;
+      if (t < n) return true;
+    }
+  }
+};
+
+struct Ctx {
+  uint32_t sbase;  // 1024-aligned shared-memory base (shared address space)
+  uint32_t tmem;   // tensor-memory base address
+  volatile uint32_t* abort_flag;
+  __device__ uint32_t bar(int i, int off_bar) const { return sbase + off_bar + 8u * i; }
+};
+
+// Bounded wait on an mbarrier phase.  Returns false (and makes every other
+// wait of the CTA return false) when the time limit is reached.
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity,
+                                      volatile uint32_t* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1u;
+      atomicCAS(&g_status, 0u, static_cast<unsigned>(FA_ERR_DEVICE_TIMEOUT));
+      return false;
+    }
+  }
+}
+
+// Wait that ignores the abort flag, with its own short limit (used only to
+// drain this CTA's own TMA loads on the abort path).
+__device__ __noinline__ void drain_bar(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > 100000000ull) return;
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b, bool bf16) {
+  if (bf16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// ---------------------------------------------------------------- TMA producer
+template <int D, int NQ>
+__device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, const CUtensorMap* tq,
+                                          const CUtensorMap* tk, const CUtensorMap* tv) {
+  using G = Geometry<D, NQ>;
+  prefetch_tmap(tq);
+  prefetch_tmap(tk);
+  prefetch_tmap(tv);
+  const uint64_t pol_kv = policy_evict_last();
+  const uint64_t pol_q = policy_evict_first();
+  uint32_t kv_it = 0, qe_phase = 0, q_issued = 0;
+  bool ok = true;
+  TileIter it(p.n_tiles);
+  int t;
+  while (ok && it.next(t)) {
+    const Tile T = get_tile<NQ>(p, t);
+    if (q_issued) {
+      if (!wait_bar(cx.bar(G::B_QEMPTY, G::OFF_BAR), qe_phase, cx.abort_flag)) { ok = false; break; }
+      qe_phase ^= 1u;
+    }
+    mbar_arrive_expect_tx(cx.bar(G::B_QFULL, G::OFF_BAR), NQ * G::Q_BYTES);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+      for (int c = 0; c < G::DCH; ++c)
+        tma_load_3d(cx.sbase + G::OFF_Q + q * G::Q_BYTES + c * G::CHUNK_Q, tq,
+                    cx.bar(G::B_QFULL, G::OFF_BAR), c * 64, T.row0 + q * kBM, T.bh, pol_q);
+    ++q_issued;
+    // K/V block order matches the MMA warp's consumption order:
+    //   NQ = 2: K0, V0, K1, V1, ...      NQ = 1: K0, K1, V0, K2, V1, ...
+    for (int s = 0; s < 2 * T.nb && ok; ++s) {
+      int j;
+      bool is_k;
+      if (s == 0) { j = 0; is_k = true; }
+      else if (NQ == 2) { j = s / 2; is_k = (s & 1) == 0; }   // s=1:V0 s=2:K1 s=3:V1 ...
+      else {                                                    // s=1:K1 s=2:V0 s=3:K2 ...
+        if (s == 2 * T.nb - 1) { j = T.nb - 1; is_k = false; }
+        else { is_k = (s & 1) == 1; j = is_k ? (s + 1) / 2 : s / 2 - 1; }
+      }
+      const int st = kv_it % G::NST;
+      if (kv_it >= (uint32_t)G::NST) {
+        if (!wait_bar(cx.bar(G::B_KVEMPTY + st, G::OFF_BAR), ((kv_it / G::NST) - 1) & 1u,
+                      cx.abort_flag)) { ok = false; break; }
+      }
+      mbar_arrive_expect_tx(cx.bar(G::B_KVFULL + st, G::OFF_BAR), G::KV_BYTES);
+#pragma unroll
+      for (int c = 0; c < G::DCH; ++c)
+        tma_load_3d(cx.sbase + G::OFF_KV + st * G::KV_BYTES + c * G::CHUNK_KV, is_k ? tk : tv,
+                    cx.bar(G::B_KVFULL + st, G::OFF_BAR), c * 64, j * kBN, T.kvz, pol_kv);
+      ++kv_it;
+    }
+  }
+  if (!ok) {  // abort: let this CTA's own loads land before the CTA exits
+    for (uint32_t n = (kv_it > (uint32_t)G::NST ? kv_it - G::NST : 0); n < kv_it; ++n)
+      drain_bar(cx.bar(G::B_KVFULL + n % G::NST, G::OFF_BAR), (n / G::NST) & 1u);
+    if (q_issued) drain_bar(cx.bar(G::B_QFULL, G::OFF_BAR), (q_issued - 1) & 1u);
+  }
+}
+
+// ---------------------------------------------------------------- MMA issuer
+template <int D, int NQ, bool BF16>
+__device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
+  using G = Geometry<D, NQ>;
+  constexpr uint32_t kIdS = idesc_f16(kBM, kBN, BF16, false);  // Q, K both K-major
+  constexpr uint32_t kIdPV = idesc_f16(kBM, D, BF16, true);    // V is N(=D)-major
+  uint32_t kv_it = 0, q_phase = 0, p_phase[2] = {0u, 0u}, oe_phase[2] = {0u, 0u};
+  bool o_pending[2] = {false, false};
+  const uint32_t tm = cx.tmem;
+  auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
+
+  auto consume = [&](int& st) -> bool {
+    st = kv_it % G::NST;
+    const bool r = wait_bar(B(G::B_KVFULL + st), (kv_it / G::NST) & 1u, cx.abort_flag);
+    ++kv_it;
+    tc_fence_after();
+    return r;
+  };
+  auto issue_S = [&](int qt, int sbuf, int st) {
+    const uint32_t qa = cx.sbase + G::OFF_Q + qt * G::Q_BYTES;
+    const uint32_t ka = cx.sbase + G::OFF_KV + st * G::KV_BYTES;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t a = sdesc_sw128(qa + (kk >> 2) * G::CHUNK_Q + (kk & 3) * 32, 16, 1024);
+      const uint64_t b = sdesc_sw128(ka + (kk >> 2) * G::CHUNK_KV + (kk & 3) * 32, 16, 1024);
+      mma_ss(tm + sbuf * 128, a, b, kIdS, kk > 0 ? 1u : 0u);
+    }
+  };
+  auto issue_PV = [&](int ot, int sbuf, int st, bool acc) {
+    const uint32_t va = cx.sbase + G::OFF_KV + st * G::KV_BYTES;
+#pragma unroll
+    for (int kk = 0; kk < kBN / 16; ++kk) {
+      const uint64_t b = sdesc_sw128(va + kk * 2048, G::CHUNK_KV, 1024);
+      mma_ts(tm + 256 + ot * D, tm + sbuf * 128 + kk * 8, b, kIdPV, (acc || kk > 0) ? 1u : 0u);
+    }
+  };
+  // Before the first PV of a tile into O_q: the previous tile's epilogue must
+  // have read O_q out of tensor memory.
+  auto o_ready = [&](int q) -> bool {
+    if (!o_pending[q]) return true;
+    if (!wait_bar(B(G::B_OEMPTY + q), oe_phase[q], cx.abort_flag)) return false;
+    oe_phase[q] ^= 1u;
+    o_pending[q] = false;
+    tc_fence_after();
+    return true;
+  };
+  auto p_ready = [&](int q) -> bool {
+    if (!wait_bar(B(G::B_PFULL + q), p_phase[q], cx.abort_flag)) return false;
+    p_phase[q] ^= 1u;
+    tc_fence_after();
+    return true;
+  };
+
+  TileIter it(p.n_tiles);
+  int t;
+  while (it.next(t)) {
+    const Tile T = get_tile<NQ>(p, t);
+    if (!wait_bar(B(G::B_QFULL), q_phase, cx.abort_flag)) return;
+    q_phase ^= 1u;
+    tc_fence_after();
+    const int nb = T.nb;
+    int kst;
+    if (!consume(kst)) return;
+    if (NQ == 2) {
+      // stream: S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
+      if (T.nblk[0] > 0) { issue_S(0, 0, kst); mma_commit(B(G::B_SFULL + 0)); }
+      if (T.nblk[1] > 0) { issue_S(1, 1, kst); mma_commit(B(G::B_SFULL + 1)); }
+      mma_commit(B(G::B_KVEMPTY + kst));
+      if (nb == 1) mma_commit(B(G::B_QEMPTY));
+      for (int j = 0; j < nb; ++j) {
+        int vst;
+        if (!consume(vst)) return;
+        if (j < T.nblk[0]) {
+          if (j == 0 && !o_ready(0)) return;
+          if (!p_ready(0)) return;
+          issue_PV(0, 0, vst, j > 0);
+          if (j == T.nblk[0] - 1) { mma_commit(B(G::B_OFULL + 0)); o_pending[0] = true; }
+        }
+        int kst2 = -1;
+        if (j + 1 < nb) {
+          if (!consume(kst2)) return;
+          if (j + 1 < T.nblk[0]) { issue_S(0, 0, kst2); mma_commit(B(G::B_SFULL + 0)); }
+        }
+        if (j < T.nblk[1]) {
+          if (j == 0 && !o_ready(1)) return;
+          if (!p_ready(1)) return;
+          issue_PV(1, 1, vst, j > 0);
+          if (j == T.nblk[1] - 1) { mma_commit(B(G::B_OFULL + 1)); o_pending[1] = true; }
+        }
+        mma_commit(B(G::B_KVEMPTY + vst));
+        if (kst2 >= 0) {
+          if (j + 1 < T.nblk[1]) { issue_S(1, 1, kst2); mma_commit(B(G::B_SFULL + 1)); }
+          mma_commit(B(G::B_KVEMPTY + kst2));
+          if (j + 1 == nb - 1) mma_commit(B(G::B_QEMPTY));
+        }
+      }
+    } else {
+      // one query tile, two S buffers: S(0) | S(j+1) PV(j) | ...
+      issue_S(0, 0, kst);
+      mma_commit(B(G::B_SFULL + 0));
+      mma_commit(B(G::B_KVEMPTY + kst));
+      if (nb == 1) mma_commit(B(G::B_QEMPTY));
+      for (int j = 0; j < nb; ++j) {
+        if (j + 1 < nb) {
+          if (!consume(kst)) return;
+          issue_S(0, (j + 1) & 1, kst);
+          mma_commit(B(G::B_SFULL + ((j + 1) & 1)));
+          mma_commit(B(G::B_KVEMPTY + kst));
+          if (j + 1 == nb - 1) mma_commit(B(G::B_QEMPTY));
+        }
+        int vst;
+        if (!consume(vst)) return;
+        if (j == 0 && !o_ready(0)) return;
+        if (!p_ready(0)) return;
+        issue_PV(0, j & 1, vst, j > 0);
+        mma_commit(B(G::B_PVDONE));
+        mma_commit(B(G::B_KVEMPTY + vst));
+        if (j == nb - 1) { mma_commit(B(G::B_OFULL + 0)); o_pending[0] = true; }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- softmax + epilogue
+template <int D, int NQ, bool BF16>
+__device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, int wg, int sub,
+                                             int lane) {
+  using G = Geometry<D, NQ>;
+  const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+  const uint32_t tm = cx.tmem + lane_off;
+  auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
+  const float c = p.c;
+  uint32_t s_phase[2] = {0u, 0u}, of_phase = 0u, pv_seen = 0u;
+  const int q = (NQ == 2) ? wg : 0;
+
+  TileIter it(p.n_tiles);
+  int t;
+  while (it.next(t)) {
+    const Tile T = get_tile<NQ>(p, t);
+    const int nblk = T.nblk[q];
+    if (nblk == 0) continue;
+    const int rfirst = T.row0 + q * kBM;
+    const int row = rfirst + sub * 32 + lane;
+    float m_used = -INFINITY, l = 0.f, l_r = 0.f;  // l: exact sum (LSE); l_r: rounded-P sum
+    for (int j = 0; j < nblk; ++j) {
+      const int sb = (NQ == 2) ? q : (j & 1);
+      bool ok = wait_bar(B(G::B_SFULL + sb), s_phase[sb], cx.abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      s_phase[sb] ^= 1u;
+      tc_fence_after();
+      uint32_t sr[kBN];
+      tmem_ld_x128(tm + sb * 128, sr);
+
+      const int kbase = j * kBN;
+      const bool masked = (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst);
+      float m_blk;
+      if (masked) {
+        int lim = p.Nk - kbase;
+        if (p.causal) lim = min(lim, row - kbase + 1);
+        m_blk = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) {
+          const float tv = (i < lim) ? __uint_as_float(sr[i]) * c : -INFINITY;
+          sr[i] = __float_as_uint(tv);
+          m_blk = fmaxf(m_blk, tv);
+        }
+      } else {
+        float mx = __uint_as_float(sr[0]);
+        if (c >= 0.f) {
+#pragma unroll
+          for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+        } else {
+#pragma unroll
+          for (int i = 1; i < kBN; ++i) mx = fminf(mx, __uint_as_float(sr[i]));
+        }
+        m_blk = mx * c;
+      }
+      // stabiliser update (log2 units); rescale only when the max grew by > 2^8
+      float alpha = 1.f;
+      bool need = false;
+      if (j == 0) {
+        m_used = m_blk;
+      } else if (m_blk > m_used + kRescaleThreshold) {
+        alpha = ex2(m_used - m_blk);
+        m_used = m_blk;
+        need = true;
+      }
+      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+      const float neg_m = -m_sub;
+      float lsum = 0.f, lsum_r = 0.f;
+      uint32_t pk[kBN / 2];
+      // bf16 only: also sum the rounded P that the PV product actually uses, and
+      // normalise O by that sum -- the weights then sum to one exactly, which
+      // removes the bf16 rounding error of the dominant weight(s) from O.
+#pragma unroll
+      for (int i = 0; i < kBN / 2; ++i) {
+        float p0, p1;
+        if (masked) {
+          p0 = ex2(__uint_as_float(sr[2 * i]) + neg_m);
+          p1 = ex2(__uint_as_float(sr[2 * i + 1]) + neg_m);
+        } else {
+          p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), c, neg_m));
+          p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), c, neg_m));
+        }
+        lsum += p0 + p1;
+        pk[i] = pack2(p0, p1, BF16);
+        if (BF16) lsum_r += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+      }
+      l = l * alpha + lsum;
+      if (BF16) l_r = l_r * alpha + lsum_r;
+      tmem_st_x64(tm + sb * 128, pk);
+      if (__any_sync(0xffffffffu, need)) {
+        if (NQ == 1) {  // PV(j-1) must have finished accumulating into O
+          ok = wait_bar(B(G::B_PVDONE), (pv_seen + j - 1) & 1u, cx.abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) return;
+          tc_fence_after();
+        }
+        const float a = need ? alpha : 1.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t orr[32];
+          tmem_ld_x32(tm + 256 + q * D + c0, orr);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) orr[x] = __float_as_uint(__uint_as_float(orr[x]) * a);
+          tmem_st_x32(tm + 256 + q * D + c0, orr);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_PFULL + q));
+    }
+    pv_seen += nblk;
+
+    // epilogue: O = O_acc / l, rounded to the input dtype; LSE in natural log
+    bool ok = wait_bar(B(G::B_OFULL + q), of_phase, cx.abort_flag);
+    if (!__all_sync(0xffffffffu, ok)) return;
+    of_phase ^= 1u;
+    tc_fence_after();
+    const float inv_l = 1.f / (BF16 ? l_r : l);
+    const bool live = row < p.Nq;
+    uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
+                     (static_cast<size_t>(T.bh) * p.Nq + (live ? row : 0)) * D;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t orr[32];
+      tmem_ld_x32(tm + 256 + q * D + c0, orr);
+      uint32_t w[16];
+#pragma unroll
+      for (int x = 0; x < 16; ++x)
+        w[x] = pack2(__uint_as_float(orr[2 * x]) * inv_l, __uint_as_float(orr[2 * x + 1]) * inv_l,
+                     BF16);
+      if (live) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+      }
+    }
+    if (p.lse != nullptr && live) {
+      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+      p.lse[static_cast<size_t>(T.bh) * p.Nq + row] = (m_sub + log2f(l)) * kLn2;
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(B(G::B_OEMPTY + q));
+  }
+}
+
+template <int D, int NQ, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using G = Geometry<D, NQ>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(gbase + G::OFF_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  Ctx cx;
+  cx.sbase = sbase;
+  cx.abort_flag = misc + 1;
+  if (threadIdx.x == 0) {
+    auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
+    mbar_init(B(G::B_QFULL), 1);
+    mbar_init(B(G::B_QEMPTY), 1);
+    for (int s = 0; s < G::NST; ++s) {
+      mbar_init(B(G::B_KVFULL + s), 1);
+      mbar_init(B(G::B_KVEMPTY + s), 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(B(G::B_SFULL + q), 1);
+      mbar_init(B(G::B_PFULL + q), 4);
+      mbar_init(B(G::B_OFULL + q), 1);
+      mbar_init(B(G::B_OEMPTY + q), 4);
+    }
+    mbar_init(B(G::B_PVDONE), 1);
+    misc[1] = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(misc), G::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cx.tmem = misc[0];
+
+  if (warp < 8) {
+    if (NQ == 2 || warp < 4) role_softmax<D, NQ, BF16>(cx, p, warp >> 2, warp & 3, lane);
+  } else if (warp == 8) {
+    if (lane == 0) role_mma<D, NQ, BF16>(cx, p);
+  } else if (warp == 9) {
+    if (lane == 0) role_load<D, NQ>(cx, p, &tm_q, &tm_k, &tm_v);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 8) {
+    if (*cx.abort_flag) {  // abort path: give issued MMAs time to retire before freeing TMEM
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 2000000ull) {
+      }
+    }
+    tmem_dealloc(cx.tmem, G::TMEM_COLS);
+  }
+}
+
+}  // namespace fa
+
+// ============================================================================ host side
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+  std::once_flag once;
+  int sms = 0;
+  bool sm100 = false;
+};
+DeviceState g_dev[kMaxDevices];
+
+// 3-D map over a [Z][rows][D] 16-bit tensor: box = 64 columns x box_rows rows x 1,
+// 128-byte swizzle (the layout the tcgen05 shared-memory descriptors describe).
+bool make_map(CUtensorMap* m, const void* ptr, int D, long long rows, long long Z, int box_rows,
+              bool bf16) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)Z};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  const cuuint32_t es[3] = {1u, 1u, 1u};
+  const CUresult r =
+      enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+          const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int nq_for(int D) { return D == 256 ? 1 : 2; }
+
+template <int D, int NQ, bool BF16>
+int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream, int dev) {
+  using G = fa::Geometry<D, NQ>;
+  static bool attr_done[kMaxDevices] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!attr_done[dev]) {
+      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, NQ, BF16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               G::SMEM_BYTES) != cudaSuccess)
+        return FA_ERR_LAUNCH;
+      attr_done[dev] = true;
+    }
+  }
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, Nq, (long long)B * Hq, fa::kBM, BF16) ||
+      !make_map(&tk, k, D, Nk, (long long)B * Hkv, fa::kBN, BF16) ||
+      !make_map(&tv, v, D, Nk, (long long)B * Hkv, fa::kBN, BF16))
+    return FA_ERR_DRIVER;
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.c = scale * 1.4426950408889634f;
+  p.qt_per_head = (Nq + NQ * fa::kBM - 1) / (NQ * fa::kBM);
+  p.n_tiles = B * Hq * p.qt_per_head;
+  p.nkb = (Nk + fa::kBN - 1) / fa::kBN;
+  const int grid = p.n_tiles < g_dev[dev].sms ? p.n_tiles : g_dev[dev].sms;
+  fa::fa_fwd_kernel<D, NQ, BF16><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL_POINTER: return "null pointer among q, k, v, o";
+    case FA_ERR_MISALIGNED: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
+    case FA_ERR_BAD_SHAPE: return "B, Hq, Hkv, Nq, Nk must be >= 1 and sizes must fit";
+    case FA_ERR_BAD_GROUPING: return "Hq must be a multiple of Hkv";
+    case FA_ERR_UNSUPPORTED_HEAD_DIM: return "head_dim must be 64, 128 or 256";
+    case FA_ERR_BAD_SCALE: return "scale must be finite";
+    case FA_ERR_BAD_DTYPE: return "dtype must be FA_FP16 or FA_BF16";
+    case FA_ERR_NO_DEVICE: return "no current CUDA device of compute capability 10.x (sm_100)";
+    case FA_ERR_LAUNCH: return "kernel launch failed";
+    case FA_ERR_DRIVER: return "tensor-map encoding failed in the CUDA driver";
+    case FA_ERR_DEVICE_TIMEOUT: return "a kernel wait reached its time limit";
+    case FA_ERR_OVERLAP: return "o or lse overlaps q, k or v";
+    default: return "unknown status";
+  }
+}
+
+long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D) {
+  if (B < 1 || Hq < 1 || Nq < 1 || (D != 64 && D != 128 && D != 256)) return 0;
+  const long long rows = (long long)nq_for(D) * fa::kBM;
+  return (long long)B * Hq * ((Nq + rows - 1) / rows);
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype) {
+  // ---- argument checks: host only, before any CUDA call
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
+  if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_BAD_SHAPE;
+  if (Hq % Hkv != 0) return FA_ERR_BAD_GROUPING;
+  const long long qo_elems = (long long)B * Hq * Nq * D, kv_elems = (long long)B * Hkv * Nk * D;
+  // work-tile count, row indices and TMA coordinates are 32-bit
+  if ((long long)B * Hq * Nq >= (1ll << 31) || (long long)B * Hkv * Nk >= (1ll << 31))
+    return FA_ERR_BAD_SHAPE;
+  if (!std::isfinite(scale)) return FA_ERR_BAD_SCALE;
+  if (!q || !k || !v || !o) return FA_ERR_NULL_POINTER;
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o) & 15u) return FA_ERR_MISALIGNED;
+  if (lse && ((uintptr_t)lse & 3u)) return FA_ERR_MISALIGNED;
+  const size_t qo_b = (size_t)qo_elems * 2, kv_b = (size_t)kv_elems * 2;
+  if (overlaps(o, qo_b, q, qo_b) || overlaps(o, qo_b, k, kv_b) || overlaps(o, qo_b, v, kv_b))
+    return FA_ERR_OVERLAP;
+  if (lse) {
+    const size_t lb = (size_t)B * Hq * Nq * 4;
+    if (overlaps(lse, lb, q, qo_b) || overlaps(lse, lb, k, kv_b) || overlaps(lse, lb, v, kv_b) ||
+        overlaps(lse, lb, o, qo_b))
+      return FA_ERR_OVERLAP;
+  }
+  // ---- device
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_NO_DEVICE;
+  DeviceState& ds = g_dev[dev];
+  std::call_once(ds.once, [&] {
+    int major = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    ds.sm100 = (major == 10);
+    ds.sms = sms;
+  });
+  if (!ds.sm100 || ds.sms < 1) return FA_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = dtype == FA_BF16;
+  switch (D) {
+    case 64:
+      return bf ? launch<64, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev)
+                : launch<64, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev);
+    case 128:
+      return bf ? launch<128, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev)
+                : launch<128, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev);
+    default:
+      return bf ? launch<256, 1, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev)
+                : launch<256, 1, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev);
+  }
+}
+
+int fa_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream) {
+  return fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, FA_FP16);
+}
+
+int fa_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream) {
+  return fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, FA_BF16);
+}
+
+int fa_device_status(int reset) {
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(v)) != cudaSuccess) return -1;
+  if (reset) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(fa::g_status, &z, sizeof(z)) != cudaSuccess) return -1;
+  }
+  return static_cast<int>(v);
+}
+
+}  // extern "C"
