@@ -104,6 +104,15 @@ const char *fa_status_string(int status);
  */
 int fa_device_status(int reset);
 
+/*
+ * Diagnostic companion of fa_device_status: where the first timed-out wait
+ * happened since the last reset, packed as
+ *   CTA index << 48 | warp << 40 | shared-memory address of the mbarrier << 8 | phase parity
+ * (0 if none).  Synchronises the device.  Returns FA_OK, FA_ERR_NULL_POINTER or
+ * FA_ERR_NO_DEVICE.
+ */
+int fa_device_timeout_site(unsigned long long *site);
+
 /* Number of work tiles (CTAs' units of work) one fa_fwd call would schedule;
  * 0 for invalid arguments.  Host only; used to count launches and to size tests. */
 long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D);

@@ -24,7 +24,7 @@ FA_ERR_DEVICE_TIMEOUT = 11
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_status_string", "fa_device_status",
-            "fa_fwd_num_tiles")
+            "fa_device_timeout_site", "fa_fwd_num_tiles")
 
 
 class FaError(RuntimeError):
@@ -56,6 +56,8 @@ def load_library() -> ctypes.CDLL:
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_device_status.argtypes = [i]
     lib.fa_device_status.restype = i
+    lib.fa_device_timeout_site.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.fa_device_timeout_site.restype = i
     lib.fa_fwd_num_tiles.argtypes = [i, i, i, i]
     lib.fa_fwd_num_tiles.restype = ctypes.c_longlong
     _lib = lib
@@ -69,6 +71,18 @@ def status_string(code: int) -> str:
 def device_status(reset: bool = False) -> int:
     """FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel gave up on a wait (synchronises the device)."""
     return int(load_library().fa_device_status(1 if reset else 0))
+
+
+def timeout_site():
+    """(cta, warp, mbarrier shared address, parity) of the first timed-out wait, or None."""
+    v = ctypes.c_ulonglong(0)
+    rc = load_library().fa_device_timeout_site(ctypes.byref(v))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_device_timeout_site")
+    x = v.value
+    if x == 0:
+        return None
+    return (x >> 48, (x >> 40) & 0xFF, (x >> 8) & 0xFFFFF, x & 1)
 
 
 def num_tiles(B: int, Hq: int, Nq: int, D: int) -> int:

@@ -50,6 +50,8 @@
 namespace fa {
 
 __device__ unsigned int g_status = 0;
+// Where the first timed-out wait was: CTA << 48 | warp << 40 | barrier shared address << 8 | parity.
+__device__ unsigned long long g_timeout_site = 0;
 
 constexpr int kBM = 128;  // query rows per query tile (MMA M)
 constexpr int kBN = 128;  // keys per key/value block (MMA N of S, K of PV)
@@ -168,7 +170,10 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity,
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1u;
-      atomicCAS(&g_status, 0u, static_cast<unsigned>(FA_ERR_DEVICE_TIMEOUT));
+      if (atomicCAS(&g_status, 0u, static_cast<unsigned>(FA_ERR_DEVICE_TIMEOUT)) == 0u)
+        g_timeout_site = (static_cast<unsigned long long>(blockIdx.x) << 48) |
+                         (static_cast<unsigned long long>(threadIdx.x >> 5) << 40) |
+                         (static_cast<unsigned long long>(bar & 0xFFFFFu) << 8) | parity;
       return false;
     }
   }
@@ -775,9 +780,20 @@ int fa_device_status(int reset) {
   if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(v)) != cudaSuccess) return -1;
   if (reset) {
     const unsigned int z = 0;
-    if (cudaMemcpyToSymbol(fa::g_status, &z, sizeof(z)) != cudaSuccess) return -1;
+    const unsigned long long zz = 0;
+    if (cudaMemcpyToSymbol(fa::g_status, &z, sizeof(z)) != cudaSuccess ||
+        cudaMemcpyToSymbol(fa::g_timeout_site, &zz, sizeof(zz)) != cudaSuccess)
+      return -1;
   }
   return static_cast<int>(v);
+}
+
+int fa_device_timeout_site(unsigned long long* site) {
+  if (!site) return FA_ERR_NULL_POINTER;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_NO_DEVICE;
+  if (cudaMemcpyFromSymbol(site, fa::g_timeout_site, sizeof(*site)) != cudaSuccess)
+    return FA_ERR_NO_DEVICE;
+  return FA_OK;
 }
 
 }  // extern "C"
