@@ -24,7 +24,7 @@ FA_ERR_DEVICE_TIMEOUT = 11
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_status_string", "fa_device_status",
-            "fa_device_timeout_site", "fa_fwd_num_tiles")
+            "fa_device_timeout_site", "fa_debug_exp2_fma", "fa_fwd_num_tiles")
 
 
 class FaError(RuntimeError):
@@ -58,6 +58,8 @@ def load_library() -> ctypes.CDLL:
     lib.fa_device_status.restype = i
     lib.fa_device_timeout_site.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
     lib.fa_device_timeout_site.restype = i
+    lib.fa_debug_exp2_fma.argtypes = [vp, vp, i, vp]
+    lib.fa_debug_exp2_fma.restype = i
     lib.fa_fwd_num_tiles.argtypes = [i, i, i, i]
     lib.fa_fwd_num_tiles.restype = ctypes.c_longlong
     _lib = lib
@@ -83,6 +85,18 @@ def timeout_site():
     if x == 0:
         return None
     return (x >> 48, (x >> 40) & 0xFF, (x >> 8) & 0xFFFFF, x & 1)
+
+
+def exp2_fma(x):
+    """2^x by the softmax's FMA-pipe approximation (diagnostics); x: float32 CUDA tensor."""
+    import torch
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    rc = load_library().fa_debug_exp2_fma(x.data_ptr(), y.data_ptr(), x.numel(),
+                                          torch.cuda.current_stream(x.device).cuda_stream or None)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_debug_exp2_fma")
+    return y
 
 
 def num_tiles(B: int, Hq: int, Nq: int, D: int) -> int:

@@ -159,7 +159,7 @@ struct Ctx {
 
 // Bounded wait on an mbarrier phase.  Returns false (and makes every other
 // wait of the CTA return false) when the time limit is reached.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity,
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity,
                                       volatile uint32_t* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -181,7 +181,7 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity,
 
 // Wait that ignores the abort flag, with its own short limit (used only to
 // drain this CTA's own TMA loads on the abort path).
-__device__ __noinline__ void drain_bar(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity))
     if (globaltimer_ns() - t0 > 100000000ull) return;
@@ -369,7 +369,11 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
         int vst;
         if (!consume(vst)) return;
         if (j == 0 && !o_ready(0)) return;
-        if (!p_ready(0)) return;
+        // P(j) lives in S buffer j & 1, and each buffer has its own p_full barrier:
+        // S(j+1) is already issued here, so a fast softmax warp may finish block j+1
+        // before a slow one finishes block j -- one barrier per buffer keeps their
+        // arrivals apart (a warp can never get two blocks ahead: S(j+2) follows PV(j)).
+        if (!p_ready(j & 1)) return;
         issue_PV(0, j & 1, vst, j > 0);
         mma_commit(B(G::B_PVDONE));
         mma_commit(B(G::B_KVEMPTY + vst));
@@ -377,6 +381,41 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
       }
     }
   }
+}
+
+// Exps of these pairs (bit k: pair index % 8 == k) run on the FMA pipe; the
+// rest on MUFU.  MUFU throughput (16 ex2 / clock / SM) alone would equal the
+// tensor-core time of S and PV at head_dim 128.
+constexpr uint32_t kEmuPairs = 0x52u;  // pairs 1, 4, 6 of every 8: 3/8 of the exps
+
+// Row max / min of 128 scores: four independent chains of 3-input max.
+__device__ __forceinline__ float row_max(const uint32_t* v) {
+  float a0 = __uint_as_float(v[0]), a1 = __uint_as_float(v[1]), a2 = __uint_as_float(v[2]),
+        a3 = __uint_as_float(v[3]);
+#pragma unroll
+  for (int i = 4; i < kBN; i += 8) {
+    a0 = fmax3(a0, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+    a1 = fmax3(a1, __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+    a2 = fmax3(a2, __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
+    a3 = fmax3(a3, __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
+  }
+  return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+}
+__device__ __forceinline__ float row_min(const uint32_t* v) {
+  float a0 = __uint_as_float(v[0]), a1 = __uint_as_float(v[1]), a2 = __uint_as_float(v[2]),
+        a3 = __uint_as_float(v[3]);
+#pragma unroll
+  for (int i = 4; i < kBN; i += 8) {
+    a0 = fmin3(a0, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+    a1 = fmin3(a1, __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+    a2 = fmin3(a2, __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
+    a3 = fmin3(a3, __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
+  }
+  return fminf(fminf(a0, a1), fminf(a2, a3));
+}
+// The two bf16 halves of a packed word, widened (exactly) to fp32.
+__device__ __forceinline__ F2 unpack_bf16x2(uint32_t w) {
+  return F2{__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)};
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
@@ -412,26 +451,15 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
       const int kbase = j * kBN;
       const bool masked = (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst);
       float m_blk;
-      if (masked) {
+      if (masked) {  // scaled scores, -inf where the key is causal-future or past Nk
         int lim = p.Nk - kbase;
         if (p.causal) lim = min(lim, row - kbase + 1);
-        m_blk = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) {
-          const float tv = (i < lim) ? __uint_as_float(sr[i]) * c : -INFINITY;
-          sr[i] = __float_as_uint(tv);
-          m_blk = fmaxf(m_blk, tv);
-        }
-      } else {
-        float mx = __uint_as_float(sr[0]);
-        if (c >= 0.f) {
-#pragma unroll
-          for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
-        } else {
-#pragma unroll
-          for (int i = 1; i < kBN; ++i) mx = fminf(mx, __uint_as_float(sr[i]));
-        }
-        m_blk = mx * c;
+        for (int i = 0; i < kBN; ++i)
+          sr[i] = __float_as_uint((i < lim) ? __uint_as_float(sr[i]) * c : -INFINITY);
+        m_blk = row_max(sr);
+      } else {  // max of raw scores; the scale (of either sign) is applied to the max
+        m_blk = (c >= 0.f ? row_max(sr) : row_min(sr)) * c;
       }
       // stabiliser update (log2 units); rescale only when the max grew by > 2^8
       float alpha = 1.f;
@@ -443,30 +471,42 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
         m_used = m_blk;
         need = true;
       }
-      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-      const float neg_m = -m_sub;
-      float lsum = 0.f, lsum_r = 0.f;
-      uint32_t pk[kBN / 2];
+      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
       // bf16 only: also sum the rounded P that the PV product actually uses, and
       // normalise O by that sum -- the weights then sum to one exactly, which
       // removes the bf16 rounding error of the dominant weight(s) from O.
+      // P goes back to tensor memory (over S) in groups of 16 packed pairs as soon
+      // as a group is ready, which keeps the live register set small.
+      F2 acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+      F2 accr[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-      for (int i = 0; i < kBN / 2; ++i) {
-        float p0, p1;
-        if (masked) {
-          p0 = ex2(__uint_as_float(sr[2 * i]) + neg_m);
-          p1 = ex2(__uint_as_float(sr[2 * i + 1]) + neg_m);
-        } else {
-          p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), c, neg_m));
-          p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), c, neg_m));
+      for (int g = 0; g < kBN / 32; ++g) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int i = g * 16 + u;
+          const F2 sv = f2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+          F2 pr;
+          if (masked) {
+            const F2 x = fadd2(sv, f2(neg_m, neg_m));
+            pr = f2(ex2(x.x), ex2(x.y));
+          } else {
+            const F2 x = ffma2(sv, f2(c, c), f2(neg_m, neg_m));
+            if ((kEmuPairs >> (i & 7)) & 1u) pr = exp2_fma2(x);  // FMA pipe
+            else pr = f2(ex2(x.x), ex2(x.y));                   // MUFU
+          }
+          acc[u & 3] = fadd2(acc[u & 3], pr);
+          pk[u] = pack2(pr.x, pr.y, BF16);
+          if (BF16) accr[u & 1] = fadd2(accr[u & 1], unpack_bf16x2(pk[u]));
         }
-        lsum += p0 + p1;
-        pk[i] = pack2(p0, p1, BF16);
-        if (BF16) lsum_r += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+        tmem_st_x16(tm + sb * 128 + g * 16, pk);
       }
-      l = l * alpha + lsum;
-      if (BF16) l_r = l_r * alpha + lsum_r;
-      tmem_st_x64(tm + sb * 128, pk);
+      const F2 a01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+      l = l * alpha + (a01.x + a01.y);
+      if (BF16) {
+        const F2 r01 = fadd2(accr[0], accr[1]);
+        l_r = l_r * alpha + (r01.x + r01.y);
+      }
       if (__any_sync(0xffffffffu, need)) {
         if (NQ == 1) {  // PV(j-1) must have finished accumulating into O
           ok = wait_bar(B(G::B_PVDONE), (pv_seen + j - 1) & 1u, cx.abort_flag);
@@ -486,7 +526,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(B(G::B_PFULL + q));
+      if (lane == 0) mbar_arrive(B(G::B_PFULL + sb));
     }
     pv_seen += nblk;
 
@@ -566,6 +606,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   cx.tmem = misc[0];
 
+  // Registers: 168 per thread at launch (384 threads, one CTA per SM); the two
+  // softmax warpgroups take 208, the MMA / TMA / idle warpgroup keeps 88
+  // (2 x 128 x 208 + 128 x 88 = 64512 = 384 x 168).  The wait helpers are
+  // inlined: ptxas cannot allocate a call inside a region resized this way.
+  if (warp < 8) setmaxnreg_inc_208();
+  else setmaxnreg_dec_88();
   if (warp < 8) {
     if (NQ == 2 || warp < 4) role_softmax<D, NQ, BF16>(cx, p, warp >> 2, warp & 3, lane);
   } else if (warp == 8) {
@@ -584,6 +630,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     tmem_dealloc(cx.tmem, G::TMEM_COLS);
+  }
+}
+
+// Evaluates the FMA-pipe exp2 used by the softmax on an array (diagnostics / tests).
+__global__ void exp2_fma_eval_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const F2 r = exp2_fma2(f2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_fma2(f2(x[i], 0.f)).x;
   }
 }
 
@@ -786,6 +844,15 @@ int fa_device_status(int reset) {
       return -1;
   }
   return static_cast<int>(v);
+}
+
+int fa_debug_exp2_fma(const float* x, float* y, int n, void* stream) {
+  if (!x || !y) return FA_ERR_NULL_POINTER;
+  if (n < 1) return FA_ERR_BAD_SHAPE;
+  const int threads = 256, pairs = (n + 1) / 2;
+  fa::exp2_fma_eval_kernel<<<(pairs + threads - 1) / threads, threads, 0,
+                             reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 int fa_device_timeout_site(unsigned long long* site) {

@@ -147,6 +147,83 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+
+// ------------------------------------------------------------------ packed fp32 pairs
+struct F2 {
+  float x, y;
+};
+__device__ __forceinline__ F2 f2(float a, float b) { return F2{a, b}; }
+__device__ __forceinline__ F2 ffma2(F2 a, F2 b, F2 c) {  // a * b + c, both lanes, one rounding
+  F2 r;
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+__device__ __forceinline__ F2 fadd2(F2 a, F2 b) {
+  F2 r;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ F2 fmul2(F2 a, F2 b) {
+  F2 r;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair, on the FMA/ALU pipes instead of the MUFU unit.
+// x = n + f with n = round(x) (by adding 1.5 * 2^23, which leaves n in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f comes from the degree-3 polynomial
+// minimising the maximum relative error on that interval (Remez fit, see
+// fit_exp2_poly.py; max relative error 7.5e-5), and 2^n is added to its
+// exponent field.  x is clamped at -125 so the exponent never underflows: the
+// result is then ~2^-125 instead of 0, negligible against the row sums it
+// feeds.  Valid for x <= 64.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+__device__ __forceinline__ F2 exp2_fma2(F2 x) {
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const F2 t = fadd2(x, f2(kRound, kRound));
+  const F2 r = fadd2(t, f2(-kRound, -kRound));  // round(x), exact
+  const F2 f = ffma2(r, f2(-1.0f, -1.0f), x);   // x - round(x), exact
+  F2 p = ffma2(f, f2(kExp2C3, kExp2C3), f2(kExp2C2, kExp2C2));
+  p = ffma2(p, f, f2(kExp2C1, kExp2C1));
+  p = ffma2(p, f, f2(kExp2C0, kExp2C0));
+  return F2{__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+            __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23))};
+}
+
+__device__ __forceinline__ void setmaxnreg_inc_208() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+}
+__device__ __forceinline__ void setmaxnreg_dec_88() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+}
+
 // ---- generated register-list wrappers (tcgen05.ld + wait in one statement; tcgen05.st) ----
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t* r) {
   asm volatile(
