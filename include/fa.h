@@ -117,8 +117,9 @@ int fa_device_timeout_site(unsigned long long *site);
  * Diagnostic: y[i] = 2^x[i] computed the way the softmax computes the share of
  * its exponentials that it moves from the MUFU unit to the FMA pipe (no
  * counterpart on the pages; it exists so tests can check that approximation):
- * round-to-nearest range reduction and a degree-3 minimax polynomial, max
- * relative error 7.5e-5 for -125 <= x <= 64; inputs below -125 give ~2^-125.
+ * round-to-nearest range reduction and a cubic minimax polynomial with p(0) = 1,
+ * max relative error 1.02e-4 for -125 <= x < 128, exact at integer x; inputs
+ * below -125 give ~2^-125.
  * x, y: device float arrays of n elements.  Asynchronous on `stream`.
  */
 int fa_debug_exp2_fma(const float *x, float *y, int n, void *stream);

@@ -99,6 +99,21 @@ def test_mixed(cuda_dev, w):
     compare(w, cuda_dev)
 
 
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_single_visible_key_is_exact(cuda_dev, dtype, D):
+    """A row that sees one key has softmax weight exactly 1: O must equal that V row bit
+    for bit.  Holds for every row when Nk = 1 and for row 0 under causal masking, for
+    positive and negative scores alike (a wrong row max shows up here first)."""
+    w = Workload("nk1", 2, 4, 2, 700, 1, D, dtype, False, seed=21)
+    (q, k, v), o, _ = run_cuda(w, cuda_dev)
+    want = v[:, :, 0].repeat_interleave(2, dim=1)[:, :, None, :].expand(-1, -1, 700, -1)
+    assert torch.equal(o.cpu(), want.contiguous())
+    wc = Workload("c-row0", 2, 4, 2, 300, 300, D, dtype, True, seed=22, q_mult=3.0)
+    (q, k, v), o, _ = run_cuda(wc, cuda_dev)
+    assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0].repeat_interleave(2, dim=1))
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.5])
 def test_scale_values(cuda_dev, scale):
     w = Workload("scale", 1, 2, 2, 300, 300, 128, "fp16", True, seed=3, scale=scale)

@@ -386,18 +386,23 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
 // Exps of these pairs (bit k: pair index % 8 == k) run on the FMA pipe; the
 // rest on MUFU.  MUFU throughput (16 ex2 / clock / SM) alone would equal the
 // tensor-core time of S and PV at head_dim 128.
-constexpr uint32_t kEmuPairs = 0x52u;  // pairs 1, 4, 6 of every 8: 3/8 of the exps
+#ifndef FA_EMU_PAIRS
+#define FA_EMU_PAIRS 0x52u  // pairs 1, 4, 6 of every 8: 3/8 of the exps
+#endif
+constexpr uint32_t kEmuPairs = FA_EMU_PAIRS;
 
-// Row max / min of 128 scores: four independent chains of 3-input max.
+// Row max / min of 128 scores: four independent chains of two-input max (min).
+// (A three-input max.f32 produced wrong maxima for masked rows in this kernel,
+// so only the two-input form is used.)
 __device__ __forceinline__ float row_max(const uint32_t* v) {
   float a0 = __uint_as_float(v[0]), a1 = __uint_as_float(v[1]), a2 = __uint_as_float(v[2]),
         a3 = __uint_as_float(v[3]);
 #pragma unroll
-  for (int i = 4; i < kBN; i += 8) {
-    a0 = fmax3(a0, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
-    a1 = fmax3(a1, __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-    a2 = fmax3(a2, __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
-    a3 = fmax3(a3, __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
+  for (int i = 4; i < kBN; i += 4) {
+    a0 = fmaxf(a0, __uint_as_float(v[i]));
+    a1 = fmaxf(a1, __uint_as_float(v[i + 1]));
+    a2 = fmaxf(a2, __uint_as_float(v[i + 2]));
+    a3 = fmaxf(a3, __uint_as_float(v[i + 3]));
   }
   return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
 }
@@ -405,11 +410,11 @@ __device__ __forceinline__ float row_min(const uint32_t* v) {
   float a0 = __uint_as_float(v[0]), a1 = __uint_as_float(v[1]), a2 = __uint_as_float(v[2]),
         a3 = __uint_as_float(v[3]);
 #pragma unroll
-  for (int i = 4; i < kBN; i += 8) {
-    a0 = fmin3(a0, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
-    a1 = fmin3(a1, __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-    a2 = fmin3(a2, __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
-    a3 = fmin3(a3, __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
+  for (int i = 4; i < kBN; i += 4) {
+    a0 = fminf(a0, __uint_as_float(v[i]));
+    a1 = fminf(a1, __uint_as_float(v[i + 1]));
+    a2 = fminf(a2, __uint_as_float(v[i + 2]));
+    a3 = fminf(a3, __uint_as_float(v[i + 3]));
   }
   return fminf(fminf(a0, a1), fminf(a2, a3));
 }

@@ -180,29 +180,18 @@ __device__ __forceinline__ F2 fmul2(F2 a, F2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return r;
 }
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-__device__ __forceinline__ float fmin3(float a, float b, float c) {
-  float r;
-  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // 2^x for a pair, on the FMA/ALU pipes instead of the MUFU unit.
 // x = n + f with n = round(x) (by adding 1.5 * 2^23, which leaves n in the low
-// mantissa bits) and f in [-1/2, 1/2]; 2^f comes from the degree-3 polynomial
-// minimising the maximum relative error on that interval (Remez fit, see
-// fit_exp2_poly.py; max relative error 7.5e-5), and 2^n is added to its
-// exponent field.  x is clamped at -125 so the exponent never underflows: the
-// result is then ~2^-125 instead of 0, negligible against the row sums it
-// feeds.  Valid for x <= 64.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716685295105f;
+// mantissa bits) and f in [-1/2, 1/2]; 2^f comes from the cubic
+// 1 + c1 f + c2 f^2 + c3 f^3 whose coefficients minimise the maximum relative
+// error on that interval (linear-programming minimax fit, see
+// fit_exp2_poly.py; max relative error 1.02e-4, exact at integer x), and 2^n
+// is added to its exponent field.  x is clamped at -125 so the exponent never
+// underflows: the result is then ~2^-125 instead of 0, negligible against the
+// row sums it feeds.  Valid for x < 128.
+constexpr float kExp2C1 = 0.693282961845398f;
+constexpr float kExp2C2 = 0.2422109991312027f;
+constexpr float kExp2C3 = 0.055008918046951294f;
 __device__ __forceinline__ F2 exp2_fma2(F2 x) {
   const float kRound = 12582912.0f;  // 1.5 * 2^23
   x.x = fmaxf(x.x, -125.0f);
@@ -212,7 +201,7 @@ __device__ __forceinline__ F2 exp2_fma2(F2 x) {
   const F2 f = ffma2(r, f2(-1.0f, -1.0f), x);   // x - round(x), exact
   F2 p = ffma2(f, f2(kExp2C3, kExp2C3), f2(kExp2C2, kExp2C2));
   p = ffma2(p, f, f2(kExp2C1, kExp2C1));
-  p = ffma2(p, f, f2(kExp2C0, kExp2C0));
+  p = ffma2(p, f, f2(1.0f, 1.0f));
   return F2{__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
             __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23))};
 }
