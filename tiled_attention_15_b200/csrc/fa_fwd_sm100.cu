@@ -274,23 +274,29 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
     tc_fence_after();
     return r;
   };
+  // Shared-memory descriptors are built once; each MMA of a K-loop only adds a
+  // constant byte offset (>> 4) to the start-address field.
+  const uint64_t dq0 = sdesc_sw128(cx.sbase + G::OFF_Q, 16, 1024);
+  const uint64_t dkv0 = sdesc_sw128(cx.sbase + G::OFF_KV, 16, 1024);
+  const uint64_t dv0 = sdesc_sw128(cx.sbase + G::OFF_KV, G::CHUNK_KV, 1024);
   auto issue_S = [&](int qt, int sbuf, int st) {
-    const uint32_t qa = cx.sbase + G::OFF_Q + qt * G::Q_BYTES;
-    const uint32_t ka = cx.sbase + G::OFF_KV + st * G::KV_BYTES;
+    const uint64_t a0 = dq0 + static_cast<uint64_t>((qt * G::Q_BYTES) >> 4);
+    const uint64_t b0 = dkv0 + static_cast<uint64_t>((st * G::KV_BYTES) >> 4);
+    const uint32_t d = tm + sbuf * 128;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t a = sdesc_sw128(qa + (kk >> 2) * G::CHUNK_Q + (kk & 3) * 32, 16, 1024);
-      const uint64_t b = sdesc_sw128(ka + (kk >> 2) * G::CHUNK_KV + (kk & 3) * 32, 16, 1024);
-      mma_ss(tm + sbuf * 128, a, b, kIdS, kk > 0 ? 1u : 0u);
+      const uint32_t off_a = ((kk >> 2) * G::CHUNK_Q + (kk & 3) * 32) >> 4;
+      const uint32_t off_b = ((kk >> 2) * G::CHUNK_KV + (kk & 3) * 32) >> 4;
+      mma_ss(d, a0 + off_a, b0 + off_b, kIdS, kk > 0 ? 1u : 0u);
     }
   };
   auto issue_PV = [&](int ot, int sbuf, int st, bool acc) {
-    const uint32_t va = cx.sbase + G::OFF_KV + st * G::KV_BYTES;
+    const uint64_t b0 = dv0 + static_cast<uint64_t>((st * G::KV_BYTES) >> 4);
+    const uint32_t d = tm + 256 + ot * D, a = tm + sbuf * 128;
 #pragma unroll
-    for (int kk = 0; kk < kBN / 16; ++kk) {
-      const uint64_t b = sdesc_sw128(va + kk * 2048, G::CHUNK_KV, 1024);
-      mma_ts(tm + 256 + ot * D, tm + sbuf * 128 + kk * 8, b, kIdPV, (acc || kk > 0) ? 1u : 0u);
-    }
+    for (int kk = 0; kk < kBN / 16; ++kk)
+      mma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), kIdPV,
+             (acc || kk > 0) ? 1u : 0u);
   };
   // Before the first PV of a tile into O_q: the previous tile's epilogue must
   // have read O_q out of tensor memory.
@@ -387,7 +393,7 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
 // rest on MUFU.  MUFU throughput (16 ex2 / clock / SM) alone would equal the
 // tensor-core time of S and PV at head_dim 128.
 #ifndef FA_EMU_PAIRS
-#define FA_EMU_PAIRS 0x52u  // pairs 1, 4, 6 of every 8: 3/8 of the exps
+#define FA_EMU_PAIRS 0x11u  // pairs 0 and 4 of every 8: 1/4 of the exps
 #endif
 constexpr uint32_t kEmuPairs = FA_EMU_PAIRS;
 
