@@ -49,6 +49,8 @@
 #ifndef FA_H_
 #define FA_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -92,6 +94,36 @@ int fa_fwd_fp16(const void *q, const void *k, const void *v, void *o, float *lse
                 int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream);
 int fa_fwd_bf16(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
                 int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream);
+
+/*
+ * fa_fwd with a caller-provided device workspace (no counterpart on the pages: it
+ * exists for load balance on this device).  With a workspace, a non-causal call
+ * whose last round of work tiles would keep at most half of the SMs busy gives
+ * each of those tiles to two CTAs, one per half of the key blocks; each half
+ * leaves its un-normalised partial output in the workspace and the second to
+ * finish merges.  Results agree with fa_fwd within rounding (the order of the
+ * additions differs).
+ *   workspace        device memory of at least fa_fwd_workspace_size(D) bytes,
+ *                    256-byte aligned (else FA_ERR_MISALIGNED), zero-filled
+ *                    before its first use.  Every call that completes leaves the
+ *                    workspace's arrival counters at zero again, so one zero-fill
+ *                    suffices.  Calls that may run concurrently need separate
+ *                    workspaces.  After FA_ERR_DEVICE_TIMEOUT, zero it again.
+ *                    NULL (or too small) gives exactly fa_fwd.
+ *   workspace_bytes  its size.
+ */
+int fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+              int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream, int dtype,
+              void *workspace, size_t workspace_bytes);
+
+/* Workspace bytes fa_fwd_ws needs on the current device for head_dim D (about 20 MB
+ * on a 148-SM B200); 0 if D is unsupported or no device is current. */
+size_t fa_fwd_workspace_size(int D);
+
+/* Process-wide cap on the CTAs (one per SM) a launch uses; 0, the default, means
+ * every SM.  Useful to leave SMs to concurrent work.  Returns the previous cap,
+ * or FA_ERR_BAD_SHAPE for n < 0. */
+int fa_set_max_ctas(int n);
 
 /* Human-readable text for a status code (static storage; never NULL). */
 const char *fa_status_string(int status);

@@ -87,3 +87,13 @@ def test_valid_arguments_reach_the_device_check(lib):
         pytest.skip("host-only check")
     assert _call() == 8  # FA_ERR_NO_DEVICE without a GPU
     assert _call(lse=0) == 8  # lse may be NULL
+
+
+def test_workspace_entry_point_host_checks(lib):
+    a = dict(GOOD)
+    args = (a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"],
+            a["D"], ctypes.c_float(a["scale"]), a["causal"], None, a["dtype"])
+    assert lib.fa_fwd_ws(*args, 7 * A + 128, 1 << 20) == 2  # workspace not 256-byte aligned
+    assert lib.fa_fwd_ws(*args[:10], 96, *args[11:], 7 * A, 1 << 20) == 5  # head_dim checked first
+    assert fa.set_max_ctas(-1) == 3
+    assert fa.set_max_ctas(0) == 0

@@ -114,6 +114,42 @@ def test_single_visible_key_is_exact(cuda_dev, dtype, D):
     assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0].repeat_interleave(2, dim=1))
 
 
+# Split tails: with the CTA cap at 8, these shapes leave a last round of at most 4 work
+# tiles, which the workspace path gives to two CTAs each (one per half of the key
+# blocks) and merges.  Ragged query/key lengths and an odd number of key blocks included.
+# (Splitting needs at least 24 key blocks of 128, so Nk >= 2945 here.)
+SPLIT = [
+    Workload("split D128 fp16", 1, 5, 5, 512, 3072, 128, "fp16", False, seed=31),
+    Workload("split D128 bf16 GQA ragged", 1, 10, 5, 300, 3500, 128, "bf16", False, seed=32),
+    Workload("split D64 fp16 odd blocks", 2, 5, 5, 256, 3201, 64, "fp16", False, seed=33),
+    Workload("split D256 bf16", 1, 5, 5, 512, 3072, 256, "bf16", False, seed=34),
+    Workload("split D256 fp16 ragged", 1, 3, 1, 333, 4000, 256, "fp16", False, seed=35),
+]
+
+
+@pytest.mark.parametrize("w", SPLIT, ids=lambda w: w.name)
+def test_split_tail(cuda_dev, w):
+    tiles = fa.num_tiles(w.B, w.Hq, w.Nq, w.D)
+    assert tiles > 8 and 0 < tiles % 8 <= 4  # the shape really exercises the split
+    prev = fa.set_max_ctas(8)
+    try:
+        o1, l1, (q, k, v), _, _ = compare(w, cuda_dev)
+        # a second call on the same workspace: counters were left at zero
+        o2, l2 = fa.fa_fwd(q.to(cuda_dev), k.to(cuda_dev), v.to(cuda_dev), scale=w.softmax_scale)
+        torch.cuda.synchronize()
+        assert fa.device_status(reset=True) == 0
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        # and agrees with the no-workspace path within rounding
+        o3, l3 = fa.fa_fwd(q.to(cuda_dev), k.to(cuda_dev), v.to(cuda_dev), scale=w.softmax_scale,
+                           use_workspace=False)
+        torch.cuda.synchronize()
+        tol = TOL[w.dtype][0]
+        assert (o1.float() - o3.float()).abs().max().item() <= tol
+        assert (l1 - l3).abs().max().item() <= 1e-4
+    finally:
+        fa.set_max_ctas(prev)
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.5])
 def test_scale_values(cuda_dev, scale):
     w = Workload("scale", 1, 2, 2, 300, 300, 128, "fp16", True, seed=3, scale=scale)

@@ -23,8 +23,9 @@ FA_OK = 0
 FA_ERR_DEVICE_TIMEOUT = 11
 
 # Every symbol include/fa.h declares (checked by the tests).
-EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_status_string", "fa_device_status",
-            "fa_device_timeout_site", "fa_debug_exp2_fma", "fa_fwd_num_tiles")
+EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
+            "fa_set_max_ctas", "fa_status_string", "fa_device_status", "fa_device_timeout_site",
+            "fa_debug_exp2_fma", "fa_fwd_num_tiles")
 
 
 class FaError(RuntimeError):
@@ -52,6 +53,12 @@ def load_library() -> ctypes.CDLL:
     for name in ("fa_fwd_fp16", "fa_fwd_bf16"):
         getattr(lib, name).argtypes = fwd_args
         getattr(lib, name).restype = i
+    lib.fa_fwd_ws.argtypes = fwd_args + [i, vp, ctypes.c_size_t]
+    lib.fa_fwd_ws.restype = i
+    lib.fa_fwd_workspace_size.argtypes = [i]
+    lib.fa_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_set_max_ctas.argtypes = [i]
+    lib.fa_set_max_ctas.restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_device_status.argtypes = [i]
@@ -103,6 +110,30 @@ def num_tiles(B: int, Hq: int, Nq: int, D: int) -> int:
     return int(load_library().fa_fwd_num_tiles(B, Hq, Nq, D))
 
 
+def set_max_ctas(n: int) -> int:
+    """Cap the CTAs a launch uses (0 = one per SM); returns the previous cap."""
+    return int(load_library().fa_set_max_ctas(int(n)))
+
+
+_workspaces = {}
+
+
+def workspace(device, stream_handle: int):
+    """Zero-filled workspace for fa_fwd_ws, one per (device, stream), large enough for any D."""
+    import torch
+    key = (device.index, int(stream_handle or 0))
+    ws = _workspaces.get(key)
+    if ws is None:
+        lib = load_library()
+        with torch.cuda.device(device):
+            size = max(int(lib.fa_fwd_workspace_size(d)) for d in (64, 128, 256))
+        if size == 0:
+            raise FaError(8, "fa_fwd_workspace_size")
+        ws = torch.zeros(size, dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
 def fa_fwd_raw(q: int, k: int, v: int, o: int, lse: Optional[int], B: int, Hq: int, Hkv: int,
                Nq: int, Nk: int, D: int, scale: float, causal: bool, stream: int,
                dtype: int) -> int:
@@ -113,12 +144,15 @@ def fa_fwd_raw(q: int, k: int, v: int, o: int, lse: Optional[int], B: int, Hq: i
 
 
 def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False,
-           return_lse: bool = True, stream=None) -> Tuple[object, Optional[object]]:
+           return_lse: bool = True, stream=None,
+           use_workspace: bool = True) -> Tuple[object, Optional[object]]:
     """Fused attention forward on the current CUDA stream.
 
     q: [B, Hq, Nq, D], k/v: [B, Hkv, Nk, D] contiguous CUDA tensors, fp16 or bf16.
     o: optional output like q; lse: optional float32 [B, Hq, Nq] output.
-    scale defaults to 1/sqrt(D).  Returns (o, lse or None).
+    scale defaults to 1/sqrt(D).  use_workspace: call fa_fwd_ws with a cached
+    per-(device, stream) workspace (split tails for load balance), else fa_fwd.
+    Returns (o, lse or None).
     """
     import torch
 
@@ -147,9 +181,14 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
     elif hasattr(stream, "cuda_stream"):
         stream = stream.cuda_stream
     dtype = FA_BF16 if q.dtype == torch.bfloat16 else FA_FP16
-    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                    lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, D,
-                    ctypes.c_float(scale), 1 if causal else 0, stream or None, dtype)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+            lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, D,
+            ctypes.c_float(scale), 1 if causal else 0, stream or None, dtype)
+    if use_workspace:
+        ws = workspace(q.device, stream)
+        rc = lib.fa_fwd_ws(*args, ws.data_ptr(), ws.numel())
+    else:
+        rc = lib.fa_fwd(*args)
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd")
     return o, lse

@@ -42,6 +42,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "fa.h"
@@ -72,8 +73,8 @@ struct Geometry {
   static constexpr int OFF_KV = NQ * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NST * KV_BYTES;
   // mbarrier indices
-  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = 2 + NST,
-                       B_SFULL = 2 + 2 * NST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
+  static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NST,
+                       B_SFULL = 4 + 2 * NST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
                        B_OEMPTY = B_OFULL + 2, B_PVDONE = B_OEMPTY + 2, NBAR = B_PVDONE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (u32)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
@@ -91,6 +92,14 @@ struct FwdParams {
   int qt_per_head;  // work tiles per (batch, head)
   int n_tiles;
   int nkb;  // key blocks: ceil(Nk / kBN)
+  // Split tail: tiles [n_whole, n_tiles) are each processed as two units, one per
+  // half of the key blocks; n_units = n_whole + 2 * (n_tiles - n_whole).  Each half
+  // leaves its un-normalised partial in the workspace and the second one to finish
+  // a row group merges (see merge_epilogue).
+  int n_whole, n_units;
+  float* ws_o;      // [split tile][half][NQ][128 rows][D] partial O (fp32)
+  float4* ws_ml;    // [split tile][half][NQ][128 rows] (m, l, l_rounded, 0)
+  int* ws_cnt;      // [split tile][NQ][4 row groups] arrival counters (left at 0)
 };
 
 struct Tile {
@@ -99,11 +108,23 @@ struct Tile {
   int kvz;    // b * Hkv + kv head
   int nblk[2];
   int nb;
+  int jb;     // first key block of this unit
+  int slot;   // split-tile index, or -1 for a whole tile
+  int half;   // which key half of a split tile
 };
 
 template <int NQ>
-__device__ __forceinline__ Tile get_tile(const FwdParams& p, int t) {
+__device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
   Tile T;
+  int t = u;
+  T.slot = -1;
+  T.half = 0;
+  if (u >= p.n_whole) {  // half of a split tile
+    const int v = u - p.n_whole;
+    t = p.n_whole + (v >> 1);
+    T.slot = v >> 1;
+    T.half = v & 1;
+  }
   const int BH = p.B * p.Hq;
   int qt;
   if (p.causal) {  // heaviest (last) query tiles first
@@ -116,13 +137,19 @@ __device__ __forceinline__ Tile get_tile(const FwdParams& p, int t) {
   T.row0 = qt * NQ * kBM;
   const int b = T.bh / p.Hq, hq = T.bh % p.Hq;
   T.kvz = b * p.Hkv + hq / p.group;
+  int kb0 = 0, kb1 = p.nkb;  // split units: non-causal only (the host guarantees it)
+  if (T.slot >= 0) {
+    kb0 = T.half ? p.nkb / 2 : 0;
+    kb1 = T.half ? p.nkb : p.nkb / 2;
+  }
+  T.jb = kb0;
   T.nb = 0;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int rf = T.row0 + q * kBM;
     int n = 0;
     if (q < NQ && rf < p.Nq) {
-      n = p.nkb;
+      n = kb1 - kb0;
       if (p.causal) {
         const int rl = min(rf + kBM - 1, p.Nq - 1);
         n = min(p.nkb, rl / kBN + 1);
@@ -207,52 +234,63 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
   prefetch_tmap(tv);
   const uint64_t pol_kv = policy_evict_last();
   const uint64_t pol_q = policy_evict_first();
-  uint32_t kv_it = 0, qe_phase = 0, q_issued = 0;
+  uint32_t kv_it = 0, qe_phase[2] = {0u, 0u}, q_issued[2] = {0u, 0u};
   bool ok = true;
-  TileIter it(p.n_tiles);
+  auto load_q = [&](const Tile& T, int q) -> bool {
+    if (q_issued[q]) {
+      if (!wait_bar(cx.bar(G::B_QEMPTY + q, G::OFF_BAR), qe_phase[q], cx.abort_flag)) return false;
+      qe_phase[q] ^= 1u;
+    }
+    mbar_arrive_expect_tx(cx.bar(G::B_QFULL + q, G::OFF_BAR), G::Q_BYTES);
+#pragma unroll
+    for (int c = 0; c < G::DCH; ++c)
+      tma_load_3d(cx.sbase + G::OFF_Q + q * G::Q_BYTES + c * G::CHUNK_Q, tq,
+                  cx.bar(G::B_QFULL + q, G::OFF_BAR), c * 64, T.row0 + q * kBM, T.bh, pol_q);
+    ++q_issued[q];
+    return true;
+  };
+  auto load_kv = [&](const Tile& T, const CUtensorMap* m, int j) -> bool {
+    const int st = kv_it % G::NST;
+    if (kv_it >= (uint32_t)G::NST) {
+      if (!wait_bar(cx.bar(G::B_KVEMPTY + st, G::OFF_BAR), ((kv_it / G::NST) - 1) & 1u,
+                    cx.abort_flag))
+        return false;
+    }
+    mbar_arrive_expect_tx(cx.bar(G::B_KVFULL + st, G::OFF_BAR), G::KV_BYTES);
+#pragma unroll
+    for (int c = 0; c < G::DCH; ++c)
+      tma_load_3d(cx.sbase + G::OFF_KV + st * G::KV_BYTES + c * G::CHUNK_KV, m,
+                  cx.bar(G::B_KVFULL + st, G::OFF_BAR), c * 64, (T.jb + j) * kBN, T.kvz, pol_kv);
+    ++kv_it;
+    return true;
+  };
+  TileIter it(p.n_units);
   int t;
   while (ok && it.next(t)) {
     const Tile T = get_tile<NQ>(p, t);
-    if (q_issued) {
-      if (!wait_bar(cx.bar(G::B_QEMPTY, G::OFF_BAR), qe_phase, cx.abort_flag)) { ok = false; break; }
-      qe_phase ^= 1u;
-    }
-    mbar_arrive_expect_tx(cx.bar(G::B_QFULL, G::OFF_BAR), NQ * G::Q_BYTES);
-#pragma unroll
-    for (int q = 0; q < NQ; ++q)
-#pragma unroll
-      for (int c = 0; c < G::DCH; ++c)
-        tma_load_3d(cx.sbase + G::OFF_Q + q * G::Q_BYTES + c * G::CHUNK_Q, tq,
-                    cx.bar(G::B_QFULL, G::OFF_BAR), c * 64, T.row0 + q * kBM, T.bh, pol_q);
-    ++q_issued;
+    // Q0, then K0 (the first S MMA of the tile needs only these), then Q1 -- each
+    // Q tile waits only for the last S MMA that read its previous contents.
     // K/V block order matches the MMA warp's consumption order:
     //   NQ = 2: K0, V0, K1, V1, ...      NQ = 1: K0, K1, V0, K2, V1, ...
-    for (int s = 0; s < 2 * T.nb && ok; ++s) {
+    if (T.nblk[0] > 0 && !load_q(T, 0)) { ok = false; break; }
+    if (!load_kv(T, tk, 0)) { ok = false; break; }
+    if (NQ == 2 && T.nblk[1] > 0 && !load_q(T, 1)) { ok = false; break; }
+    for (int s = 1; s < 2 * T.nb && ok; ++s) {
       int j;
       bool is_k;
-      if (s == 0) { j = 0; is_k = true; }
-      else if (NQ == 2) { j = s / 2; is_k = (s & 1) == 0; }   // s=1:V0 s=2:K1 s=3:V1 ...
-      else {                                                    // s=1:K1 s=2:V0 s=3:K2 ...
+      if (NQ == 2) { j = s / 2; is_k = (s & 1) == 0; }   // s=1:V0 s=2:K1 s=3:V1 ...
+      else {                                              // s=1:K1 s=2:V0 s=3:K2 ...
         if (s == 2 * T.nb - 1) { j = T.nb - 1; is_k = false; }
         else { is_k = (s & 1) == 1; j = is_k ? (s + 1) / 2 : s / 2 - 1; }
       }
-      const int st = kv_it % G::NST;
-      if (kv_it >= (uint32_t)G::NST) {
-        if (!wait_bar(cx.bar(G::B_KVEMPTY + st, G::OFF_BAR), ((kv_it / G::NST) - 1) & 1u,
-                      cx.abort_flag)) { ok = false; break; }
-      }
-      mbar_arrive_expect_tx(cx.bar(G::B_KVFULL + st, G::OFF_BAR), G::KV_BYTES);
-#pragma unroll
-      for (int c = 0; c < G::DCH; ++c)
-        tma_load_3d(cx.sbase + G::OFF_KV + st * G::KV_BYTES + c * G::CHUNK_KV, is_k ? tk : tv,
-                    cx.bar(G::B_KVFULL + st, G::OFF_BAR), c * 64, j * kBN, T.kvz, pol_kv);
-      ++kv_it;
+      if (!load_kv(T, is_k ? tk : tv, j)) ok = false;
     }
   }
   if (!ok) {  // abort: let this CTA's own loads land before the CTA exits
     for (uint32_t n = (kv_it > (uint32_t)G::NST ? kv_it - G::NST : 0); n < kv_it; ++n)
       drain_bar(cx.bar(G::B_KVFULL + n % G::NST, G::OFF_BAR), (n / G::NST) & 1u);
-    if (q_issued) drain_bar(cx.bar(G::B_QFULL, G::OFF_BAR), (q_issued - 1) & 1u);
+    for (int q = 0; q < 2; ++q)
+      if (q_issued[q]) drain_bar(cx.bar(G::B_QFULL + q, G::OFF_BAR), (q_issued[q] - 1) & 1u);
   }
 }
 
@@ -262,7 +300,7 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
   using G = Geometry<D, NQ>;
   constexpr uint32_t kIdS = idesc_f16(kBM, kBN, BF16, false);  // Q, K both K-major
   constexpr uint32_t kIdPV = idesc_f16(kBM, D, BF16, true);    // V is N(=D)-major
-  uint32_t kv_it = 0, q_phase = 0, p_phase[2] = {0u, 0u}, oe_phase[2] = {0u, 0u};
+  uint32_t kv_it = 0, q_phase[2] = {0u, 0u}, p_phase[2] = {0u, 0u}, oe_phase[2] = {0u, 0u};
   bool o_pending[2] = {false, false};
   const uint32_t tm = cx.tmem;
   auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
@@ -308,6 +346,12 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
     tc_fence_after();
     return true;
   };
+  auto q_ready = [&](int q) -> bool {
+    if (!wait_bar(B(G::B_QFULL + q), q_phase[q], cx.abort_flag)) return false;
+    q_phase[q] ^= 1u;
+    tc_fence_after();
+    return true;
+  };
   auto p_ready = [&](int q) -> bool {
     if (!wait_bar(B(G::B_PFULL + q), p_phase[q], cx.abort_flag)) return false;
     p_phase[q] ^= 1u;
@@ -315,22 +359,29 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
     return true;
   };
 
-  TileIter it(p.n_tiles);
+  TileIter it(p.n_units);
   int t;
   while (it.next(t)) {
     const Tile T = get_tile<NQ>(p, t);
-    if (!wait_bar(B(G::B_QFULL), q_phase, cx.abort_flag)) return;
-    q_phase ^= 1u;
-    tc_fence_after();
     const int nb = T.nb;
     int kst;
     if (!consume(kst)) return;
     if (NQ == 2) {
       // stream: S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
-      if (T.nblk[0] > 0) { issue_S(0, 0, kst); mma_commit(B(G::B_SFULL + 0)); }
-      if (T.nblk[1] > 0) { issue_S(1, 1, kst); mma_commit(B(G::B_SFULL + 1)); }
+      // q_empty[q] is committed right after the last S MMA that reads Q_q.
+      if (T.nblk[0] > 0) {
+        if (!q_ready(0)) return;
+        issue_S(0, 0, kst);
+        mma_commit(B(G::B_SFULL + 0));
+        if (T.nblk[0] == 1) mma_commit(B(G::B_QEMPTY + 0));
+      }
+      if (T.nblk[1] > 0) {
+        if (!q_ready(1)) return;
+        issue_S(1, 1, kst);
+        mma_commit(B(G::B_SFULL + 1));
+        if (T.nblk[1] == 1) mma_commit(B(G::B_QEMPTY + 1));
+      }
       mma_commit(B(G::B_KVEMPTY + kst));
-      if (nb == 1) mma_commit(B(G::B_QEMPTY));
       for (int j = 0; j < nb; ++j) {
         int vst;
         if (!consume(vst)) return;
@@ -343,7 +394,11 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
         int kst2 = -1;
         if (j + 1 < nb) {
           if (!consume(kst2)) return;
-          if (j + 1 < T.nblk[0]) { issue_S(0, 0, kst2); mma_commit(B(G::B_SFULL + 0)); }
+          if (j + 1 < T.nblk[0]) {
+            issue_S(0, 0, kst2);
+            mma_commit(B(G::B_SFULL + 0));
+            if (j + 1 == T.nblk[0] - 1) mma_commit(B(G::B_QEMPTY + 0));
+          }
         }
         if (j < T.nblk[1]) {
           if (j == 0 && !o_ready(1)) return;
@@ -353,24 +408,28 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
         }
         mma_commit(B(G::B_KVEMPTY + vst));
         if (kst2 >= 0) {
-          if (j + 1 < T.nblk[1]) { issue_S(1, 1, kst2); mma_commit(B(G::B_SFULL + 1)); }
+          if (j + 1 < T.nblk[1]) {
+            issue_S(1, 1, kst2);
+            mma_commit(B(G::B_SFULL + 1));
+            if (j + 1 == T.nblk[1] - 1) mma_commit(B(G::B_QEMPTY + 1));
+          }
           mma_commit(B(G::B_KVEMPTY + kst2));
-          if (j + 1 == nb - 1) mma_commit(B(G::B_QEMPTY));
         }
       }
     } else {
       // one query tile, two S buffers: S(0) | S(j+1) PV(j) | ...
+      if (!q_ready(0)) return;
       issue_S(0, 0, kst);
       mma_commit(B(G::B_SFULL + 0));
       mma_commit(B(G::B_KVEMPTY + kst));
-      if (nb == 1) mma_commit(B(G::B_QEMPTY));
+      if (nb == 1) mma_commit(B(G::B_QEMPTY + 0));
       for (int j = 0; j < nb; ++j) {
         if (j + 1 < nb) {
           if (!consume(kst)) return;
           issue_S(0, (j + 1) & 1, kst);
           mma_commit(B(G::B_SFULL + ((j + 1) & 1)));
           mma_commit(B(G::B_KVEMPTY + kst));
-          if (j + 1 == nb - 1) mma_commit(B(G::B_QEMPTY));
+          if (j + 1 == nb - 1) mma_commit(B(G::B_QEMPTY + 0));
         }
         int vst;
         if (!consume(vst)) return;
@@ -429,6 +488,85 @@ __device__ __forceinline__ F2 unpack_bf16x2(uint32_t w) {
   return F2{__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)};
 }
 
+// Epilogue of one half of a split tile, for the 32 rows of this warp.  Each half
+// stores its un-normalised O row (fp32), its stabiliser m and sums l, l_r; then
+// the warp bumps the counter of its row group.  The warp that arrives second
+// reads the other half's partial and writes the merged, normalised row:
+//   M = max(m0, m1),  a_h = 2^(m_h - M),  L = a0 l0 + a1 l1,
+//   O = (a0 O0 + a1 O1) / L,  LSE = (M + log2 L) ln 2,
+// and resets the counter to 0 for the next call.  Neither half waits for the
+// other, so no cross-CTA wait exists.
+template <int D, int NQ, bool BF16>
+__device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T, int q, int sub,
+                                               int lane, int row, bool live, uint32_t ocol,
+                                               float m, float l, float l_r) {
+  const int r = sub * 32 + lane;
+  const size_t mine = ((static_cast<size_t>(T.slot) * 2 + T.half) * NQ + q) * kBM + r;
+  const size_t theirs = ((static_cast<size_t>(T.slot) * 2 + (T.half ^ 1)) * NQ + q) * kBM + r;
+  p.ws_ml[mine] = make_float4(m, l, l_r, 0.f);
+  float4* my_o = reinterpret_cast<float4*>(p.ws_o + mine * D);
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t orr[32];
+    tmem_ld_x32(ocol + c0, orr);
+#pragma unroll
+    for (int x = 0; x < 8; ++x)
+      my_o[c0 / 4 + x] = make_float4(__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
+                                     __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3]));
+  }
+  __threadfence();
+  __syncwarp();
+  int* cnt = p.ws_cnt + (T.slot * NQ + q) * 4 + sub;
+  int old = 0;
+  if (lane == 0) old = atomicAdd(cnt, 1);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (old != 1) return;  // the other half merges these rows
+  __threadfence();
+  // Combine in a fixed order (half 0, then half 1), so the result does not depend
+  // on which half happens to finish second.
+  const float4 o_ml = __ldcg(p.ws_ml + theirs);
+  const bool first = T.half == 0;
+  const float m0 = first ? m : o_ml.x, m1 = first ? o_ml.x : m;
+  const float l0 = first ? l : o_ml.y, l1 = first ? o_ml.y : l;
+  const float r0 = first ? l_r : o_ml.z, r1 = first ? o_ml.z : l_r;
+  const float M = fmaxf(m0, m1);
+  const float a0 = ex2(m0 - M), a1 = ex2(m1 - M);
+  const float L = fmaf(a0, l0, a1 * l1), Lr = fmaf(a0, r0, a1 * r1);
+  const float inv = 1.f / (BF16 ? Lr : L);
+  const float s0 = a0 * inv, s1 = a1 * inv;
+  const float4* th_o = reinterpret_cast<const float4*>(p.ws_o + theirs * D);
+  uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
+                   (static_cast<size_t>(T.bh) * p.Nq + (live ? row : 0)) * D;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t orr[32];
+    tmem_ld_x32(ocol + c0, orr);
+    uint32_t w[16];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const float4 t4 = __ldcg(th_o + c0 / 4 + x);
+      const float u[4] = {__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
+                          __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3])};
+      const float v[4] = {t4.x, t4.y, t4.z, t4.w};
+      float z[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) z[e] = first ? fmaf(u[e], s0, v[e] * s1) : fmaf(v[e], s0, u[e] * s1);
+      w[2 * x] = pack2(z[0], z[1], BF16);
+      w[2 * x + 1] = pack2(z[2], z[3], BF16);
+    }
+    if (live) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+    }
+  }
+  if (p.lse != nullptr && live)
+    p.lse[static_cast<size_t>(T.bh) * p.Nq + row] = (M + log2f(L)) * kLn2;
+  __syncwarp();
+  if (lane == 0) *cnt = 0;
+}
+
 // ---------------------------------------------------------------- softmax + epilogue
 template <int D, int NQ, bool BF16>
 __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, int wg, int sub,
@@ -441,7 +579,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   uint32_t s_phase[2] = {0u, 0u}, of_phase = 0u, pv_seen = 0u;
   const int q = (NQ == 2) ? wg : 0;
 
-  TileIter it(p.n_tiles);
+  TileIter it(p.n_units);
   int t;
   while (it.next(t)) {
     const Tile T = get_tile<NQ>(p, t);
@@ -459,7 +597,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
       uint32_t sr[kBN];
       tmem_ld_x128(tm + sb * 128, sr);
 
-      const int kbase = j * kBN;
+      const int kbase = (T.jb + j) * kBN;
       const bool masked = (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst);
       float m_blk;
       if (masked) {  // scaled scores, -inf where the key is causal-future or past Nk
@@ -546,28 +684,32 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     if (!__all_sync(0xffffffffu, ok)) return;
     of_phase ^= 1u;
     tc_fence_after();
-    const float inv_l = 1.f / (BF16 ? l_r : l);
     const bool live = row < p.Nq;
-    uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
-                     (static_cast<size_t>(T.bh) * p.Nq + (live ? row : 0)) * D;
+    const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+    if (T.slot >= 0) {
+      merge_epilogue<D, NQ, BF16>(p, T, q, sub, lane, row, live, tm + 256 + q * D, m_sub, l, l_r);
+    } else {
+      const float inv_l = 1.f / (BF16 ? l_r : l);
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
+                       (static_cast<size_t>(T.bh) * p.Nq + (live ? row : 0)) * D;
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t orr[32];
-      tmem_ld_x32(tm + 256 + q * D + c0, orr);
-      uint32_t w[16];
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t orr[32];
+        tmem_ld_x32(tm + 256 + q * D + c0, orr);
+        uint32_t w[16];
 #pragma unroll
-      for (int x = 0; x < 16; ++x)
-        w[x] = pack2(__uint_as_float(orr[2 * x]) * inv_l, __uint_as_float(orr[2 * x + 1]) * inv_l,
-                     BF16);
-      if (live) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+        for (int x = 0; x < 16; ++x)
+          w[x] = pack2(__uint_as_float(orr[2 * x]) * inv_l, __uint_as_float(orr[2 * x + 1]) * inv_l,
+                       BF16);
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+          for (int x = 0; x < 4; ++x)
+            dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+        }
       }
-    }
-    if (p.lse != nullptr && live) {
-      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-      p.lse[static_cast<size_t>(T.bh) * p.Nq + row] = (m_sub + log2f(l)) * kLn2;
+      if (p.lse != nullptr && live)
+        p.lse[static_cast<size_t>(T.bh) * p.Nq + row] = (m_sub + log2f(l)) * kLn2;
     }
     tc_fence_before();
     __syncwarp();
@@ -592,8 +734,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   cx.abort_flag = misc + 1;
   if (threadIdx.x == 0) {
     auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
-    mbar_init(B(G::B_QFULL), 1);
-    mbar_init(B(G::B_QEMPTY), 1);
+    for (int q = 0; q < 2; ++q) {  // one pair per query tile: the next tile's Q0 loads early
+      mbar_init(B(G::B_QFULL + q), 1);
+      mbar_init(B(G::B_QEMPTY + q), 1);
+    }
     for (int s = 0; s < G::NST; ++s) {
       mbar_init(B(G::B_KVFULL + s), 1);
       mbar_init(B(G::B_KVEMPTY + s), 1);
@@ -708,9 +852,31 @@ bool make_map(CUtensorMap* m, const void* ptr, int D, long long rows, long long 
 
 int nq_for(int D) { return D == 256 ? 1 : 2; }
 
+std::atomic<int> g_max_ctas{0};
+
+// Workspace partition for split tails.  The arrival counters come first, at a
+// fixed place whatever the call (they must stay zero between calls); the
+// partial results of up to max_split tiles follow.  Offsets are multiples of
+// 256 bytes.
+constexpr int kMaxSplit = 1024;  // >= half the SMs of any device
+constexpr int kMinSplitBlocks = 24;
+struct WsLayout {
+  size_t cnt_off, ml_off, o_off, total;
+};
+WsLayout ws_layout(int D, int NQ, int max_split) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  WsLayout L;
+  L.cnt_off = 0;
+  L.ml_off = up(static_cast<size_t>(kMaxSplit) * 2 * 4 * sizeof(int));
+  L.o_off = L.ml_off + up(static_cast<size_t>(max_split) * 2 * NQ * 128 * sizeof(float4));
+  L.total = L.o_off + up(static_cast<size_t>(max_split) * 2 * NQ * 128 * D * sizeof(float));
+  return L;
+}
+
 template <int D, int NQ, bool BF16>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-           int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream, int dev) {
+           int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream, int dev,
+           void* ws, size_t ws_bytes) {
   using G = fa::Geometry<D, NQ>;
   static bool attr_done[kMaxDevices] = {};
   static std::mutex mu;
@@ -743,7 +909,34 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.qt_per_head = (Nq + NQ * fa::kBM - 1) / (NQ * fa::kBM);
   p.n_tiles = B * Hq * p.qt_per_head;
   p.nkb = (Nk + fa::kBN - 1) / fa::kBN;
-  const int grid = p.n_tiles < g_dev[dev].sms ? p.n_tiles : g_dev[dev].sms;
+  int ctas = g_dev[dev].sms;
+  const int cap = g_max_ctas.load();
+  if (cap > 0 && cap < ctas) ctas = cap;
+  const int grid = p.n_tiles < ctas ? p.n_tiles : ctas;
+  // Split tail: if the last round of tiles would keep at most half of the CTAs
+  // busy, give each of those tiles to two CTAs, one per half of the key blocks.
+  // Below kMinSplitBlocks key blocks the halves are too short to pay for writing
+  // and re-reading the fp32 partials (measured on the LLaMA-7B layer shape).
+  int n_split = 0;
+  const int rem = p.n_tiles % grid;
+  if (ws != nullptr && !causal && p.nkb >= kMinSplitBlocks && p.n_tiles > grid && rem > 0 &&
+      2 * rem <= grid && rem <= kMaxSplit) {
+    const WsLayout L = ws_layout(D, NQ, rem);
+    if (ws_bytes >= L.total) {
+      n_split = rem;
+      char* base = static_cast<char*>(ws);
+      p.ws_o = reinterpret_cast<float*>(base + L.o_off);
+      p.ws_ml = reinterpret_cast<float4*>(base + L.ml_off);
+      p.ws_cnt = reinterpret_cast<int*>(base + L.cnt_off);
+    }
+  }
+  if (n_split == 0) {
+    p.ws_o = nullptr;
+    p.ws_ml = nullptr;
+    p.ws_cnt = nullptr;
+  }
+  p.n_whole = p.n_tiles - n_split;
+  p.n_units = p.n_tiles + n_split;
   fa::fa_fwd_kernel<D, NQ, BF16><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
@@ -782,8 +975,9 @@ long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D) {
   return (long long)B * Hq * ((Nq + rows - 1) / rows);
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-           int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                    int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype,
+                    void* ws, size_t ws_bytes) {
   // ---- argument checks: host only, before any CUDA call
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
   if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;
@@ -822,15 +1016,43 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   const bool bf = dtype == FA_BF16;
   switch (D) {
     case 64:
-      return bf ? launch<64, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev)
-                : launch<64, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev);
+      return bf ? launch<64, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes)
+                : launch<64, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes);
     case 128:
-      return bf ? launch<128, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev)
-                : launch<128, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev);
+      return bf ? launch<128, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes)
+                : launch<128, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes);
     default:
-      return bf ? launch<256, 1, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev)
-                : launch<256, 1, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev);
+      return bf ? launch<256, 1, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes)
+                : launch<256, 1, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes);
   }
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, nullptr, 0);
+}
+
+size_t fa_fwd_workspace_size(int D) {
+  if (D != 64 && D != 128 && D != 256) return 0;
+  int dev = -1, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
+    return 0;
+  return ws_layout(D, nq_for(D), sms / 2 < kMaxSplit ? sms / 2 : kMaxSplit).total;
+}
+
+int fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+              int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype,
+              void* workspace, size_t workspace_bytes) {
+  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return FA_ERR_MISALIGNED;
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, workspace,
+                  workspace_bytes);
+}
+
+int fa_set_max_ctas(int n) {
+  if (n < 0) return FA_ERR_BAD_SHAPE;
+  return g_max_ctas.exchange(n);
 }
 
 int fa_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
