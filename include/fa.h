@@ -70,7 +70,8 @@ enum fa_status {
   FA_ERR_LAUNCH = 9,               /* the CUDA runtime refused the launch          */
   FA_ERR_DRIVER = 10,              /* tensor-map encoding via the driver failed    */
   FA_ERR_DEVICE_TIMEOUT = 11,      /* (device status) a kernel wait hit its limit  */
-  FA_ERR_OVERLAP = 12              /* o or lse overlaps q, k or v                  */
+  FA_ERR_OVERLAP = 12,             /* o or lse overlaps q, k or v                  */
+  FA_ERR_SCRATCH_TOO_SMALL = 13    /* fa_fwd_noalloc: static scratch too small     */
 };
 
 /*
@@ -119,6 +120,33 @@ int fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float *lse, 
 /* Workspace bytes fa_fwd_ws needs on the current device for head_dim D (about 20 MB
  * on a 148-SM B200); 0 if D is unsupported or no device is current. */
 size_t fa_fwd_workspace_size(int D);
+
+/*
+ * fa_fwd_ws for callers that cannot allocate device memory.  The pages have no
+ * counterpart: this entry point exists for callers such as a serving engine
+ * whose memory pool already owns all of the device's free memory, or a plug-in
+ * interface that hands the library only its inputs and outputs -- there a
+ * cudaMalloc would fail, or stall the device while the caller's stream is busy.
+ * It takes exactly fa_fwd's arguments and allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library routine); the split-tail scratch is a
+ * file-scope device array of fa_fwd_noalloc_scratch_bytes() bytes (24 MiB) that
+ * every GPU loading this library holds until the process exits.
+ *   - The first call on each device looks up that array's device address
+ *     (cudaGetSymbolAddress) with the device current; make that first call
+ *     before any stream capture.
+ *   - Each call clears the array's arrival counters on `stream` before its
+ *     kernel; all calls share the one array, so calls whose work overlaps on
+ *     the GPU (other streams, other threads) race and must not be issued.
+ *   - A problem whose split tail would need more scratch than the array holds
+ *     returns FA_ERR_SCRATCH_TOO_SMALL and launches nothing.
+ * Results equal fa_fwd_ws's for the same arguments.
+ */
+int fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream,
+                   int dtype);
+
+/* Size in bytes of fa_fwd_noalloc's static scratch array. */
+size_t fa_fwd_noalloc_scratch_bytes(void);
 
 /* Process-wide cap on the CTAs (one per SM) a launch uses; 0, the default, means
  * every SM.  Useful to leave SMs to concurrent work.  Returns the previous cap,

@@ -24,7 +24,8 @@ FA_ERR_DEVICE_TIMEOUT = 11
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
-            "fa_set_max_ctas", "fa_status_string", "fa_device_status", "fa_device_timeout_site",
+            "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
+            "fa_status_string", "fa_device_status", "fa_device_timeout_site",
             "fa_debug_exp2_fma", "fa_fwd_num_tiles")
 
 
@@ -55,6 +56,10 @@ def load_library() -> ctypes.CDLL:
         getattr(lib, name).restype = i
     lib.fa_fwd_ws.argtypes = fwd_args + [i, vp, ctypes.c_size_t]
     lib.fa_fwd_ws.restype = i
+    lib.fa_fwd_noalloc.argtypes = fwd_args + [i]
+    lib.fa_fwd_noalloc.restype = i
+    lib.fa_fwd_noalloc_scratch_bytes.argtypes = []
+    lib.fa_fwd_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.fa_fwd_workspace_size.argtypes = [i]
     lib.fa_fwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_set_max_ctas.argtypes = [i]

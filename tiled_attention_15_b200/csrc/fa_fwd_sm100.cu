@@ -873,10 +873,15 @@ WsLayout ws_layout(int D, int NQ, int max_split) {
   return L;
 }
 
+// Scratch modes of a launch: a caller workspace (split only if it fits), or the
+// library's static scratch (a split that does not fit is an error, and the
+// arrival counters are cleared on the stream before the kernel).
+enum class Scratch { kCaller, kStatic };
+
 template <int D, int NQ, bool BF16>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
            int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream, int dev,
-           void* ws, size_t ws_bytes) {
+           void* ws, size_t ws_bytes, Scratch mode) {
   using G = fa::Geometry<D, NQ>;
   static bool attr_done[kMaxDevices] = {};
   static std::mutex mu;
@@ -922,7 +927,11 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   if (ws != nullptr && !causal && p.nkb >= kMinSplitBlocks && p.n_tiles > grid && rem > 0 &&
       2 * rem <= grid && rem <= kMaxSplit) {
     const WsLayout L = ws_layout(D, NQ, rem);
+    if (ws_bytes < L.total && mode == Scratch::kStatic) return FA_ERR_SCRATCH_TOO_SMALL;
     if (ws_bytes >= L.total) {
+      if (mode == Scratch::kStatic &&
+          cudaMemsetAsync(ws, 0, L.ml_off, stream) != cudaSuccess)  // the counters start at zero
+        return FA_ERR_LAUNCH;
       n_split = rem;
       char* base = static_cast<char*>(ws);
       p.ws_o = reinterpret_cast<float*>(base + L.o_off);
@@ -965,6 +974,9 @@ const char* fa_status_string(int s) {
     case FA_ERR_DRIVER: return "tensor-map encoding failed in the CUDA driver";
     case FA_ERR_DEVICE_TIMEOUT: return "a kernel wait reached its time limit";
     case FA_ERR_OVERLAP: return "o or lse overlaps q, k or v";
+    case FA_ERR_SCRATCH_TOO_SMALL:
+      return "fa_fwd_noalloc: this problem needs more scratch than the static buffer holds; "
+             "use fa_fwd_ws";
     default: return "unknown status";
   }
 }
@@ -977,7 +989,7 @@ long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D) {
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                     int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype,
-                    void* ws, size_t ws_bytes) {
+                    void* ws, size_t ws_bytes, Scratch mode = Scratch::kCaller) {
   // ---- argument checks: host only, before any CUDA call
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
   if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;
@@ -1016,14 +1028,14 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   const bool bf = dtype == FA_BF16;
   switch (D) {
     case 64:
-      return bf ? launch<64, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes)
-                : launch<64, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes);
+      return bf ? launch<64, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode)
+                : launch<64, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode);
     case 128:
-      return bf ? launch<128, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes)
-                : launch<128, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes);
+      return bf ? launch<128, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode)
+                : launch<128, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode);
     default:
-      return bf ? launch<256, 1, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes)
-                : launch<256, 1, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes);
+      return bf ? launch<256, 1, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode)
+                : launch<256, 1, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode);
   }
 }
 
@@ -1049,6 +1061,36 @@ int fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, 
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, workspace,
                   workspace_bytes);
 }
+
+// ---- fa_fwd_noalloc: the split-tail launch with library-owned scratch ----------
+// For callers that cannot allocate device memory (see include/fa.h): the
+// scratch of the split tail lives in this file-scope device array, which every
+// GPU that loads the library holds until the process exits.  In host code the
+// array's name is only a host-side stand-in, so its device address is fetched
+// with cudaGetSymbolAddress once per device, on that device's first call.
+constexpr size_t kNoAllocScratchBytes = size_t(24) << 20;  // 24 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocDevice {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaErrorUnknown;
+};
+NoAllocDevice g_noalloc[kMaxDevices];
+
+int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream,
+                   int dtype) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_NO_DEVICE;
+  NoAllocDevice& nd = g_noalloc[dev];
+  std::call_once(nd.once, [&] { nd.err = cudaGetSymbolAddress(&nd.ptr, g_noalloc_scratch); });
+  if (nd.err != cudaSuccess || nd.ptr == nullptr) return FA_ERR_NO_DEVICE;
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, nd.ptr,
+                  kNoAllocScratchBytes, Scratch::kStatic);
+}
+
+size_t fa_fwd_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 int fa_set_max_ctas(int n) {
   if (n < 0) return FA_ERR_BAD_SHAPE;
