@@ -49,6 +49,22 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank measurement over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flops_per_step: float, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job throughput: every rank runs its own replica of the workload."""
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def workloads():
     from fa_inputs import llama7b
     return [llama7b(False), llama7b(True)]
@@ -262,14 +278,10 @@ def main():
     barrier()
     per_launch = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)] for j in range(len(ws))]
     step_ms = [sum(per_launch[j][i] for j in range(len(ws))) for i in range(K)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     assert fa.device_status(reset=True) == 0
     flops_step = sum(w.flops() for w in ws)
-    value = world * flops_step * K / (total_ms * 1e-3) / 1e12
+    value = aggregate_tflops(flops_step, K, total_ms, world)
 
     # ---- end to end: pinned host inputs -> device -> both passes -> O and LSE back to host
     hq, hk, hv = (x.pin_memory() for x in inputs[0][1:])
@@ -299,12 +311,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops_step * E / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = aggregate_tflops(flops_step, E, e2e_ms, world)
 
     # ---- gate configs (N = 4096 / 8192, D = 128), a few launches each, L2 flushed
     gate = {}

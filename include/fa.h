@@ -98,12 +98,13 @@ int fa_fwd_bf16(const void *q, const void *k, const void *v, void *o, float *lse
 
 /*
  * fa_fwd with a caller-provided device workspace (no counterpart on the pages: it
- * exists for load balance on this device).  With a workspace, a non-causal call
- * whose last round of work tiles would keep at most half of the SMs busy gives
- * each of those tiles to two CTAs, one per half of the key blocks; each half
- * leaves its un-normalised partial output in the workspace and the second to
- * finish merges.  Results agree with fa_fwd within rounding (the order of the
- * additions differs).
+ * exists for load balance on this device).  With a workspace, non-causal calls
+ * take their work tiles from a counter in the workspace (dynamic schedule), and
+ * a call whose last round of tiles would keep at most half of the SMs busy
+ * gives each of those tiles to two CTAs, one per half of the key blocks (from
+ * 24 key blocks up); each half leaves its un-normalised partial output in the
+ * workspace and the second to finish merges.  Results agree with fa_fwd within
+ * rounding (the order of the additions differs).
  *   workspace        device memory of at least fa_fwd_workspace_size(D) bytes,
  *                    256-byte aligned (else FA_ERR_MISALIGNED), zero-filled
  *                    before its first use.  Every call that completes leaves the
@@ -183,6 +184,16 @@ int fa_device_timeout_site(unsigned long long *site);
  * x, y: device float arrays of n elements.  Asynchronous on `stream`.
  */
 int fa_debug_exp2_fma(const float *x, float *y, int n, void *stream);
+
+/*
+ * Diagnostic for the failure detection of the kernels' waits (no counterpart on
+ * the pages): enqueues one warp that runs the same bounded mbarrier wait as the
+ * attention kernels on a barrier nothing ever arrives on.  After the wait limit
+ * (about 1 s) it records FA_ERR_DEVICE_TIMEOUT in the device status word and the
+ * site in fa_device_timeout_site, and returns; nothing hangs or faults.  Reset
+ * the status word (fa_device_status(1)) afterwards.
+ */
+int fa_debug_wait_timeout(void *stream);
 
 /* Number of work tiles (CTAs' units of work) one fa_fwd call would schedule;
  * 0 for invalid arguments.  Host only; used to count launches and to size tests. */

@@ -26,7 +26,7 @@ FA_ERR_DEVICE_TIMEOUT = 11
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
             "fa_status_string", "fa_device_status", "fa_device_timeout_site",
-            "fa_debug_exp2_fma", "fa_fwd_num_tiles")
+            "fa_debug_exp2_fma", "fa_debug_wait_timeout", "fa_fwd_num_tiles")
 
 
 class FaError(RuntimeError):
@@ -70,6 +70,8 @@ def load_library() -> ctypes.CDLL:
     lib.fa_device_status.restype = i
     lib.fa_device_timeout_site.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
     lib.fa_device_timeout_site.restype = i
+    lib.fa_debug_wait_timeout.argtypes = [vp]
+    lib.fa_debug_wait_timeout.restype = i
     lib.fa_debug_exp2_fma.argtypes = [vp, vp, i, vp]
     lib.fa_debug_exp2_fma.restype = i
     lib.fa_fwd_num_tiles.argtypes = [i, i, i, i]

@@ -60,6 +60,7 @@ constexpr int kThreads = 384;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
 constexpr float kRescaleThreshold = 8.0f;         // log2 units: P <= 2^8 between rescales
 constexpr float kLn2 = 0.69314718055994530942f;
+constexpr int kTileRing = 4;  // units the TMA thread may hand out ahead of the consumers
 
 template <int D, int NQ>
 struct Geometry {
@@ -75,9 +76,11 @@ struct Geometry {
   // mbarrier indices
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NST,
                        B_SFULL = 4 + 2 * NST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
-                       B_OEMPTY = B_OFULL + 2, B_PVDONE = B_OEMPTY + 2, NBAR = B_PVDONE + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (u32)
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+                       B_OEMPTY = B_OFULL + 2, B_PVDONE = B_OEMPTY + 2, B_TFULL = B_PVDONE + 1,
+                       B_TEMPTY = B_TFULL + kTileRing, NBAR = B_TEMPTY + kTileRing;
+  // tmem base (u32), abort flag (u32), then the ring of unit indices (kTileRing x s32)
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 8 + 4 * kTileRing + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(NQ == 2 ? (256 + 2 * D <= 512) : (256 + D <= 512), "tensor memory budget");
@@ -100,6 +103,9 @@ struct FwdParams {
   float* ws_o;      // [split tile][half][NQ][128 rows][D] partial O (fp32)
   float4* ws_ml;    // [split tile][half][NQ][128 rows] (m, l, l_rounded, 0)
   int* ws_cnt;      // [split tile][NQ][4 row groups] arrival counters (left at 0)
+  // Dynamic schedule (with a workspace): sched[0] hands out units beyond the
+  // first gridDim.x, sched[1] counts finished CTAs; the last CTA resets both.
+  int* sched;
 };
 
 struct Tile {
@@ -181,29 +187,38 @@ struct Ctx {
   uint32_t sbase;  // 1024-aligned shared-memory base (shared address space)
   uint32_t tmem;   // tensor-memory base address
   volatile uint32_t* abort_flag;
+  volatile int* ring;  // unit indices published by the TMA thread (dynamic schedule)
   __device__ uint32_t bar(int i, int off_bar) const { return sbase + off_bar + 8u * i; }
 };
 
 // Bounded wait on an mbarrier phase.  Returns false (and makes every other
-// wait of the CTA return false) when the time limit is reached.
+// wait of the CTA return false) when the time limit is reached.  A wait that
+// times out only stores a packed site word in the CTA's abort flag (first one
+// wins); publish_abort() turns it into the device status word at teardown.
+// This keeps each of the many inlined wait sites small.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity,
-                                      volatile uint32_t* abort_flag) {
+                                         volatile uint32_t* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+  while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1u;
-      if (atomicCAS(&g_status, 0u, static_cast<unsigned>(FA_ERR_DEVICE_TIMEOUT)) == 0u)
-        g_timeout_site = (static_cast<unsigned long long>(blockIdx.x) << 48) |
-                         (static_cast<unsigned long long>(threadIdx.x >> 5) << 40) |
-                         (static_cast<unsigned long long>(bar & 0xFFFFFu) << 8) | parity;
+      const uint32_t site = 0x80000000u | ((threadIdx.x >> 5) << 24) | ((bar & 0x3FFFFu) << 1) | parity;
+      atomicCAS(const_cast<uint32_t*>(abort_flag), 0u, site);
       return false;
     }
   }
+  return true;
+}
+
+// Thread 0 at teardown: record the CTA's timed-out wait (if any) in the device
+// status word and, for the first CTA to do so, its site.
+__device__ __forceinline__ void publish_abort(uint32_t flag) {
+  if (flag == 0u) return;
+  if (atomicCAS(&g_status, 0u, static_cast<unsigned>(FA_ERR_DEVICE_TIMEOUT)) == 0u)
+    g_timeout_site = (static_cast<unsigned long long>(blockIdx.x) << 48) |
+                     (static_cast<unsigned long long>((flag >> 24) & 0x3Fu) << 40) |
+                     (static_cast<unsigned long long>((flag >> 1) & 0x3FFFFu) << 8) | (flag & 1u);
 }
 
 // Wait that ignores the abort flag, with its own short limit (used only to
@@ -212,6 +227,45 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity))
     if (globaltimer_ns() - t0 > 100000000ull) return;
+}
+
+// Work units of a CTA.  Static schedule (p.sched == nullptr): the zig-zag
+// TileIter.  Dynamic schedule: the TMA thread takes unit blockIdx.x first, then
+// gridDim.x + atomicAdd(sched[0], 1) each time (heaviest units have the lowest
+// indices), and publishes every index -- or -1 at the end -- in a shared-memory
+// ring (t_full: written; t_empty: read by the MMA thread and every softmax warp,
+// 4 per query tile).
+template <int D, int NQ>
+__device__ __forceinline__ bool produce_unit(const Ctx& cx, const FwdParams& p, TileIter& it,
+                                             uint32_t& n, int& u) {
+  if (p.sched == nullptr) return it.next(u);
+  using G = Geometry<D, NQ>;
+  u = (n == 0) ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
+  const int k = n % kTileRing;
+  if (n >= (uint32_t)kTileRing &&
+      !wait_bar(cx.bar(G::B_TEMPTY + k, G::OFF_BAR), ((n / kTileRing) - 1) & 1u, cx.abort_flag))
+    return false;
+  const int pub = u < p.n_units ? u : -1;
+  cx.ring[k] = pub;
+  mbar_arrive(cx.bar(G::B_TFULL + k, G::OFF_BAR));  // release: the index is visible after the wait
+  ++n;
+  return pub >= 0;
+}
+// Consumer side; `lane` < 0 for the single MMA thread, else the softmax warp's lane.
+template <int D, int NQ>
+__device__ __forceinline__ bool consume_unit(const Ctx& cx, const FwdParams& p, TileIter& it,
+                                             uint32_t& n, int& u, int lane) {
+  if (p.sched == nullptr) return it.next(u);
+  using G = Geometry<D, NQ>;
+  const int k = n % kTileRing;
+  bool ok = wait_bar(cx.bar(G::B_TFULL + k, G::OFF_BAR), (n / kTileRing) & 1u, cx.abort_flag);
+  if (lane >= 0) ok = __all_sync(0xffffffffu, ok);
+  if (!ok) return false;
+  u = cx.ring[k];
+  ++n;
+  if (lane >= 0) __syncwarp();
+  if (lane <= 0) mbar_arrive(cx.bar(G::B_TEMPTY + k, G::OFF_BAR));
+  return u >= 0;
 }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b, bool bf16) {
@@ -265,8 +319,9 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
     return true;
   };
   TileIter it(p.n_units);
+  uint32_t n_units_seen = 0;
   int t;
-  while (ok && it.next(t)) {
+  while (ok && produce_unit<D, NQ>(cx, p, it, n_units_seen, t)) {
     const Tile T = get_tile<NQ>(p, t);
     // Q0, then K0 (the first S MMA of the tile needs only these), then Q1 -- each
     // Q tile waits only for the last S MMA that read its previous contents.
@@ -360,8 +415,9 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
   };
 
   TileIter it(p.n_units);
+  uint32_t n_units_seen = 0;
   int t;
-  while (it.next(t)) {
+  while (consume_unit<D, NQ>(cx, p, it, n_units_seen, t, -1)) {
     const Tile T = get_tile<NQ>(p, t);
     const int nb = T.nb;
     int kst;
@@ -580,8 +636,9 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   const int q = (NQ == 2) ? wg : 0;
 
   TileIter it(p.n_units);
+  uint32_t n_units_seen = 0;
   int t;
-  while (it.next(t)) {
+  while (consume_unit<D, NQ>(cx, p, it, n_units_seen, t, lane)) {
     const Tile T = get_tile<NQ>(p, t);
     const int nblk = T.nblk[q];
     if (nblk == 0) continue;
@@ -621,6 +678,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
         need = true;
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+      const float cs = masked ? 1.f : c;
       // bf16 only: also sum the rounded P that the PV product actually uses, and
       // normalise O by that sum -- the weights then sum to one exactly, which
       // removes the bf16 rounding error of the dominant weight(s) from O.
@@ -635,15 +693,12 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
         for (int u = 0; u < 16; ++u) {
           const int i = g * 16 + u;
           const F2 sv = f2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+          // masked blocks hold already scaled scores (cs = 1); masked keys are -inf:
+          // 0 from MUFU, ~2^-125 from the FMA-pipe exp2 (negligible against l >= 1)
+          const F2 x = ffma2(sv, f2(cs, cs), f2(neg_m, neg_m));
           F2 pr;
-          if (masked) {
-            const F2 x = fadd2(sv, f2(neg_m, neg_m));
-            pr = f2(ex2(x.x), ex2(x.y));
-          } else {
-            const F2 x = ffma2(sv, f2(c, c), f2(neg_m, neg_m));
-            if ((kEmuPairs >> (i & 7)) & 1u) pr = exp2_fma2(x);  // FMA pipe
-            else pr = f2(ex2(x.x), ex2(x.y));                   // MUFU
-          }
+          if ((kEmuPairs >> (i & 7)) & 1u) pr = exp2_fma2(x);  // FMA pipe
+          else pr = f2(ex2(x.x), ex2(x.y));                   // MUFU
           acc[u & 3] = fadd2(acc[u & 3], pr);
           pk[u] = pack2(pr.x, pr.y, BF16);
           if (BF16) accr[u & 1] = fadd2(accr[u & 1], unpack_bf16x2(pk[u]));
@@ -732,6 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Ctx cx;
   cx.sbase = sbase;
   cx.abort_flag = misc + 1;
+  cx.ring = reinterpret_cast<volatile int*>(misc + 2);
   if (threadIdx.x == 0) {
     auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
     for (int q = 0; q < 2; ++q) {  // one pair per query tile: the next tile's Q0 loads early
@@ -749,6 +805,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(B(G::B_OEMPTY + q), 4);
     }
     mbar_init(B(G::B_PVDONE), 1);
+    for (int k = 0; k < kTileRing; ++k) {
+      mbar_init(B(G::B_TFULL + k), 1);
+      mbar_init(B(G::B_TEMPTY + k), 1 + 4 * NQ);  // the MMA thread and the softmax warps
+    }
     misc[1] = 0u;
     fence_mbar_init();
   }
@@ -778,6 +838,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) publish_abort(*cx.abort_flag);
+  if (threadIdx.x == 0 && p.sched != nullptr) {  // the last CTA to finish resets the schedule
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      p.sched[0] = 0;
+      p.sched[1] = 0;
+      __threadfence();
+    }
+  }
   if (warp == 8) {
     if (*cx.abort_flag) {  // abort path: give issued MMAs time to retire before freeing TMEM
       const uint64_t t0 = globaltimer_ns();
@@ -785,6 +854,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     tmem_dealloc(cx.tmem, G::TMEM_COLS);
+  }
+}
+
+// Runs the kernels' bounded wait on an mbarrier that nothing arrives on: after the
+// time limit it records FA_ERR_DEVICE_TIMEOUT and the site, and returns (tests the
+// failure detection without hanging or faulting the device).
+__global__ void wait_timeout_probe_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    wait_bar(smem_u32(&bar), 0u, &abort_flag);
+    publish_abort(abort_flag);
   }
 }
 
@@ -866,8 +953,8 @@ struct WsLayout {
 WsLayout ws_layout(int D, int NQ, int max_split) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   WsLayout L;
-  L.cnt_off = 0;
-  L.ml_off = up(static_cast<size_t>(kMaxSplit) * 2 * 4 * sizeof(int));
+  L.cnt_off = 0;  // split counters, then the two schedule counters
+  L.ml_off = up(static_cast<size_t>(kMaxSplit) * 2 * 4 * sizeof(int) + 2 * sizeof(int));
   L.o_off = L.ml_off + up(static_cast<size_t>(max_split) * 2 * NQ * 128 * sizeof(float4));
   L.total = L.o_off + up(static_cast<size_t>(max_split) * 2 * NQ * 128 * D * sizeof(float));
   return L;
@@ -944,6 +1031,13 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.ws_ml = nullptr;
     p.ws_cnt = nullptr;
   }
+  // Dynamic schedule for non-causal launches with a workspace in which a CTA gets
+  // several units (for causal ones the static heavy-first zig-zag measured as
+  // fast or faster).
+  p.sched = nullptr;
+  if (ws != nullptr && !causal && ws_bytes >= ws_layout(D, NQ, 0).ml_off &&
+      p.n_tiles + n_split > grid)
+    p.sched = reinterpret_cast<int*>(static_cast<char*>(ws) + kMaxSplit * 2 * 4 * sizeof(int));
   p.n_whole = p.n_tiles - n_split;
   p.n_units = p.n_tiles + n_split;
   fa::fa_fwd_kernel<D, NQ, BF16><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(tq, tk, tv, p);
@@ -1119,6 +1213,11 @@ int fa_device_status(int reset) {
       return -1;
   }
   return static_cast<int>(v);
+}
+
+int fa_debug_wait_timeout(void* stream) {
+  fa::wait_timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 int fa_debug_exp2_fma(const float* x, float* y, int n, void* stream) {
