@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gate", action="store_true", help="skip the N=4096/8192 gate configs")
+    ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurement")
     return ap.parse_args()
 
 
@@ -341,6 +342,35 @@ def main():
             del gq, gk, gv, go, gl
         assert fa.device_status(reset=True) == 0
 
+    # ---- KV-cache decode (one query row per head, 32K-token cache, GQA 4): HBM-bound
+    decode = {}
+    if not args.no_decode:
+        from fa_inputs import Workload
+        wd = Workload("decode B8 Hq32 Hkv8 Nq1 Nk32768 D128 fp16", 8, 32, 8, 1, 32768, 128, "fp16",
+                      False, seed=0)
+        dq, dk, dv = (x.to(dev) for x in make_qkv(wd))
+        do_, dl_ = torch.empty_like(dq), torch.empty(dq.shape[:3], dtype=torch.float32, device=dev)
+        ts = []
+        for i in range(13):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fa.fa_fwd(dq, dk, dv, o=do_, lse=dl_, scale=wd.softmax_scale, stream=sptr)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        ms = statistics.median(ts)
+        nbytes = wd.io_bytes()
+        hbm = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"] \
+            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 6650.0
+        decode = {"workload": wd.name, "ms": round(ms, 4), "bytes": nbytes,
+                  "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                  "frac_of_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 3),
+                  "tflops": round(wd.flops() / (ms * 1e-3) / 1e12, 2)}
+        del dq, dk, dv, do_, dl_
+        assert fa.device_status(reset=True) == 0
+
     peak, peak_sus, peak_kind = peaks()
     launch_ms = total_ms / world / (K * len(ws)) if world > 1 else total_ms / (K * len(ws))
     achieved = (flops_step / len(ws)) / (launch_ms * 1e-3) / 1e12
@@ -368,6 +398,7 @@ def main():
         "gpu_launches": K * len(ws),
         "clocks": clk.summary(),
         "gate_d128": gate,
+        "decode": decode,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle

@@ -150,6 +150,42 @@ def test_split_tail(cuda_dev, w):
         fa.set_max_ctas(prev)
 
 
+# KV-cache decode shapes: a few query rows per head against a long key range.
+# With Hq > Hkv and Hq/Hkv * Nq <= 128 one tile packs all query heads of a key/value
+# head; with a workspace every tile's key range is also split across CTAs (split-K)
+# when there are fewer tiles than SMs.
+DECODE = [
+    Workload("decode GQA4 Nq1 D128 fp16", 4, 32, 8, 1, 8192, 128, "fp16", False, seed=51),
+    Workload("decode GQA4 Nq1 D128 bf16 ragged Nk", 2, 16, 4, 1, 5000, 128, "bf16", False, seed=52),
+    Workload("decode GQA8 Nq4 D64 fp16", 2, 32, 4, 4, 4096, 64, "fp16", False, seed=53),
+    Workload("decode MQA Nq2 D256 bf16", 2, 16, 1, 2, 3000, 256, "bf16", False, seed=54),
+    Workload("decode GQA8 Nq16 D128 fp16 (128 rows)", 1, 16, 2, 16, 4096, 128, "fp16", False, seed=55),
+    Workload("decode GQA8 Nq17 D128 fp16 (not packed)", 1, 8, 1, 17, 2048, 128, "fp16", False, seed=56),
+    Workload("decode MHA Nq1 D128 fp16", 2, 16, 16, 1, 8192, 128, "fp16", False, seed=57),
+    Workload("decode GQA4 Nq3 D128 fp16 short Nk", 1, 8, 2, 3, 300, 128, "fp16", False, seed=58),
+]
+
+
+@pytest.mark.parametrize("use_ws", [True, False])
+@pytest.mark.parametrize("w", DECODE, ids=lambda w: w.name)
+def test_decode_shapes(cuda_dev, w, use_ws):
+    q, k, v = make_qkv(w)
+    o, lse = fa.fa_fwd(q.to(cuda_dev), k.to(cuda_dev), v.to(cuda_dev), scale=w.softmax_scale,
+                       use_workspace=use_ws)
+    torch.cuda.synchronize()
+    assert fa.device_status(reset=True) == 0
+    ref_o, ref_l = oracle.attention(q, k, v, w.softmax_scale, False)
+    do = np.abs(o.float().cpu().numpy() - ref_o).max()
+    dl = np.abs(lse.cpu().numpy() - ref_l).max()
+    report = os.environ.get("FA_PARITY_REPORT")
+    if report:
+        with open(report, "a") as f:
+            f.write(json.dumps({"case": w.name + (" ws" if use_ws else " nows"), "dtype": w.dtype,
+                                "rows": "all", "max_abs_dO": float(do), "max_abs_dLSE": float(dl)}) + "\n")
+    assert do <= TOL[w.dtype][0], f"{w.name}: max|dO| = {do:.3e}"
+    assert dl <= TOL[w.dtype][1], f"{w.name}: max|dLSE| = {dl:.3e}"
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.5])
 def test_scale_values(cuda_dev, scale):
     w = Workload("scale", 1, 2, 2, 300, 300, 128, "fp16", True, seed=3, scale=scale)

@@ -95,13 +95,17 @@ struct FwdParams {
   int qt_per_head;  // work tiles per (batch, head)
   int n_tiles;
   int nkb;  // key blocks: ceil(Nk / kBN)
-  // Split tail: tiles [n_whole, n_tiles) are each processed as two units, one per
-  // half of the key blocks; n_units = n_whole + 2 * (n_tiles - n_whole).  Each half
-  // leaves its un-normalised partial in the workspace and the second one to finish
-  // a row group merges (see merge_epilogue).
-  int n_whole, n_units;
-  float* ws_o;      // [split tile][half][NQ][128 rows][D] partial O (fp32)
-  float4* ws_ml;    // [split tile][half][NQ][128 rows] (m, l, l_rounded, 0)
+  // Split tiles: tiles [n_whole, n_tiles) are each processed as nsplit units, one
+  // per part of the key blocks; n_units = n_whole + nsplit * (n_tiles - n_whole).
+  // Each part leaves its un-normalised partial in the workspace and the last one
+  // to finish a row group merges (see merge_epilogue).
+  int n_whole, n_units, nsplit;
+  int ws_rows;      // partial rows stored per split unit (rows of the tile that exist)
+  // GQA packing (pack_g > 1): a work tile holds all pack_g query heads of one
+  // key/value head, row r = (head r / Nq, query r % Nq), pack_g * Nq <= 128.
+  int pack_g;
+  float* ws_o;      // [split tile][part][ws_rows][D] partial O (fp32)
+  float4* ws_ml;    // [split tile][part][ws_rows] (m, l, l_rounded, 0)
   int* ws_cnt;      // [split tile][NQ][4 row groups] arrival counters (left at 0)
   // Dynamic schedule (with a workspace): sched[0] hands out units beyond the
   // first gridDim.x, sched[1] counts finished CTAs; the last CTA resets both.
@@ -116,7 +120,7 @@ struct Tile {
   int nb;
   int jb;     // first key block of this unit
   int slot;   // split-tile index, or -1 for a whole tile
-  int half;   // which key half of a split tile
+  int half;   // which key part of a split tile
 };
 
 template <int NQ>
@@ -125,28 +129,35 @@ __device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
   int t = u;
   T.slot = -1;
   T.half = 0;
-  if (u >= p.n_whole) {  // half of a split tile
+  if (u >= p.n_whole) {  // one key part of a split tile
     const int v = u - p.n_whole;
-    t = p.n_whole + (v >> 1);
-    T.slot = v >> 1;
-    T.half = v & 1;
+    T.slot = v / p.nsplit;
+    T.half = v - T.slot * p.nsplit;
+    t = p.n_whole + T.slot;
   }
-  const int BH = p.B * p.Hq;
   int qt;
-  if (p.causal) {  // heaviest (last) query tiles first
-    qt = p.qt_per_head - 1 - t / BH;
-    T.bh = t % BH;
-  } else {  // tiles of one head adjacent: K/V of a head stay hot in L2
-    T.bh = t / p.qt_per_head;
-    qt = t % p.qt_per_head;
+  if (p.pack_g > 1) {  // one tile per (batch, key/value head)
+    qt = 0;
+    T.kvz = t;
+    T.bh = (t / p.Hkv) * p.Hq + (t % p.Hkv) * p.pack_g;  // first query head of the group
+  } else {
+    const int BH = p.B * p.Hq;
+    if (p.causal) {  // heaviest (last) query tiles first
+      qt = p.qt_per_head - 1 - t / BH;
+      T.bh = t % BH;
+    } else {  // tiles of one head adjacent: K/V of a head stay hot in L2
+      T.bh = t / p.qt_per_head;
+      qt = t % p.qt_per_head;
+    }
+    const int b = T.bh / p.Hq, hq = T.bh % p.Hq;
+    T.kvz = b * p.Hkv + hq / p.group;
   }
   T.row0 = qt * NQ * kBM;
-  const int b = T.bh / p.Hq, hq = T.bh % p.Hq;
-  T.kvz = b * p.Hkv + hq / p.group;
+  const int rows = p.pack_g > 1 ? p.pack_g * p.Nq : p.Nq;  // rows of the (packed) tile space
   int kb0 = 0, kb1 = p.nkb;  // split units: non-causal only (the host guarantees it)
   if (T.slot >= 0) {
-    kb0 = T.half ? p.nkb / 2 : 0;
-    kb1 = T.half ? p.nkb : p.nkb / 2;
+    kb0 = (T.half * p.nkb) / p.nsplit;
+    kb1 = ((T.half + 1) * p.nkb) / p.nsplit;
   }
   T.jb = kb0;
   T.nb = 0;
@@ -154,9 +165,9 @@ __device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
   for (int q = 0; q < 2; ++q) {
     const int rf = T.row0 + q * kBM;
     int n = 0;
-    if (q < NQ && rf < p.Nq) {
+    if (q < NQ && rf < rows) {
       n = kb1 - kb0;
-      if (p.causal) {
+      if (p.causal && p.pack_g <= 1) {
         const int rl = min(rf + kBM - 1, p.Nq - 1);
         n = min(p.nkb, rl / kBN + 1);
       }
@@ -165,6 +176,30 @@ __device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
     T.nb = max(T.nb, n);
   }
   return T;
+}
+
+// Where row r (0..127) of query tile q of a work tile goes: its flat output row
+// ((b * Hq + hq) * Nq + position), its query position (for the causal mask) and
+// whether it exists.
+struct RowInfo {
+  size_t out_row;
+  int pos;
+  bool live;
+};
+__device__ __forceinline__ RowInfo row_info(const FwdParams& p, const Tile& T, int q, int r) {
+  RowInfo ri;
+  const int tr = T.row0 + q * kBM + r;  // row in the tile space
+  if (p.pack_g > 1) {
+    const int h = tr / p.Nq;
+    ri.pos = tr - h * p.Nq;
+    ri.live = h < p.pack_g;
+    ri.out_row = (static_cast<size_t>(T.bh) + (ri.live ? h : 0)) * p.Nq + ri.pos;
+  } else {
+    ri.pos = tr;
+    ri.live = tr < p.Nq;
+    ri.out_row = static_cast<size_t>(T.bh) * p.Nq + (ri.live ? tr : 0);
+  }
+  return ri;
 }
 
 // Work tiles of this CTA, in a zig-zag over rounds of gridDim.x tiles so that
@@ -281,9 +316,10 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, bool bf16) {
 // ---------------------------------------------------------------- TMA producer
 template <int D, int NQ>
 __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, const CUtensorMap* tq,
-                                          const CUtensorMap* tk, const CUtensorMap* tv) {
+                                          const CUtensorMap* tq4, const CUtensorMap* tk,
+                                          const CUtensorMap* tv) {
   using G = Geometry<D, NQ>;
-  prefetch_tmap(tq);
+  prefetch_tmap(p.pack_g > 1 ? tq4 : tq);
   prefetch_tmap(tk);
   prefetch_tmap(tv);
   const uint64_t pol_kv = policy_evict_last();
@@ -295,11 +331,19 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
       if (!wait_bar(cx.bar(G::B_QEMPTY + q, G::OFF_BAR), qe_phase[q], cx.abort_flag)) return false;
       qe_phase[q] ^= 1u;
     }
-    mbar_arrive_expect_tx(cx.bar(G::B_QFULL + q, G::OFF_BAR), G::Q_BYTES);
+    if (p.pack_g > 1) {  // all pack_g heads of the group: one box of pack_g * Nq rows
+      mbar_arrive_expect_tx(cx.bar(G::B_QFULL + q, G::OFF_BAR), p.pack_g * p.Nq * 128 * G::DCH);
 #pragma unroll
-    for (int c = 0; c < G::DCH; ++c)
-      tma_load_3d(cx.sbase + G::OFF_Q + q * G::Q_BYTES + c * G::CHUNK_Q, tq,
-                  cx.bar(G::B_QFULL + q, G::OFF_BAR), c * 64, T.row0 + q * kBM, T.bh, pol_q);
+      for (int c = 0; c < G::DCH; ++c)
+        tma_load_3d(cx.sbase + G::OFF_Q + q * G::Q_BYTES + c * G::CHUNK_Q, tq4,
+                    cx.bar(G::B_QFULL + q, G::OFF_BAR), c * 64, 0, T.kvz, pol_q);
+    } else {
+      mbar_arrive_expect_tx(cx.bar(G::B_QFULL + q, G::OFF_BAR), G::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < G::DCH; ++c)
+        tma_load_3d(cx.sbase + G::OFF_Q + q * G::Q_BYTES + c * G::CHUNK_Q, tq,
+                    cx.bar(G::B_QFULL + q, G::OFF_BAR), c * 64, T.row0 + q * kBM, T.bh, pol_q);
+    }
     ++q_issued[q];
     return true;
   };
@@ -544,31 +588,35 @@ __device__ __forceinline__ F2 unpack_bf16x2(uint32_t w) {
   return F2{__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)};
 }
 
-// Epilogue of one half of a split tile, for the 32 rows of this warp.  Each half
-// stores its un-normalised O row (fp32), its stabiliser m and sums l, l_r; then
-// the warp bumps the counter of its row group.  The warp that arrives second
-// reads the other half's partial and writes the merged, normalised row:
-//   M = max(m0, m1),  a_h = 2^(m_h - M),  L = a0 l0 + a1 l1,
-//   O = (a0 O0 + a1 O1) / L,  LSE = (M + log2 L) ln 2,
-// and resets the counter to 0 for the next call.  Neither half waits for the
-// other, so no cross-CTA wait exists.
+// Epilogue of one key part of a split tile, for the 32 rows of this warp.  Each
+// part stores its un-normalised O row (fp32), its stabiliser m and sums l, l_r;
+// then the warp bumps the counter of its row group.  The warp that arrives last
+// (the nsplit-th) reads all parts, in part order, and writes the merged row:
+//   M = max_s m_s,  a_s = 2^(m_s - M),  L = sum_s a_s l_s,
+//   O = sum_s a_s O_s / L,  LSE = (M + log2 L) ln 2,
+// then resets the counter to 0 for the next call.  No part waits for another,
+// so no cross-CTA wait exists, and the result does not depend on which part
+// finished last.
 template <int D, int NQ, bool BF16>
 __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T, int q, int sub,
-                                               int lane, int row, bool live, uint32_t ocol,
+                                               int lane, const RowInfo& ri, uint32_t ocol,
                                                float m, float l, float l_r) {
-  const int r = sub * 32 + lane;
-  const size_t mine = ((static_cast<size_t>(T.slot) * 2 + T.half) * NQ + q) * kBM + r;
-  const size_t theirs = ((static_cast<size_t>(T.slot) * 2 + (T.half ^ 1)) * NQ + q) * kBM + r;
-  p.ws_ml[mine] = make_float4(m, l, l_r, 0.f);
-  float4* my_o = reinterpret_cast<float4*>(p.ws_o + mine * D);
+  const int rr = q * kBM + sub * 32 + lane;  // row of the work tile
+  const bool stored = rr < p.ws_rows;         // rows beyond ws_rows do not exist
+  const size_t base = static_cast<size_t>(T.slot) * p.nsplit;
+  auto idx = [&](int part) { return (base + part) * p.ws_rows + rr; };
+  if (stored) p.ws_ml[idx(T.half)] = make_float4(m, l, l_r, 0.f);
+  float4* my_o = reinterpret_cast<float4*>(p.ws_o + idx(stored ? T.half : 0) * D);
 #pragma unroll 1
   for (int c0 = 0; c0 < D; c0 += 32) {
     uint32_t orr[32];
-    tmem_ld_x32(ocol + c0, orr);
+    tmem_ld_x32(ocol + c0, orr);  // warp-collective: every lane takes part
+    if (stored) {
 #pragma unroll
-    for (int x = 0; x < 8; ++x)
-      my_o[c0 / 4 + x] = make_float4(__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
-                                     __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3]));
+      for (int x = 0; x < 8; ++x)
+        my_o[c0 / 4 + x] = make_float4(__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
+                                       __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3]));
+    }
   }
   __threadfence();
   __syncwarp();
@@ -576,49 +624,39 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
   int old = 0;
   if (lane == 0) old = atomicAdd(cnt, 1);
   old = __shfl_sync(0xffffffffu, old, 0);
-  if (old != 1) return;  // the other half merges these rows
+  if (old != p.nsplit - 1) return;  // a later part merges these rows
   __threadfence();
-  // Combine in a fixed order (half 0, then half 1), so the result does not depend
-  // on which half happens to finish second.
-  const float4 o_ml = __ldcg(p.ws_ml + theirs);
-  const bool first = T.half == 0;
-  const float m0 = first ? m : o_ml.x, m1 = first ? o_ml.x : m;
-  const float l0 = first ? l : o_ml.y, l1 = first ? o_ml.y : l;
-  const float r0 = first ? l_r : o_ml.z, r1 = first ? o_ml.z : l_r;
-  const float M = fmaxf(m0, m1);
-  const float a0 = ex2(m0 - M), a1 = ex2(m1 - M);
-  const float L = fmaf(a0, l0, a1 * l1), Lr = fmaf(a0, r0, a1 * r1);
-  const float inv = 1.f / (BF16 ? Lr : L);
-  const float s0 = a0 * inv, s1 = a1 * inv;
-  const float4* th_o = reinterpret_cast<const float4*>(p.ws_o + theirs * D);
-  uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
-                   (static_cast<size_t>(T.bh) * p.Nq + (live ? row : 0)) * D;
+  if (stored) {
+    float M = -INFINITY;
+    for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, __ldcg(p.ws_ml + idx(s)).x);
+    float L = 0.f, Lr = 0.f;
+    for (int s = 0; s < p.nsplit; ++s) {
+      const float4 ml = __ldcg(p.ws_ml + idx(s));
+      const float a = ex2(ml.x - M);
+      L = fmaf(a, ml.y, L);
+      Lr = fmaf(a, ml.z, Lr);
+    }
+    const float inv = 1.f / (BF16 ? Lr : L);
+    uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
 #pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    uint32_t orr[32];
-    tmem_ld_x32(ocol + c0, orr);
-    uint32_t w[16];
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const float4 t4 = __ldcg(th_o + c0 / 4 + x);
-      const float u[4] = {__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
-                          __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3])};
-      const float v[4] = {t4.x, t4.y, t4.z, t4.w};
-      float z[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) z[e] = first ? fmaf(u[e], s0, v[e] * s1) : fmaf(v[e], s0, u[e] * s1);
-      w[2 * x] = pack2(z[0], z[1], BF16);
-      w[2 * x + 1] = pack2(z[2], z[3], BF16);
+    for (int c0 = 0; c0 < D; c0 += 8) {
+      float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < p.nsplit; ++s) {
+        const float sc = ex2(__ldcg(p.ws_ml + idx(s)).x - M) * inv;
+        const float4* po = reinterpret_cast<const float4*>(p.ws_o + idx(s) * D + c0);
+        const float4 u0 = __ldcg(po), u1 = __ldcg(po + 1);
+        z[0] = fmaf(u0.x, sc, z[0]); z[1] = fmaf(u0.y, sc, z[1]);
+        z[2] = fmaf(u0.z, sc, z[2]); z[3] = fmaf(u0.w, sc, z[3]);
+        z[4] = fmaf(u1.x, sc, z[4]); z[5] = fmaf(u1.y, sc, z[5]);
+        z[6] = fmaf(u1.z, sc, z[6]); z[7] = fmaf(u1.w, sc, z[7]);
+      }
+      if (ri.live)
+        *reinterpret_cast<uint4*>(orow + c0) =
+            make_uint4(pack2(z[0], z[1], BF16), pack2(z[2], z[3], BF16), pack2(z[4], z[5], BF16),
+                       pack2(z[6], z[7], BF16));
     }
-    if (live) {
-      uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-        dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
-    }
+    if (p.lse != nullptr && ri.live) p.lse[ri.out_row] = (M + log2f(L)) * kLn2;
   }
-  if (p.lse != nullptr && live)
-    p.lse[static_cast<size_t>(T.bh) * p.Nq + row] = (M + log2f(L)) * kLn2;
   __syncwarp();
   if (lane == 0) *cnt = 0;
 }
@@ -643,6 +681,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     const int nblk = T.nblk[q];
     if (nblk == 0) continue;
     const int rfirst = T.row0 + q * kBM;
+    // query position of this thread's row (causal mask; packing is non-causal only)
     const int row = rfirst + sub * 32 + lane;
     float m_used = -INFINITY, l = 0.f, l_r = 0.f;  // l: exact sum (LSE); l_r: rounded-P sum
     for (int j = 0; j < nblk; ++j) {
@@ -739,14 +778,14 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     if (!__all_sync(0xffffffffu, ok)) return;
     of_phase ^= 1u;
     tc_fence_after();
-    const bool live = row < p.Nq;
+    const RowInfo ri = row_info(p, T, q, sub * 32 + lane);
+    const bool live = ri.live;
     const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
     if (T.slot >= 0) {
-      merge_epilogue<D, NQ, BF16>(p, T, q, sub, lane, row, live, tm + 256 + q * D, m_sub, l, l_r);
+      merge_epilogue<D, NQ, BF16>(p, T, q, sub, lane, ri, tm + 256 + q * D, m_sub, l, l_r);
     } else {
       const float inv_l = 1.f / (BF16 ? l_r : l);
-      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
-                       (static_cast<size_t>(T.bh) * p.Nq + (live ? row : 0)) * D;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t orr[32];
@@ -764,7 +803,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
         }
       }
       if (p.lse != nullptr && live)
-        p.lse[static_cast<size_t>(T.bh) * p.Nq + row] = (m_sub + log2f(l)) * kLn2;
+        p.lse[ri.out_row] = (m_sub + log2f(l)) * kLn2;
     }
     tc_fence_before();
     __syncwarp();
@@ -774,8 +813,9 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
 
 template <int D, int NQ, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q4,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const FwdParams p) {
   using G = Geometry<D, NQ>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -822,17 +862,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   cx.tmem = misc[0];
 
   // Registers: 168 per thread at launch (384 threads, one CTA per SM); the two
-  // softmax warpgroups take 208, the MMA / TMA / idle warpgroup keeps 88
-  // (2 x 128 x 208 + 128 x 88 = 64512 = 384 x 168).  The wait helpers are
-  // inlined: ptxas cannot allocate a call inside a region resized this way.
-  if (warp < 8) setmaxnreg_inc_208();
-  else setmaxnreg_dec_88();
+  // softmax warpgroups take kSoftmaxRegs, the MMA / TMA / idle warpgroup keeps
+  // the rest (2 x 128 x 208 + 128 x 88 = 2 x 128 x 200 + 128 x 104 = 64512 =
+  // 384 x 168); bf16 needs the larger softmax share (it also sums rounded P).
+  // The wait helpers are inlined: ptxas cannot allocate a call inside a region
+  // resized this way.
+  constexpr int kSoftmaxRegs = BF16 ? 208 : 200;
+  constexpr int kOtherRegs = (384 * 168 - 256 * kSoftmaxRegs) / 128;
+  if (warp < 8) setmaxnreg_inc<kSoftmaxRegs>();
+  else setmaxnreg_dec<kOtherRegs>();
   if (warp < 8) {
     if (NQ == 2 || warp < 4) role_softmax<D, NQ, BF16>(cx, p, warp >> 2, warp & 3, lane);
   } else if (warp == 8) {
     if (lane == 0) role_mma<D, NQ, BF16>(cx, p);
   } else if (warp == 9) {
-    if (lane == 0) role_load<D, NQ>(cx, p, &tm_q, &tm_k, &tm_v);
+    if (lane == 0) role_load<D, NQ>(cx, p, &tm_q, &tm_q4, &tm_k, &tm_v);
   }
   __syncwarp();
   tc_fence_before();
@@ -947,16 +991,20 @@ std::atomic<int> g_max_ctas{0};
 // 256 bytes.
 constexpr int kMaxSplit = 1024;  // >= half the SMs of any device
 constexpr int kMinSplitBlocks = 24;
+constexpr int kMinPartBlocks = 4;  // key blocks per part when a launch splits every tile
+constexpr int kMaxParts = 32;
 struct WsLayout {
   size_t cnt_off, ml_off, o_off, total;
 };
-WsLayout ws_layout(int D, int NQ, int max_split) {
+// Partial results: n_split tiles x nsplit parts x rows per tile.
+WsLayout ws_layout(int D, int rows, int n_split, int nsplit) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   WsLayout L;
   L.cnt_off = 0;  // split counters, then the two schedule counters
   L.ml_off = up(static_cast<size_t>(kMaxSplit) * 2 * 4 * sizeof(int) + 2 * sizeof(int));
-  L.o_off = L.ml_off + up(static_cast<size_t>(max_split) * 2 * NQ * 128 * sizeof(float4));
-  L.total = L.o_off + up(static_cast<size_t>(max_split) * 2 * NQ * 128 * D * sizeof(float));
+  const size_t units = static_cast<size_t>(n_split) * nsplit * rows;
+  L.o_off = L.ml_off + up(units * sizeof(float4));
+  L.total = L.o_off + up(units * D * sizeof(float));
   return L;
 }
 
@@ -982,11 +1030,21 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
       attr_done[dev] = true;
     }
   }
-  CUtensorMap tq, tk, tv;
+  // GQA packing: when a key/value head's query heads fit one 128-row tile
+  // together (decode-like shapes), one tile holds all of them.
+  const int g = Hq / Hkv;
+  const bool pack = g > 1 && !causal && g * Nq <= fa::kBM;
+  CUtensorMap tq, tq4, tk, tv;
   if (!make_map(&tq, q, D, Nq, (long long)B * Hq, fa::kBM, BF16) ||
       !make_map(&tk, k, D, Nk, (long long)B * Hkv, fa::kBN, BF16) ||
       !make_map(&tv, v, D, Nk, (long long)B * Hkv, fa::kBN, BF16))
     return FA_ERR_DRIVER;
+  if (pack) {  // q viewed as [B*Hkv][g*Nq][D]: a group's query rows are contiguous
+    if (!make_map(&tq4, q, D, (long long)g * Nq, (long long)B * Hkv, g * Nq, BF16))
+      return FA_ERR_DRIVER;
+  } else {
+    tq4 = tq;
+  }
   fa::FwdParams p;
   p.o = o;
   p.lse = lse;
@@ -995,31 +1053,55 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.Hkv = Hkv;
   p.Nq = Nq;
   p.Nk = Nk;
-  p.group = Hq / Hkv;
+  p.group = g;
   p.causal = causal ? 1 : 0;
   p.c = scale * 1.4426950408889634f;
-  p.qt_per_head = (Nq + NQ * fa::kBM - 1) / (NQ * fa::kBM);
-  p.n_tiles = B * Hq * p.qt_per_head;
+  p.pack_g = pack ? g : 1;
+  p.qt_per_head = pack ? 1 : (Nq + NQ * fa::kBM - 1) / (NQ * fa::kBM);
+  p.n_tiles = pack ? B * Hkv : B * Hq * p.qt_per_head;
   p.nkb = (Nk + fa::kBN - 1) / fa::kBN;
   int ctas = g_dev[dev].sms;
   const int cap = g_max_ctas.load();
   if (cap > 0 && cap < ctas) ctas = cap;
-  const int grid = p.n_tiles < ctas ? p.n_tiles : ctas;
-  // Split tail: if the last round of tiles would keep at most half of the CTAs
-  // busy, give each of those tiles to two CTAs, one per half of the key blocks.
-  // Below kMinSplitBlocks key blocks the halves are too short to pay for writing
-  // and re-reading the fp32 partials (measured on the LLaMA-7B layer shape).
-  int n_split = 0;
-  const int rem = p.n_tiles % grid;
-  if (ws != nullptr && !causal && p.nkb >= kMinSplitBlocks && p.n_tiles > grid && rem > 0 &&
-      2 * rem <= grid && rem <= kMaxSplit) {
-    const WsLayout L = ws_layout(D, NQ, rem);
-    if (ws_bytes < L.total && mode == Scratch::kStatic) return FA_ERR_SCRATCH_TOO_SMALL;
-    if (ws_bytes >= L.total) {
+  // rows of a work tile that exist (partials are stored for these only)
+  p.ws_rows = pack ? g * Nq : (p.qt_per_head == 1 ? (Nq < NQ * fa::kBM ? Nq : NQ * fa::kBM)
+                                                   : NQ * fa::kBM);
+  int n_split = 0, nsplit = 1;
+  if (ws != nullptr && !causal) {
+    if (p.n_tiles < ctas && p.nkb >= 2 * kMinPartBlocks && p.n_tiles <= kMaxSplit) {
+      // Split-K: fewer tiles than SMs (decode-like shapes) -- every tile is cut
+      // into nsplit parts of the key blocks so that the units fill the device.
+      nsplit = (ctas + p.n_tiles - 1) / p.n_tiles;
+      if (nsplit > p.nkb / kMinPartBlocks) nsplit = p.nkb / kMinPartBlocks;
+      if (nsplit > kMaxParts) nsplit = kMaxParts;
+      while (nsplit >= 2 && ws_layout(D, p.ws_rows, p.n_tiles, nsplit).total > ws_bytes) --nsplit;
+      if (nsplit >= 2) n_split = p.n_tiles;
+      else nsplit = 1;
+    } else {
+      // Split tail: if the last round of tiles would keep at most half of the
+      // CTAs busy, give each of those tiles to two CTAs, one per half of the key
+      // blocks.  Below kMinSplitBlocks key blocks the halves are too short to pay
+      // for writing and re-reading the fp32 partials (measured on the LLaMA-7B
+      // layer shape).
+      const int grid0 = p.n_tiles < ctas ? p.n_tiles : ctas;
+      const int rem = p.n_tiles % grid0;
+      if (p.nkb >= kMinSplitBlocks && p.n_tiles > grid0 && rem > 0 && 2 * rem <= grid0 &&
+          rem <= kMaxSplit) {
+        n_split = rem;
+        nsplit = 2;
+      }
+    }
+  }
+  if (n_split > 0) {
+    const WsLayout L = ws_layout(D, p.ws_rows, n_split, nsplit);
+    if (ws_bytes < L.total) {
+      if (mode == Scratch::kStatic) return FA_ERR_SCRATCH_TOO_SMALL;
+      n_split = 0;
+      nsplit = 1;
+    } else {
       if (mode == Scratch::kStatic &&
           cudaMemsetAsync(ws, 0, L.ml_off, stream) != cudaSuccess)  // the counters start at zero
         return FA_ERR_LAUNCH;
-      n_split = rem;
       char* base = static_cast<char*>(ws);
       p.ws_o = reinterpret_cast<float*>(base + L.o_off);
       p.ws_ml = reinterpret_cast<float4*>(base + L.ml_off);
@@ -1031,16 +1113,17 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.ws_ml = nullptr;
     p.ws_cnt = nullptr;
   }
+  p.nsplit = nsplit;
+  p.n_whole = p.n_tiles - n_split;
+  p.n_units = p.n_whole + nsplit * n_split;
+  const int grid = p.n_units < ctas ? p.n_units : ctas;
   // Dynamic schedule for non-causal launches with a workspace in which a CTA gets
   // several units (for causal ones the static heavy-first zig-zag measured as
   // fast or faster).
   p.sched = nullptr;
-  if (ws != nullptr && !causal && ws_bytes >= ws_layout(D, NQ, 0).ml_off &&
-      p.n_tiles + n_split > grid)
+  if (ws != nullptr && !causal && ws_bytes >= ws_layout(D, 0, 0, 0).ml_off && p.n_units > grid)
     p.sched = reinterpret_cast<int*>(static_cast<char*>(ws) + kMaxSplit * 2 * 4 * sizeof(int));
-  p.n_whole = p.n_tiles - n_split;
-  p.n_units = p.n_tiles + n_split;
-  fa::fa_fwd_kernel<D, NQ, BF16><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  fa::fa_fwd_kernel<D, NQ, BF16><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(tq, tq4, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -1144,7 +1227,7 @@ size_t fa_fwd_workspace_size(int D) {
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
     return 0;
-  return ws_layout(D, nq_for(D), sms / 2 < kMaxSplit ? sms / 2 : kMaxSplit).total;
+  return ws_layout(D, nq_for(D) * 128, sms / 2 < kMaxSplit ? sms / 2 : kMaxSplit, 2).total;
 }
 
 int fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,

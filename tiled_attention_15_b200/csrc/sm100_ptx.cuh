@@ -205,11 +205,15 @@ __device__ __forceinline__ F2 exp2_fma2(F2 x) {
             __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23))};
 }
 
-__device__ __forceinline__ void setmaxnreg_inc_208() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+// Register re-partitioning between warpgroups (setmaxnreg counts must be
+// compile-time immediates): the softmax warpgroups grow, the others shrink.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ void setmaxnreg_dec_88() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N) : "memory");
 }
 
 // ---- generated register-list wrappers (tcgen05.ld + wait in one statement; tcgen05.st) ----
