@@ -8,8 +8,8 @@ nothing and keeps the split tail's scratch in a file-scope device array.
 Each case calls it through the C ABI twice in a row and checks both results
 against the existing workspace entry point (fa_fwd_ws with a caller-allocated
 workspace), within the parity tolerances of the other GPU tests.  The cases
-include shapes whose last round of tiles is split (so the static scratch is
-really used) and a causal one (no split).  The file name makes pytest collect
+include shapes whose last round of tiles is split and a decode shape split
+stream-K (so the static scratch is really used), and a causal one (no split).  The file name makes pytest collect
 it last, so a failure here leaves every other test already run.
 """
 import ctypes
@@ -31,6 +31,8 @@ CASES = [
     (Workload("capped D128 bf16 GQA ragged", 1, 10, 5, 300, 3500, 128, "bf16", False, seed=41), 8),
     (Workload("capped D256 fp16", 1, 5, 5, 512, 3072, 256, "fp16", False, seed=42), 8),
     (Workload("causal D64 bf16 (no split)", 2, 8, 2, 1000, 1000, 64, "bf16", True, seed=43), 0),
+    # 32 packed decode tiles on 148 SMs: stream-K partials in the static scratch
+    (Workload("decode GQA4 Nq1 D128 bf16 stream-K", 4, 32, 8, 1, 8192, 128, "bf16", False, seed=44), 0),
 ]
 
 

@@ -69,7 +69,9 @@ struct Geometry {
   static constexpr int KV_BYTES = kBN * D * 2;
   static constexpr int CHUNK_Q = kBM * 128;   // one 64-column chunk of a Q tile
   static constexpr int CHUNK_KV = kBN * 128;  // one 64-column chunk of a K/V block
-  static constexpr int NST = D == 64 ? 8 : (D == 128 ? 4 : 2);
+  // K/V stages: what the shared memory left by the Q tiles holds (one query
+  // tile leaves room for deeper staging, which decode-like launches need)
+  static constexpr int NST = NQ == 2 ? (D == 64 ? 8 : 4) : (D == 64 ? 12 : (D == 128 ? 6 : 2));
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = NQ * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NST * KV_BYTES;
@@ -80,7 +82,8 @@ struct Geometry {
                        B_TEMPTY = B_TFULL + kTileRing, NBAR = B_TEMPTY + kTileRing;
   // tmem base (u32), abort flag (u32), then the ring of unit indices (kTileRing x s32)
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 8 + 4 * kTileRing + 1024;  // + alignment slack
+  // ... then this CTA's stream-K unit range (2 x s32)
+  static constexpr int SMEM_BYTES = OFF_MISC + 8 + 4 * kTileRing + 8 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(NQ == 2 ? (256 + 2 * D <= 512) : (256 + D <= 512), "tensor memory budget");
@@ -104,12 +107,21 @@ struct FwdParams {
   // GQA packing (pack_g > 1): a work tile holds all pack_g query heads of one
   // key/value head, row r = (head r / Nq, query r % Nq), pack_g * Nq <= 128.
   int pack_g;
-  float* ws_o;      // [split tile][part][ws_rows][D] partial O (fp32)
-  float4* ws_ml;    // [split tile][part][ws_rows] (m, l, l_rounded, 0)
+  float* ws_o;      // [partial][ws_rows][D] partial O (fp32); a tile's parts are consecutive
+  float4* ws_ml;    // [partial][ws_rows] (m, l, l_rounded, 0)
   int* ws_cnt;      // [split tile][NQ][4 row groups] arrival counters (left at 0)
   // Dynamic schedule (with a workspace): sched[0] hands out units beyond the
   // first gridDim.x, sched[1] counts finished CTAs; the last CTA resets both.
   int* sched;
+  // Stream-K (sk_w > 0; non-causal launches with fewer tiles than CTAs): the
+  // sk_w = n_tiles * nkb key blocks of all tiles, flattened tile-major, are cut
+  // into gridDim.x equal contiguous ranges, one per CTA.  CTA c runs one unit
+  // per tile t that its range touches, with unit id c + t; the id also indexes
+  // the unit's partial in the workspace (ids grow with (t, c), never repeat).
+  // The host keeps sk_w * gridDim.x below 2^31.  The TMA thread publishes
+  // these units through the unit ring, like the dynamic schedule's.
+  int sk_w;
+  int use_ring;  // units come through the shared-memory ring (sched or sk_w)
 };
 
 struct Tile {
@@ -119,21 +131,43 @@ struct Tile {
   int nblk[2];
   int nb;
   int jb;     // first key block of this unit
-  int slot;   // split-tile index, or -1 for a whole tile
-  int half;   // which key part of a split tile
+  int slot;    // split-tile index, or -1 for a whole tile
+  int part;    // which key part of a split tile
+  int nparts;  // key parts of this split tile
+  int store0;  // workspace index of part 0 (parts are stored consecutively)
 };
 
 template <int NQ>
 __device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
   Tile T;
   int t = u;
+  int kb0 = 0, kb1 = p.nkb;  // split units: non-causal only (the host guarantees it)
   T.slot = -1;
-  T.half = 0;
-  if (u >= p.n_whole) {  // one key part of a split tile
+  T.part = 0;
+  T.nparts = 1;
+  T.store0 = 0;
+  if (p.sk_w > 0) {  // stream-K: this CTA's share of tile t
+    const int c = blockIdx.x, C = gridDim.x, W = p.sk_w, nkb = p.nkb;
+    t = u - c;
+    const int base = t * nkb;
+    const int b0 = c * W / C, b1 = (c + 1) * W / C;
+    kb0 = max(b0, base) - base;
+    kb1 = min(b1, base + nkb) - base;
+    // key block b belongs to CTA ((b + 1) * C - 1) / W
+    const int cf = ((base + 1) * C - 1) / W, cl = ((base + nkb) * C - 1) / W;
+    T.slot = t;
+    T.part = c - cf;
+    T.nparts = cl - cf + 1;
+    T.store0 = cf + t;
+  } else if (u >= p.n_whole) {  // one of nsplit equal key parts of a split tile
     const int v = u - p.n_whole;
     T.slot = v / p.nsplit;
-    T.half = v - T.slot * p.nsplit;
+    T.part = v - T.slot * p.nsplit;
+    T.nparts = p.nsplit;
+    T.store0 = T.slot * p.nsplit;
     t = p.n_whole + T.slot;
+    kb0 = (T.part * p.nkb) / p.nsplit;
+    kb1 = ((T.part + 1) * p.nkb) / p.nsplit;
   }
   int qt;
   if (p.pack_g > 1) {  // one tile per (batch, key/value head)
@@ -154,11 +188,6 @@ __device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
   }
   T.row0 = qt * NQ * kBM;
   const int rows = p.pack_g > 1 ? p.pack_g * p.Nq : p.Nq;  // rows of the (packed) tile space
-  int kb0 = 0, kb1 = p.nkb;  // split units: non-causal only (the host guarantees it)
-  if (T.slot >= 0) {
-    kb0 = (T.half * p.nkb) / p.nsplit;
-    kb1 = ((T.half + 1) * p.nkb) / p.nsplit;
-  }
   T.jb = kb0;
   T.nb = 0;
 #pragma unroll
@@ -264,23 +293,31 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > 100000000ull) return;
 }
 
-// Work units of a CTA.  Static schedule (p.sched == nullptr): the zig-zag
-// TileIter.  Dynamic schedule: the TMA thread takes unit blockIdx.x first, then
+// Work units of a CTA.  Static schedule (no ring): the zig-zag TileIter.
+// Dynamic schedule: the TMA thread takes unit blockIdx.x first, then
 // gridDim.x + atomicAdd(sched[0], 1) each time (heaviest units have the lowest
-// indices), and publishes every index -- or -1 at the end -- in a shared-memory
-// ring (t_full: written; t_empty: read by the MMA thread and every softmax warp,
-// 4 per query tile).
+// indices); stream-K: the TMA thread takes the CTA's fixed unit range.  Either
+// way it publishes every index -- or -1 at the end -- in a shared-memory ring
+// (t_full: written; t_empty: read by the MMA thread and every softmax warp, 4
+// per query tile).
 template <int D, int NQ>
 __device__ __forceinline__ bool produce_unit(const Ctx& cx, const FwdParams& p, TileIter& it,
                                              uint32_t& n, int& u) {
-  if (p.sched == nullptr) return it.next(u);
+  if (!p.use_ring) return it.next(u);
   using G = Geometry<D, NQ>;
-  u = (n == 0) ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
+  int end = p.n_units;
+  if (p.sk_w > 0) {  // stream-K: this CTA's fixed range, left by the prologue after the ring
+    const volatile int* sk = cx.ring + kTileRing;
+    u = sk[0] + static_cast<int>(n);
+    end = sk[1];
+  } else {
+    u = (n == 0) ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
+  }
   const int k = n % kTileRing;
   if (n >= (uint32_t)kTileRing &&
       !wait_bar(cx.bar(G::B_TEMPTY + k, G::OFF_BAR), ((n / kTileRing) - 1) & 1u, cx.abort_flag))
     return false;
-  const int pub = u < p.n_units ? u : -1;
+  const int pub = u < end ? u : -1;
   cx.ring[k] = pub;
   mbar_arrive(cx.bar(G::B_TFULL + k, G::OFF_BAR));  // release: the index is visible after the wait
   ++n;
@@ -290,7 +327,7 @@ __device__ __forceinline__ bool produce_unit(const Ctx& cx, const FwdParams& p, 
 template <int D, int NQ>
 __device__ __forceinline__ bool consume_unit(const Ctx& cx, const FwdParams& p, TileIter& it,
                                              uint32_t& n, int& u, int lane) {
-  if (p.sched == nullptr) return it.next(u);
+  if (!p.use_ring) return it.next(u);
   using G = Geometry<D, NQ>;
   const int k = n % kTileRing;
   bool ok = wait_bar(cx.bar(G::B_TFULL + k, G::OFF_BAR), (n / kTileRing) & 1u, cx.abort_flag);
@@ -591,7 +628,7 @@ __device__ __forceinline__ F2 unpack_bf16x2(uint32_t w) {
 // Epilogue of one key part of a split tile, for the 32 rows of this warp.  Each
 // part stores its un-normalised O row (fp32), its stabiliser m and sums l, l_r;
 // then the warp bumps the counter of its row group.  The warp that arrives last
-// (the nsplit-th) reads all parts, in part order, and writes the merged row:
+// (the nparts-th) reads all parts, in part order, and writes the merged row:
 //   M = max_s m_s,  a_s = 2^(m_s - M),  L = sum_s a_s l_s,
 //   O = sum_s a_s O_s / L,  LSE = (M + log2 L) ln 2,
 // then resets the counter to 0 for the next call.  No part waits for another,
@@ -603,10 +640,9 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
                                                float m, float l, float l_r) {
   const int rr = q * kBM + sub * 32 + lane;  // row of the work tile
   const bool stored = rr < p.ws_rows;         // rows beyond ws_rows do not exist
-  const size_t base = static_cast<size_t>(T.slot) * p.nsplit;
-  auto idx = [&](int part) { return (base + part) * p.ws_rows + rr; };
-  if (stored) p.ws_ml[idx(T.half)] = make_float4(m, l, l_r, 0.f);
-  float4* my_o = reinterpret_cast<float4*>(p.ws_o + idx(stored ? T.half : 0) * D);
+  auto idx = [&](int part) { return (static_cast<size_t>(T.store0) + part) * p.ws_rows + rr; };
+  if (stored) p.ws_ml[idx(T.part)] = make_float4(m, l, l_r, 0.f);
+  float4* my_o = reinterpret_cast<float4*>(p.ws_o + idx(stored ? T.part : 0) * D);
 #pragma unroll 1
   for (int c0 = 0; c0 < D; c0 += 32) {
     uint32_t orr[32];
@@ -624,13 +660,13 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
   int old = 0;
   if (lane == 0) old = atomicAdd(cnt, 1);
   old = __shfl_sync(0xffffffffu, old, 0);
-  if (old != p.nsplit - 1) return;  // a later part merges these rows
+  if (old != T.nparts - 1) return;  // a later part merges these rows
   __threadfence();
   if (stored) {
     float M = -INFINITY;
-    for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, __ldcg(p.ws_ml + idx(s)).x);
+    for (int s = 0; s < T.nparts; ++s) M = fmaxf(M, __ldcg(p.ws_ml + idx(s)).x);
     float L = 0.f, Lr = 0.f;
-    for (int s = 0; s < p.nsplit; ++s) {
+    for (int s = 0; s < T.nparts; ++s) {
       const float4 ml = __ldcg(p.ws_ml + idx(s));
       const float a = ex2(ml.x - M);
       L = fmaf(a, ml.y, L);
@@ -641,7 +677,7 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 8) {
       float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int s = 0; s < p.nsplit; ++s) {
+      for (int s = 0; s < T.nparts; ++s) {
         const float sc = ex2(__ldcg(p.ws_ml + idx(s)).x - M) * inv;
         const float4* po = reinterpret_cast<const float4*>(p.ws_o + idx(s) * D + c0);
         const float4 u0 = __ldcg(po), u1 = __ldcg(po + 1);
@@ -677,10 +713,16 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   uint32_t n_units_seen = 0;
   int t;
   while (consume_unit<D, NQ>(cx, p, it, n_units_seen, t, lane)) {
-    const Tile T = get_tile<NQ>(p, t);
-    const int nblk = T.nblk[q];
+    // Only what the key loop needs stays live across it; the epilogue decodes
+    // the unit again (registers are the softmax warps' tightest resource).
+    int nblk, rfirst, jb;
+    {
+      const Tile T0 = get_tile<NQ>(p, t);
+      nblk = T0.nblk[q];
+      rfirst = T0.row0 + q * kBM;
+      jb = T0.jb;
+    }
     if (nblk == 0) continue;
-    const int rfirst = T.row0 + q * kBM;
     // query position of this thread's row (causal mask; packing is non-causal only)
     const int row = rfirst + sub * 32 + lane;
     float m_used = -INFINITY, l = 0.f, l_r = 0.f;  // l: exact sum (LSE); l_r: rounded-P sum
@@ -693,7 +735,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
       uint32_t sr[kBN];
       tmem_ld_x128(tm + sb * 128, sr);
 
-      const int kbase = (T.jb + j) * kBN;
+      const int kbase = (jb + j) * kBN;
       const bool masked = (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst);
       float m_blk;
       if (masked) {  // scaled scores, -inf where the key is causal-future or past Nk
@@ -778,6 +820,9 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     if (!__all_sync(0xffffffffu, ok)) return;
     of_phase ^= 1u;
     tc_fence_after();
+    int t_again;  // opaque copy: the compiler must not keep the first decode live
+    asm volatile("mov.b32 %0, %1;" : "=r"(t_again) : "r"(t));
+    const Tile T = get_tile<NQ>(p, t_again);
     const RowInfo ri = row_info(p, T, q, sub * 32 + lane);
     const bool live = ri.live;
     const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
@@ -850,6 +895,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(B(G::B_TEMPTY + k), 1 + 4 * NQ);  // the MMA thread and the softmax warps
     }
     misc[1] = 0u;
+    if (p.sk_w > 0) {  // stream-K: the units c + t, t over the tiles this CTA's range touches
+      const int c = blockIdx.x, C = gridDim.x, W = p.sk_w;
+      int* sk = reinterpret_cast<int*>(misc + 2 + kTileRing);
+      sk[0] = c + c * W / C / p.nkb;
+      sk[1] = c + ((c + 1) * W / C - 1) / p.nkb + 1;
+    }
     fence_mbar_init();
   }
   if (warp == 8) {
@@ -983,6 +1034,13 @@ bool make_map(CUtensorMap* m, const void* ptr, int D, long long rows, long long 
 
 int nq_for(int D) { return D == 256 ? 1 : 2; }
 
+// GQA packing: when the query heads of one key/value head fit one 128-row tile
+// together (decode-like shapes), one work tile holds all of them.
+bool pack_heads(int Hq, int Hkv, int Nq, int causal) {
+  const int g = Hq / Hkv;
+  return g > 1 && !causal && static_cast<long long>(g) * Nq <= fa::kBM;
+}
+
 std::atomic<int> g_max_ctas{0};
 
 // Workspace partition for split tails.  The arrival counters come first, at a
@@ -991,8 +1049,7 @@ std::atomic<int> g_max_ctas{0};
 // 256 bytes.
 constexpr int kMaxSplit = 1024;  // >= half the SMs of any device
 constexpr int kMinSplitBlocks = 24;
-constexpr int kMinPartBlocks = 4;  // key blocks per part when a launch splits every tile
-constexpr int kMaxParts = 32;
+constexpr int kMinPartBlocks = 4;  // least key blocks per CTA under stream-K
 struct WsLayout {
   size_t cnt_off, ml_off, o_off, total;
 };
@@ -1030,10 +1087,8 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
       attr_done[dev] = true;
     }
   }
-  // GQA packing: when a key/value head's query heads fit one 128-row tile
-  // together (decode-like shapes), one tile holds all of them.
   const int g = Hq / Hkv;
-  const bool pack = g > 1 && !causal && g * Nq <= fa::kBM;
+  const bool pack = pack_heads(Hq, Hkv, Nq, causal);
   CUtensorMap tq, tq4, tk, tv;
   if (!make_map(&tq, q, D, Nq, (long long)B * Hq, fa::kBM, BF16) ||
       !make_map(&tk, k, D, Nk, (long long)B * Hkv, fa::kBN, BF16) ||
@@ -1067,16 +1122,21 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.ws_rows = pack ? g * Nq : (p.qt_per_head == 1 ? (Nq < NQ * fa::kBM ? Nq : NQ * fa::kBM)
                                                    : NQ * fa::kBM);
   int n_split = 0, nsplit = 1;
+  int sk_w = 0, sk_grid = 0;
   if (ws != nullptr && !causal) {
-    if (p.n_tiles < ctas && p.nkb >= 2 * kMinPartBlocks && p.n_tiles <= kMaxSplit) {
-      // Split-K: fewer tiles than SMs (decode-like shapes) -- every tile is cut
-      // into nsplit parts of the key blocks so that the units fill the device.
-      nsplit = (ctas + p.n_tiles - 1) / p.n_tiles;
-      if (nsplit > p.nkb / kMinPartBlocks) nsplit = p.nkb / kMinPartBlocks;
-      if (nsplit > kMaxParts) nsplit = kMaxParts;
-      while (nsplit >= 2 && ws_layout(D, p.ws_rows, p.n_tiles, nsplit).total > ws_bytes) --nsplit;
-      if (nsplit >= 2) n_split = p.n_tiles;
-      else nsplit = 1;
+    if (p.n_tiles < ctas && p.n_tiles <= kMaxSplit) {
+      // Stream-K: fewer tiles than CTAs (decode-like shapes).  The key blocks of
+      // all tiles are shared out evenly over C CTAs, each with at least
+      // kMinPartBlocks of them; C shrinks until the partials fit the workspace.
+      const long long W = static_cast<long long>(p.n_tiles) * p.nkb;
+      long long C = W / kMinPartBlocks < ctas ? W / kMinPartBlocks : ctas;
+      while (C > p.n_tiles &&
+             ws_layout(D, p.ws_rows, static_cast<int>(C) + p.n_tiles, 1).total > ws_bytes)
+        C -= (C - p.n_tiles + 7) / 8;
+      if (C > p.n_tiles && (W + 1) * C < (1ll << 31)) {  // the kernel's index math is 32-bit
+        sk_w = static_cast<int>(W);
+        sk_grid = static_cast<int>(C);
+      }
     } else {
       // Split tail: if the last round of tiles would keep at most half of the
       // CTAs busy, give each of those tiles to two CTAs, one per half of the key
@@ -1092,9 +1152,10 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
       }
     }
   }
-  if (n_split > 0) {
-    const WsLayout L = ws_layout(D, p.ws_rows, n_split, nsplit);
-    if (ws_bytes < L.total) {
+  if (n_split > 0 || sk_w > 0) {
+    const WsLayout L = sk_w > 0 ? ws_layout(D, p.ws_rows, sk_grid + p.n_tiles, 1)
+                                : ws_layout(D, p.ws_rows, n_split, nsplit);
+    if (ws_bytes < L.total) {  // split tail only: stream-K was sized to fit
       if (mode == Scratch::kStatic) return FA_ERR_SCRATCH_TOO_SMALL;
       n_split = 0;
       nsplit = 1;
@@ -1108,21 +1169,24 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
       p.ws_cnt = reinterpret_cast<int*>(base + L.cnt_off);
     }
   }
-  if (n_split == 0) {
+  if (n_split == 0 && sk_w == 0) {
     p.ws_o = nullptr;
     p.ws_ml = nullptr;
     p.ws_cnt = nullptr;
   }
+  p.sk_w = sk_w;
   p.nsplit = nsplit;
-  p.n_whole = p.n_tiles - n_split;
-  p.n_units = p.n_whole + nsplit * n_split;
-  const int grid = p.n_units < ctas ? p.n_units : ctas;
+  p.n_whole = sk_w > 0 ? 0 : p.n_tiles - n_split;
+  p.n_units = sk_w > 0 ? sk_grid + p.n_tiles : p.n_whole + nsplit * n_split;
+  const int grid = sk_w > 0 ? sk_grid : (p.n_units < ctas ? p.n_units : ctas);
   // Dynamic schedule for non-causal launches with a workspace in which a CTA gets
   // several units (for causal ones the static heavy-first zig-zag measured as
-  // fast or faster).
+  // fast or faster; stream-K fixes each CTA's units).
   p.sched = nullptr;
-  if (ws != nullptr && !causal && ws_bytes >= ws_layout(D, 0, 0, 0).ml_off && p.n_units > grid)
+  if (ws != nullptr && !causal && sk_w == 0 && ws_bytes >= ws_layout(D, 0, 0, 0).ml_off &&
+      p.n_units > grid)
     p.sched = reinterpret_cast<int*>(static_cast<char*>(ws) + kMaxSplit * 2 * 4 * sizeof(int));
+  p.use_ring = (p.sched != nullptr || sk_w > 0) ? 1 : 0;
   fa::fa_fwd_kernel<D, NQ, BF16><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(tq, tq4, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
@@ -1203,17 +1267,22 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   if (!ds.sm100 || ds.sms < 1) return FA_ERR_NO_DEVICE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA_BF16;
+  // A work tile of at most 128 rows (short queries, or a packed GQA group) runs
+  // the one-query-tile kernel: its two S buffers let the softmax of key block j
+  // overlap the S MMA of block j + 1, and its K/V staging is deeper.
+  const bool one_tile = (pack_heads(Hq, Hkv, Nq, causal) ? (Hq / Hkv) * Nq : Nq) <= fa::kBM;
+#define FA_ARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode
   switch (D) {
     case 64:
-      return bf ? launch<64, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode)
-                : launch<64, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode);
+      if (one_tile) return bf ? launch<64, 1, true>(FA_ARGS) : launch<64, 1, false>(FA_ARGS);
+      return bf ? launch<64, 2, true>(FA_ARGS) : launch<64, 2, false>(FA_ARGS);
     case 128:
-      return bf ? launch<128, 2, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode)
-                : launch<128, 2, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode);
+      if (one_tile) return bf ? launch<128, 1, true>(FA_ARGS) : launch<128, 1, false>(FA_ARGS);
+      return bf ? launch<128, 2, true>(FA_ARGS) : launch<128, 2, false>(FA_ARGS);
     default:
-      return bf ? launch<256, 1, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode)
-                : launch<256, 1, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode);
+      return bf ? launch<256, 1, true>(FA_ARGS) : launch<256, 1, false>(FA_ARGS);
   }
+#undef FA_ARGS
 }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
