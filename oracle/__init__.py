@@ -50,6 +50,13 @@ def _load():
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
             ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
             ctypes.c_int]
+        lib.oracle_attention_ex.restype = ctypes.c_int
+        lib.oracle_attention_ex.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+            ctypes.c_int64, ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -71,12 +78,17 @@ def max_threads() -> int:
 
 
 def attention(q, k, v, scale: float, causal: bool, rows: Optional[np.ndarray] = None,
-              nthreads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+              nthreads: int = 0, window: Tuple[int, int] = (-1, -1),
+              bias=None) -> Tuple[np.ndarray, np.ndarray]:
     """Reference attention in float64.
 
     q: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] (torch tensors or numpy arrays).
     rows: optional sorted int64 array of query positions; only those rows are
     computed (then the result has R = len(rows) rows per head).
+    window: (left, right): key j is visible to query i iff i - left <= j <= i + right;
+    a negative bound is no bound (causal is right = 0).
+    bias: optional additive score bias broadcastable to [B, Hq, Nq, Nk] (float32
+    values; -inf removes a key).  A row with no key left gets O = 0, LSE = -inf.
     Returns (O [B, Hq, R, D] float64, LSE [B, Hq, R] float64).
     """
     lib = _load()
@@ -97,9 +109,23 @@ def attention(q, k, v, scale: float, causal: bool, rows: Optional[np.ndarray] = 
         pos_ptr = None
     o = np.empty((B, Hq, R, D), dtype=np.float64)
     lse = np.empty((B, Hq, R), dtype=np.float64)
-    rc = lib.oracle_attention(qf.ctypes.data, pos_ptr, R, kf.ctypes.data, vf.ctypes.data,
-                              o.ctypes.data, lse.ctypes.data, B, Hq, Hkv, Nq, Nk, D,
-                              float(scale), int(bool(causal)), int(nthreads))
+    bias_ptr, sb, sh, sq = None, 0, 0, 0
+    if bias is not None:
+        bf = _as_f32(bias)
+        while bf.ndim < 4:
+            bf = bf[None]
+        if bf.ndim != 4 or bf.shape[3] != Nk or any(
+                n not in (1, full) for n, full in zip(bf.shape[:3], (B, Hq, Nq))):
+            raise ValueError("bias must broadcast to [B, Hq, Nq, Nk] with its last dim Nk")
+        bf = np.ascontiguousarray(bf)
+        # element strides; a broadcast dim gets stride 0
+        st = [0 if bf.shape[d] == 1 else int(np.prod(bf.shape[d + 1:])) for d in range(3)]
+        bias_ptr, (sb, sh, sq) = bf.ctypes.data, st
+    wl, wr = (int(x) for x in window)
+    rc = lib.oracle_attention_ex(qf.ctypes.data, pos_ptr, R, kf.ctypes.data, vf.ctypes.data,
+                                 o.ctypes.data, lse.ctypes.data, B, Hq, Hkv, Nq, Nk, D,
+                                 float(scale), int(bool(causal)), wl, wr, bias_ptr, sb, sh, sq,
+                                 int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_attention rejected its arguments (code {rc})")
     return o, lse

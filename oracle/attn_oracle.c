@@ -38,27 +38,38 @@
 #include <omp.h>
 #endif
 
-/* One query row.  q: [D], k and v: [Nk, D] of one kv head.  s: scratch [Nk]. */
-static void attend_row(const float *q, const float *k, const float *v, int64_t n_vis,
-                       int64_t D, double scale, double *s, double *o, double *lse) {
+/*
+ * One query row over the keys j0 .. j0 + n_vis - 1 of one kv head.
+ * q: [D]; k, v: [Nk, D]; bias: NULL or the row's additive score bias [Nk]
+ * (-inf removes a key); s: scratch [Nk].  A row with no key left (n_vis == 0,
+ * or every biased score -inf) has no softmax: O = 0 and LSE = -inf.
+ */
+static void attend_row(const float *q, const float *k, const float *v, const float *bias,
+                       int64_t j0, int64_t n_vis, int64_t D, double scale, double *s, double *o,
+                       double *lse) {
     /* pass 1: scores */
     double M = -INFINITY;
-    for (int64_t j = 0; j < n_vis; ++j) {
+    for (int64_t j = j0; j < j0 + n_vis; ++j) {
         double acc = 0.0;
         const float *kj = k + j * D;
         for (int64_t d = 0; d < D; ++d) acc += (double)q[d] * (double)kj[d];
         s[j] = scale * acc;
+        if (bias) s[j] += (double)bias[j];
         if (s[j] > M) M = s[j];
+    }
+    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    if (M == -INFINITY) { /* no visible key */
+        *lse = -INFINITY;
+        return;
     }
     /* pass 2: softmax weights */
     double Z = 0.0;
-    for (int64_t j = 0; j < n_vis; ++j) {
+    for (int64_t j = j0; j < j0 + n_vis; ++j) {
         s[j] = exp(s[j] - M);
         Z += s[j];
     }
     /* pass 3: weighted sum of values */
-    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
-    for (int64_t j = 0; j < n_vis; ++j) {
+    for (int64_t j = j0; j < j0 + n_vis; ++j) {
         const double p = s[j] / Z;
         const float *vj = v + j * D;
         for (int64_t d = 0; d < D; ++d) o[d] += p * (double)vj[d];
@@ -71,12 +82,25 @@ static void attend_row(const float *q, const float *k, const float *v, int64_t n
  * q_pos:  [R] position of each supplied row in 0..Nq-1, or NULL (then R must equal Nq)
  * k, v:   [B, Hkv, Nk, D] float32
  * o:      [B, Hq, R, D] float64 output;  lse: [B, Hq, R] float64 output (may be NULL)
+ *
+ * Masks beyond causal (the pages put the mask step on the vector unit, and
+ * PyTorch's scaled_dot_product_attention, which the mooersco.com page calls,
+ * takes an attn_mask).  Readings taken:
+ *   - a key window: key j is visible to query i iff i - window_left <= j and
+ *     j <= i + window_right, a negative bound meaning no bound on that side;
+ *     causal is the right bound 0 (top-left alignment, as above);
+ *   - an additive bias (float attn_mask): bias[b, h, i, j] is added to the
+ *     scaled score, -inf removing the key.  Element (b, hq, i, j) sits at
+ *     b * bias_sb + hq * bias_sh + i * bias_sq + j (a zero stride broadcasts);
+ *     bias may be NULL;
+ *   - a row with no key left has no softmax: O = 0 and LSE = -inf.
  * Returns 0, or a negative number for invalid arguments.
  */
-int oracle_attention(const float *q, const int64_t *q_pos, int64_t R, const float *k,
-                     const float *v, double *o, double *lse, int64_t B, int64_t Hq,
-                     int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D, double scale, int causal,
-                     int nthreads) {
+int oracle_attention_ex(const float *q, const int64_t *q_pos, int64_t R, const float *k,
+                        const float *v, double *o, double *lse, int64_t B, int64_t Hq,
+                        int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D, double scale, int causal,
+                        int64_t window_left, int64_t window_right, const float *bias,
+                        int64_t bias_sb, int64_t bias_sh, int64_t bias_sq, int nthreads) {
     if (!q || !k || !v || !o) return -1;
     if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || D < 1 || R < 1) return -2;
     if (Hq % Hkv != 0) return -3;
@@ -84,6 +108,7 @@ int oracle_attention(const float *q, const int64_t *q_pos, int64_t R, const floa
     if (q_pos)
         for (int64_t r = 0; r < R; ++r)
             if (q_pos[r] < 0 || q_pos[r] >= Nq) return -5;
+    if (bias && (bias_sb < 0 || bias_sh < 0 || bias_sq < 0)) return -7;
     const int64_t group = Hq / Hkv;
     const int64_t total = B * Hq * R;
     int err = 0;
@@ -107,17 +132,31 @@ int oracle_attention(const float *q, const int64_t *q_pos, int64_t R, const floa
             const int64_t b = bh / Hq, hq = bh % Hq;
             const int64_t kvh = hq / group;
             const int64_t i = q_pos ? q_pos[r] : r;
-            int64_t n_vis = Nk;
-            if (causal) n_vis = (i + 1 < Nk) ? i + 1 : Nk;
+            /* visible keys: j0 .. j1 (inclusive), clipped to 0 .. Nk-1 */
+            int64_t j0 = 0, j1 = Nk - 1;
+            if (causal && i < j1) j1 = i;
+            if (window_right >= 0 && i + window_right < j1) j1 = i + window_right;
+            if (window_left >= 0 && i - window_left > j0) j0 = i - window_left;
+            const int64_t n_vis = j1 >= j0 ? j1 - j0 + 1 : 0;
             const float *kb = k + (b * Hkv + kvh) * Nk * D;
             const float *vb = v + (b * Hkv + kvh) * Nk * D;
+            const float *brow = bias ? bias + b * bias_sb + hq * bias_sh + i * bias_sq : NULL;
             double lse_row;
-            attend_row(q + t * D, kb, vb, n_vis, D, scale, s, o + t * D, &lse_row);
+            attend_row(q + t * D, kb, vb, brow, j0, n_vis, D, scale, s, o + t * D, &lse_row);
             if (lse) lse[t] = lse_row;
         }
         free(s);
     }
     return err;
+}
+
+/* The unmasked / causal oracle: oracle_attention_ex with no window and no bias. */
+int oracle_attention(const float *q, const int64_t *q_pos, int64_t R, const float *k,
+                     const float *v, double *o, double *lse, int64_t B, int64_t Hq,
+                     int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D, double scale, int causal,
+                     int nthreads) {
+    return oracle_attention_ex(q, q_pos, R, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                               -1, -1, NULL, 0, 0, 0, nthreads);
 }
 
 int oracle_max_threads(void) {
