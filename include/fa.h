@@ -71,7 +71,8 @@ enum fa_status {
   FA_ERR_DRIVER = 10,              /* tensor-map encoding via the driver failed    */
   FA_ERR_DEVICE_TIMEOUT = 11,      /* (device status) a kernel wait hit its limit  */
   FA_ERR_OVERLAP = 12,             /* o or lse overlaps q, k or v                  */
-  FA_ERR_SCRATCH_TOO_SMALL = 13    /* fa_fwd_noalloc: static scratch too small     */
+  FA_ERR_SCRATCH_TOO_SMALL = 13,   /* fa_fwd_noalloc: static scratch too small     */
+  FA_ERR_BAD_WINDOW = 14           /* fa_fwd_window: bound < -1, or causal + right > 0 */
 };
 
 /*
@@ -99,12 +100,15 @@ int fa_fwd_bf16(const void *q, const void *k, const void *v, void *o, float *lse
 /*
  * fa_fwd with a caller-provided device workspace (no counterpart on the pages: it
  * exists for load balance on this device).  With a workspace, non-causal calls
- * take their work tiles from a counter in the workspace (dynamic schedule), and
- * a call whose last round of tiles would keep at most half of the SMs busy
- * gives each of those tiles to two CTAs, one per half of the key blocks (from
- * 24 key blocks up); each half leaves its un-normalised partial output in the
- * workspace and the second to finish merges.  Results agree with fa_fwd within
- * rounding (the order of the additions differs).
+ * take their work tiles from a counter in the workspace (dynamic schedule); a
+ * call whose last round of tiles would keep at most half of the SMs busy gives
+ * each of those tiles to two CTAs, one per half of the key blocks (from 24 key
+ * blocks up); and a call with fewer work tiles than SMs (KV-cache decode: the
+ * query heads of a GQA group share one tile when they fit its 128 rows) shares
+ * the key blocks of all tiles out evenly over the SMs (stream-K).  Every part
+ * leaves its un-normalised partial output in the workspace and the last to
+ * finish merges them, in a fixed order.  Results agree with fa_fwd within
+ * rounding (the order of the additions differs) and repeat bit for bit.
  *   workspace        device memory of at least fa_fwd_workspace_size(D) bytes,
  *                    256-byte aligned (else FA_ERR_MISALIGNED), zero-filled
  *                    before its first use.  Every call that completes leaves the
@@ -121,6 +125,25 @@ int fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float *lse, 
 /* Workspace bytes fa_fwd_ws needs on the current device for head_dim D (about 20 MB
  * on a 148-SM B200); 0 if D is unsupported or no device is current. */
 size_t fa_fwd_workspace_size(int D);
+
+/*
+ * Attention with a key window (a mask beyond causal: the pages place the mask
+ * step on the vector unit, and the scaled_dot_product_attention call of the
+ * mooersco.com page takes an attn_mask).  Query i sees key j iff
+ *     i - window_left <= j <= i + window_right      (0-based, top-left aligned),
+ * a bound of -1 meaning no bound on that side; causal = 1 is window_right = 0
+ * (window_right must then be -1 or 0).  A query row that sees no key (only
+ * when Nq > Nk + window_left) gets O = 0 and LSE = -inf.  Key blocks wholly
+ * outside a tile's windows are not read.  Other arguments, layout and errors
+ * as fa_fwd_ws (the workspace is optional and only balances the schedule:
+ * windowed calls are never split); FA_ERR_BAD_WINDOW for a bound below -1 or
+ * a causal call with window_right > 0.  window_left = window_right = -1 gives
+ * fa_fwd_ws's result within rounding.
+ */
+int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                  int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
+                  int window_left, int window_right, void *stream, int dtype, void *workspace,
+                  size_t workspace_bytes);
 
 /*
  * fa_fwd_ws for callers that cannot allocate device memory.  The pages have no

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 14):
+    for code in range(0, 15):
         s = fa.status_string(code)
         assert s and s != "unknown status", code
     assert fa.status_string(99) == "unknown status"
@@ -97,3 +97,21 @@ def test_workspace_entry_point_host_checks(lib):
     assert lib.fa_fwd_ws(*args[:10], 96, *args[11:], 7 * A, 1 << 20) == 5  # head_dim checked first
     assert fa.set_max_ctas(-1) == 3
     assert fa.set_max_ctas(0) == 0
+
+
+def test_window_entry_point_host_checks(lib):
+    import torch
+    a = dict(GOOD)
+
+    def call(wl, wr, causal=0, ws=None, dtype=a["dtype"], D=a["D"]):
+        return lib.fa_fwd_window(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"],
+                                 a["Hkv"], a["Nq"], a["Nk"], D, ctypes.c_float(a["scale"]),
+                                 causal, wl, wr, None, dtype, ws, 0)
+    bad = fa.FA_ERR_BAD_WINDOW
+    assert call(-2, 3) == bad and call(4, -2) == bad
+    assert call(8, 1, causal=1) == bad  # causal fixes the right bound at 0
+    assert call(8, 0, ws=7 * A + 128) == 2  # workspace not 256-byte aligned
+    assert call(8, 0, dtype=5) == 7 and call(8, 0, D=80) == 5
+    if not torch.cuda.is_available():
+        for wl, wr, causal in ((-1, -1, 0), (0, 0, 0), (16, -1, 1), (16, 0, 1), (3, 7, 0)):
+            assert call(wl, wr, causal) == 8  # valid: reaches the device check

@@ -21,9 +21,11 @@ LIB_PATH = os.path.join(_HERE, "libfa.so")
 FA_FP16, FA_BF16 = 0, 1
 FA_OK = 0
 FA_ERR_DEVICE_TIMEOUT = 11
+FA_ERR_BAD_WINDOW = 14
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
+            "fa_fwd_window",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
             "fa_status_string", "fa_device_status", "fa_device_timeout_site",
             "fa_debug_exp2_fma", "fa_debug_wait_timeout", "fa_fwd_num_tiles")
@@ -56,6 +58,8 @@ def load_library() -> ctypes.CDLL:
         getattr(lib, name).restype = i
     lib.fa_fwd_ws.argtypes = fwd_args + [i, vp, ctypes.c_size_t]
     lib.fa_fwd_ws.restype = i
+    lib.fa_fwd_window.argtypes = fwd_args[:13] + [i, i, vp, i, vp, ctypes.c_size_t]
+    lib.fa_fwd_window.restype = i
     lib.fa_fwd_noalloc.argtypes = fwd_args + [i]
     lib.fa_fwd_noalloc.restype = i
     lib.fa_fwd_noalloc_scratch_bytes.argtypes = []
@@ -151,14 +155,15 @@ def fa_fwd_raw(q: int, k: int, v: int, o: int, lse: Optional[int], B: int, Hq: i
 
 
 def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False,
-           return_lse: bool = True, stream=None,
-           use_workspace: bool = True) -> Tuple[object, Optional[object]]:
+           return_lse: bool = True, stream=None, use_workspace: bool = True,
+           window: Tuple[int, int] = (-1, -1)) -> Tuple[object, Optional[object]]:
     """Fused attention forward on the current CUDA stream.
 
     q: [B, Hq, Nq, D], k/v: [B, Hkv, Nk, D] contiguous CUDA tensors, fp16 or bf16.
     o: optional output like q; lse: optional float32 [B, Hq, Nq] output.
     scale defaults to 1/sqrt(D).  use_workspace: call fa_fwd_ws with a cached
-    per-(device, stream) workspace (split tails for load balance), else fa_fwd.
+    per-(device, stream) workspace (load balance), else fa_fwd.  window:
+    (left, right) key window, -1 = unbounded (fa_fwd_window when either is set).
     Returns (o, lse or None).
     """
     import torch
@@ -191,7 +196,13 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
             lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, D,
             ctypes.c_float(scale), 1 if causal else 0, stream or None, dtype)
-    if use_workspace:
+    wl, wr = (int(x) for x in window)
+    if (wl, wr) != (-1, -1):
+        ws = workspace(q.device, stream) if use_workspace else None
+        rc = lib.fa_fwd_window(*args[:13], wl, wr, args[13], dtype,
+                               ws.data_ptr() if ws is not None else None,
+                               ws.numel() if ws is not None else 0)
+    elif use_workspace:
         ws = workspace(q.device, stream)
         rc = lib.fa_fwd_ws(*args, ws.data_ptr(), ws.numel())
     else:

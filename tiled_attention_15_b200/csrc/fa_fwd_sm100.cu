@@ -94,6 +94,11 @@ struct FwdParams {
   float* lse;
   int B, Hq, Hkv, Nq, Nk, group;
   int causal;
+  // Key window: query i sees keys i - wl .. i + wr; -1 is no bound.  wr is 0
+  // for causal launches.  Windowed launches (wl >= 0, or wr >= 0 without
+  // causal) use one query tile per work tile and are not split.  (Two fields,
+  // not a third flag: a larger parameter block made the two-tile kernels spill.)
+  int wl, wr;
   float c;          // scale * log2(e)
   int qt_per_head;  // work tiles per (batch, head)
   int n_tiles;
@@ -196,7 +201,14 @@ __device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
     int n = 0;
     if (q < NQ && rf < rows) {
       n = kb1 - kb0;
-      if (p.causal && p.pack_g <= 1) {
+      if (NQ == 1 && (p.wl >= 0 || (p.wr >= 0 && !p.causal))) {  // this tile's own block range, at least one block
+        const int rl = min(rf + kBM - 1, p.Nq - 1);
+        const int hi = p.wr >= 0 ? min(p.Nk - 1, rl + p.wr) : p.Nk - 1;
+        const int lo = p.wl >= 0 ? max(0, rf - p.wl) : 0;
+        const int b_lo = min(lo / kBN, p.nkb - 1);
+        T.jb = b_lo;
+        n = max(1, hi / kBN + 1 - b_lo);  // rows that see no key still get O = 0, LSE = -inf
+      } else if (p.causal && p.pack_g <= 1) {
         const int rl = min(rf + kBM - 1, p.Nq - 1);
         n = min(p.nkb, rl / kBN + 1);
       }
@@ -706,6 +718,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   const uint32_t tm = cx.tmem + lane_off;
   auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
   const float c = p.c;
+  constexpr bool kWin = NQ == 1;  // key windows: one-query-tile kernels only
   uint32_t s_phase[2] = {0u, 0u}, of_phase = 0u, pv_seen = 0u;
   const int q = (NQ == 2) ? wg : 0;
 
@@ -736,14 +749,28 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
       tmem_ld_x128(tm + sb * 128, sr);
 
       const int kbase = (jb + j) * kBN;
-      const bool masked = (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst);
+      // (key windows exist in the one-query-tile kernels only)
+      const bool masked =
+          kWin ? (kbase + kBN > p.Nk) || (p.wr >= 0 && kbase + kBN - 1 > rfirst + p.wr) ||
+                     (p.wl >= 0 && kbase < rfirst + kBM - 1 - p.wl)
+               : (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst);
       float m_blk;
-      if (masked) {  // scaled scores, -inf where the key is causal-future or past Nk
-        int lim = p.Nk - kbase;
-        if (p.causal) lim = min(lim, row - kbase + 1);
+      if (masked) {  // scaled scores, -inf where the key is outside the window or past Nk
+        int lim = p.Nk - kbase;  // keys [lo, lim) of the block are visible to this row
+        if (kWin) {
+          if (p.wr >= 0) lim = min(lim, row + p.wr - kbase + 1);
+          const int lo = p.wl >= 0 ? row - p.wl - kbase : 0;
+          const uint32_t span = static_cast<uint32_t>(max(lim - lo, 0));
 #pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          sr[i] = __float_as_uint((i < lim) ? __uint_as_float(sr[i]) * c : -INFINITY);
+          for (int i = 0; i < kBN; ++i)
+            sr[i] = __float_as_uint(static_cast<uint32_t>(i - lo) < span ? __uint_as_float(sr[i]) * c
+                                                                          : -INFINITY);
+        } else {
+          if (p.causal) lim = min(lim, row - kbase + 1);
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            sr[i] = __float_as_uint((i < lim) ? __uint_as_float(sr[i]) * c : -INFINITY);
+        }
         m_blk = row_max(sr);
       } else {  // max of raw scores; the scale (of either sign) is applied to the max
         m_blk = (c >= 0.f ? row_max(sr) : row_min(sr)) * c;
@@ -829,7 +856,9 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     if (T.slot >= 0) {
       merge_epilogue<D, NQ, BF16>(p, T, q, sub, lane, ri, tm + 256 + q * D, m_sub, l, l_r);
     } else {
-      const float inv_l = 1.f / (BF16 ? l_r : l);
+      // a row that saw no key (key windows only) has no softmax: O = 0, LSE = -inf
+      const bool empty = kWin && m_used == -INFINITY;
+      const float inv_l = empty ? 0.f : 1.f / (BF16 ? l_r : l);
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -848,7 +877,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
         }
       }
       if (p.lse != nullptr && live)
-        p.lse[ri.out_row] = (m_sub + log2f(l)) * kLn2;
+        p.lse[ri.out_row] = empty ? -INFINITY : (m_sub + log2f(l)) * kLn2;
     }
     tc_fence_before();
     __syncwarp();
@@ -1072,8 +1101,8 @@ enum class Scratch { kCaller, kStatic };
 
 template <int D, int NQ, bool BF16>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-           int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream, int dev,
-           void* ws, size_t ws_bytes, Scratch mode) {
+           int Hkv, int Nq, int Nk, float scale, int causal, int wl, int wr, cudaStream_t stream,
+           int dev, void* ws, size_t ws_bytes, Scratch mode) {
   using G = fa::Geometry<D, NQ>;
   static bool attr_done[kMaxDevices] = {};
   static std::mutex mu;
@@ -1088,7 +1117,8 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     }
   }
   const int g = Hq / Hkv;
-  const bool pack = pack_heads(Hq, Hkv, Nq, causal);
+  const bool windowed = wl >= 0 || wr >= 0;
+  const bool pack = !windowed && pack_heads(Hq, Hkv, Nq, causal);
   CUtensorMap tq, tq4, tk, tv;
   if (!make_map(&tq, q, D, Nq, (long long)B * Hq, fa::kBM, BF16) ||
       !make_map(&tk, k, D, Nk, (long long)B * Hkv, fa::kBN, BF16) ||
@@ -1110,6 +1140,8 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.Nk = Nk;
   p.group = g;
   p.causal = causal ? 1 : 0;
+  p.wl = wl;
+  p.wr = causal ? 0 : wr;
   p.c = scale * 1.4426950408889634f;
   p.pack_g = pack ? g : 1;
   p.qt_per_head = pack ? 1 : (Nq + NQ * fa::kBM - 1) / (NQ * fa::kBM);
@@ -1123,7 +1155,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
                                                    : NQ * fa::kBM);
   int n_split = 0, nsplit = 1;
   int sk_w = 0, sk_grid = 0;
-  if (ws != nullptr && !causal) {
+  if (ws != nullptr && !causal && !windowed) {
     if (p.n_tiles < ctas && p.n_tiles <= kMaxSplit) {
       // Stream-K: fewer tiles than CTAs (decode-like shapes).  The key blocks of
       // all tiles are shared out evenly over C CTAs, each with at least
@@ -1218,6 +1250,8 @@ const char* fa_status_string(int s) {
     case FA_ERR_SCRATCH_TOO_SMALL:
       return "fa_fwd_noalloc: this problem needs more scratch than the static buffer holds; "
              "use fa_fwd_ws";
+    case FA_ERR_BAD_WINDOW:
+      return "key window bounds must be >= -1, and a causal launch cannot have window_right > 0";
     default: return "unknown status";
   }
 }
@@ -1230,9 +1264,11 @@ long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D) {
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                     int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype,
-                    void* ws, size_t ws_bytes, Scratch mode = Scratch::kCaller) {
+                    void* ws, size_t ws_bytes, Scratch mode = Scratch::kCaller, int wl = -1,
+                    int wr = -1) {
   // ---- argument checks: host only, before any CUDA call
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
+  if (wl < -1 || wr < -1 || (causal && wr > 0)) return FA_ERR_BAD_WINDOW;
   if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_BAD_SHAPE;
   if (Hq % Hkv != 0) return FA_ERR_BAD_GROUPING;
@@ -1270,8 +1306,11 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   // A work tile of at most 128 rows (short queries, or a packed GQA group) runs
   // the one-query-tile kernel: its two S buffers let the softmax of key block j
   // overlap the S MMA of block j + 1, and its K/V staging is deeper.
-  const bool one_tile = (pack_heads(Hq, Hkv, Nq, causal) ? (Hq / Hkv) * Nq : Nq) <= fa::kBM;
-#define FA_ARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, st, dev, ws, ws_bytes, mode
+  // Windowed launches too: each tile gets its own key block range.
+  const bool windowed = wl >= 0 || wr >= 0;
+  const bool one_tile =
+      windowed || (pack_heads(Hq, Hkv, Nq, causal) ? (Hq / Hkv) * Nq : Nq) <= fa::kBM;
+#define FA_ARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, wl, wr, st, dev, ws, ws_bytes, mode
   switch (D) {
     case 64:
       if (one_tile) return bf ? launch<64, 1, true>(FA_ARGS) : launch<64, 1, false>(FA_ARGS);
@@ -1288,6 +1327,17 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
            int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype) {
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, nullptr, 0);
+}
+
+int fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                  int Hkv, int Nq, int Nk, int D, float scale, int causal, int window_left,
+                  int window_right, void* stream, int dtype, void* workspace,
+                  size_t workspace_bytes) {
+  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return FA_ERR_MISALIGNED;
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype,
+                  workspace, workspace != nullptr ? workspace_bytes : 0, Scratch::kCaller,
+                  window_left, window_right);
 }
 
 size_t fa_fwd_workspace_size(int D) {
