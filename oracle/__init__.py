@@ -57,6 +57,9 @@ def _load():
             ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
             ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
             ctypes.c_int64, ctypes.c_int]
+        lib.oracle_attention_bwd.restype = ctypes.c_int
+        lib.oracle_attention_bwd.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64] * 6 + [
+            ctypes.c_double, ctypes.c_int, ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -129,3 +132,29 @@ def attention(q, k, v, scale: float, causal: bool, rows: Optional[np.ndarray] = 
     if rc != 0:
         raise ValueError(f"oracle_attention rejected its arguments (code {rc})")
     return o, lse
+
+
+def attention_bwd(q, k, v, dout, scale: float, causal: bool, nthreads: int = 0):
+    """Gradients of attention in float64 for the upstream gradient dout.
+
+    q, dout: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] (torch tensors or numpy arrays).
+    Returns (dQ [B, Hq, Nq, D], dK [B, Hkv, Nk, D], dV [B, Hkv, Nk, D],
+    Delta [B, Hq, Nq]) as float64 numpy arrays; Delta_i = dO_i . O_i.
+    """
+    lib = _load()
+    qf, kf, vf, gf = _as_f32(q), _as_f32(k), _as_f32(v), _as_f32(dout)
+    B, Hq, Nq, D = qf.shape
+    Bk, Hkv, Nk, Dk = kf.shape
+    if (Bk, Dk) != (B, D) or vf.shape != kf.shape or gf.shape != qf.shape:
+        raise ValueError("shape mismatch between q, k, v, dout")
+    dq = np.empty((B, Hq, Nq, D), dtype=np.float64)
+    dk = np.empty((B, Hkv, Nk, D), dtype=np.float64)
+    dv = np.empty((B, Hkv, Nk, D), dtype=np.float64)
+    delta = np.empty((B, Hq, Nq), dtype=np.float64)
+    rc = lib.oracle_attention_bwd(qf.ctypes.data, kf.ctypes.data, vf.ctypes.data, gf.ctypes.data,
+                                  dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, delta.ctypes.data,
+                                  B, Hq, Hkv, Nq, Nk, D, float(scale), int(bool(causal)),
+                                  int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_bwd rejected its arguments (code {rc})")
+    return dq, dk, dv, delta

@@ -1,5 +1,6 @@
 /*
- * Oracle for the attention forward pass -- TEST INFRASTRUCTURE ONLY.
+ * Oracle for the attention forward pass (and its gradients, below) -- TEST
+ * INFRASTRUCTURE ONLY.
  *
  * Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline leg may
  * load this library.  It shares no code with the CUDA path.
@@ -157,6 +158,111 @@ int oracle_attention(const float *q, const int64_t *q_pos, int64_t R, const floa
                      int nthreads) {
     return oracle_attention_ex(q, q_pos, R, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal,
                                -1, -1, NULL, 0, 0, 0, nthreads);
+}
+
+/*
+ * Gradients of the attention forward pass -- TEST INFRASTRUCTURE ONLY.
+ *
+ * The pages mention training only to say that back-propagation has to keep
+ * the gradients (hwcomputing.csdn.net page, section "标准Attention：一次摊开整本
+ * 词典").  Reading: the backward pass is the exact gradient of the operation
+ * above, O = softmax(scale * Q K^T) V (causal: keys j <= i only), for a given
+ * upstream gradient dO.  Written out by the chain rule, per query row i of one
+ * head, in double precision, with P recomputed here from Q and K:
+ *
+ *   P_ij   = exp(scale * q_i . k_j - LSE_i)          (the forward softmax)
+ *   dV_j  += P_ij dO_i
+ *   dP_ij  = dO_i . v_j
+ *   Delta_i = sum_j P_ij dP_ij                        (= dO_i . O_i)
+ *   dS_ij  = P_ij (dP_ij - Delta_i)
+ *   dQ_i   = scale * sum_j dS_ij k_j
+ *   dK_j  += scale * dS_ij q_i
+ *
+ * GQA: dK and dV of a key/value head sum over the query heads of its group.
+ * All arrays are float32 inputs (rounded values) and float64 outputs:
+ * q, dout [B, Hq, Nq, D]; k, v [B, Hkv, Nk, D]; dq [B, Hq, Nq, D];
+ * dk, dv [B, Hkv, Nk, D]; delta [B, Hq, Nq] (may be NULL).
+ * Returns 0, or a negative number for invalid arguments.
+ */
+int oracle_attention_bwd(const float *q, const float *k, const float *v, const float *dout,
+                         double *dq, double *dk, double *dv, double *delta, int64_t B,
+                         int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
+                         double scale, int causal, int nthreads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || D < 1) return -2;
+    if (Hq % Hkv != 0) return -3;
+    const int64_t group = Hq / Hkv;
+    int err = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    /* one (b, kv head) per task: its dK and dV rows are written by that task only */
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)Nk);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)Nk);
+        if (!p || !dp) {
+#pragma omp atomic write
+            err = -6;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bk = 0; bk < B * Hkv; ++bk) {
+            if (!p || !dp) continue;
+            const int64_t b = bk / Hkv, kvh = bk % Hkv;
+            const float *kb = k + bk * Nk * D;
+            const float *vb = v + bk * Nk * D;
+            double *dkb = dk + bk * Nk * D;
+            double *dvb = dv + bk * Nk * D;
+            for (int64_t x = 0; x < Nk * D; ++x) dkb[x] = dvb[x] = 0.0;
+            for (int64_t hq = kvh * group; hq < (kvh + 1) * group; ++hq) {
+                const int64_t bh = b * Hq + hq;
+                for (int64_t i = 0; i < Nq; ++i) {
+                    const float *qi = q + (bh * Nq + i) * D;
+                    const float *gi = dout + (bh * Nq + i) * D;
+                    double *dqi = dq + (bh * Nq + i) * D;
+                    const int64_t n_vis = causal ? (i + 1 < Nk ? i + 1 : Nk) : Nk;
+                    /* forward softmax of the row */
+                    double M = -INFINITY;
+                    for (int64_t j = 0; j < n_vis; ++j) {
+                        double acc = 0.0;
+                        for (int64_t d = 0; d < D; ++d) acc += (double)qi[d] * (double)kb[j * D + d];
+                        p[j] = scale * acc;
+                        if (p[j] > M) M = p[j];
+                    }
+                    double Z = 0.0;
+                    for (int64_t j = 0; j < n_vis; ++j) {
+                        p[j] = exp(p[j] - M);
+                        Z += p[j];
+                    }
+                    for (int64_t j = 0; j < n_vis; ++j) p[j] /= Z;
+                    /* dP, Delta */
+                    double dl = 0.0;
+                    for (int64_t j = 0; j < n_vis; ++j) {
+                        double acc = 0.0;
+                        for (int64_t d = 0; d < D; ++d) acc += (double)gi[d] * (double)vb[j * D + d];
+                        dp[j] = acc;
+                        dl += p[j] * acc;
+                    }
+                    if (delta) delta[bh * Nq + i] = dl;
+                    /* dS, then the three gradients */
+                    for (int64_t d = 0; d < D; ++d) dqi[d] = 0.0;
+                    for (int64_t j = 0; j < n_vis; ++j) {
+                        const double ds = p[j] * (dp[j] - dl);
+                        for (int64_t d = 0; d < D; ++d) {
+                            dqi[d] += scale * ds * (double)kb[j * D + d];
+                            dkb[j * D + d] += scale * ds * (double)qi[d];
+                            dvb[j * D + d] += p[j] * (double)gi[d];
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(dp);
+    }
+    return err;
 }
 
 int oracle_max_threads(void) {

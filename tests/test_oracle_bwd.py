@@ -1,0 +1,131 @@
+"""Pins for the oracle's gradients (CPU only).
+
+The backward oracle (``oracle_attention_bwd``) writes out the chain rule for
+O = softmax(scale * Q K^T) V.  It is pinned against things that do not come
+from its own formulas, so that a dropped scale, a missing Delta, a transposed
+operand, a wrong GQA sum or a causal off-by-one fails at least one test:
+
+* central finite differences of L = sum(dO * O) in float64 (the forward used
+  there is checked against the forward oracle first);
+* torch autograd through scaled_dot_product_attention in float64 on the CPU;
+* invariants: the key-sum of dK is zero, the key-sum of dV is the query-sum of
+  dO, Delta = dO . O; scale 0 and a single key give dQ = dK = 0;
+* GQA equals repeated K/V heads with dK, dV summed over each group.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+
+def _rand(shape, seed, scale=1.0):
+    return (scale * np.random.default_rng(seed).standard_normal(shape)).astype(np.float32)
+
+
+def _forward64(q, k, v, scale, causal):
+    """softmax(scale q k^T) v in float64 (numpy), GQA by repeating K/V heads."""
+    g = q.shape[1] // k.shape[1]
+    kr, vr = np.repeat(k, g, axis=1), np.repeat(v, g, axis=1)
+    s = scale * np.einsum("bhid,bhjd->bhij", q, kr)
+    if causal:
+        i, j = np.meshgrid(np.arange(q.shape[2]), np.arange(k.shape[2]), indexing="ij")
+        s = np.where(j <= i, s, -np.inf)
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=-1, keepdims=True)
+    return np.einsum("bhij,bhjd->bhid", p, vr)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_forward64_matches_oracle(causal):
+    q, k, v = _rand((1, 4, 7, 5), 1), _rand((1, 2, 9, 5), 2), _rand((1, 2, 9, 5), 3)
+    o, _ = oracle.attention(q, k, v, 0.6, causal)
+    np.testing.assert_allclose(_forward64(q.astype(np.float64), k.astype(np.float64),
+                                          v.astype(np.float64), 0.6, causal), o, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_finite_differences(causal):
+    q, k, v = _rand((1, 2, 5, 3), 4), _rand((1, 1, 6, 3), 5), _rand((1, 1, 6, 3), 6)
+    g = _rand((1, 2, 5, 3), 7)
+    scale = 0.8
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, scale, causal)
+    x = [q.astype(np.float64), k.astype(np.float64), v.astype(np.float64)]
+    h = 1e-5
+
+    def loss(xs):
+        return float(np.sum(g.astype(np.float64) * _forward64(*xs, scale, causal)))
+
+    for which, grad in enumerate((dq, dk, dv)):
+        fd = np.zeros_like(grad)
+        for idx in np.ndindex(*grad.shape):
+            xp = [a.copy() for a in x]
+            xm = [a.copy() for a in x]
+            xp[which][idx] += h
+            xm[which][idx] -= h
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * h)
+        np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal,nq,nk,hq,hkv", [(False, 33, 47, 4, 2), (True, 40, 40, 2, 2),
+                                                 (True, 25, 31, 6, 1), (False, 1, 17, 2, 1)])
+def test_against_torch_autograd(causal, nq, nk, hq, hkv):
+    q, k, v = _rand((2, hq, nq, 16), 8), _rand((2, hkv, nk, 16), 9), _rand((2, hkv, nk, 16), 10)
+    g = _rand((2, hq, nq, 16), 11)
+    dq, dk, dv, delta = oracle.attention_bwd(q, k, v, g, 0.3, causal)
+    qt, kt, vt = (torch.from_numpy(a).double().requires_grad_() for a in (q, k, v))
+    grp = hq // hkv
+    o = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt.repeat_interleave(grp, dim=1), vt.repeat_interleave(grp, dim=1), is_causal=causal,
+        scale=0.3)
+    o.backward(torch.from_numpy(g).double())
+    np.testing.assert_allclose(dq, qt.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(delta, (g.astype(np.float64) * o.detach().numpy()).sum(-1),
+                               rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sum_invariants(causal):
+    q, k, v = _rand((2, 4, 20, 8), 12), _rand((2, 2, 24, 8), 13), _rand((2, 2, 24, 8), 14)
+    g = _rand((2, 4, 20, 8), 15)
+    _, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.5, causal)
+    # every row of dS sums to zero -> the key-sum of dK vanishes
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+    # every row of P sums to one -> the key-sum of dV is the query-sum of dO over the group
+    want = g.astype(np.float64).reshape(2, 2, 2, 20, 8).sum(axis=(2, 3))
+    np.testing.assert_allclose(dv.sum(axis=2), want, rtol=1e-12, atol=1e-12)
+
+
+def test_scale_zero_and_single_key():
+    q, k, v = _rand((1, 2, 6, 4), 16), _rand((1, 2, 9, 4), 17), _rand((1, 2, 9, 4), 18)
+    g = _rand((1, 2, 6, 4), 19)
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.0, False)
+    assert np.all(dq == 0.0) and np.all(dk == 0.0)
+    np.testing.assert_allclose(dv, np.repeat(g.astype(np.float64).sum(axis=2, keepdims=True) / 9,
+                                             9, axis=2), rtol=1e-13, atol=1e-14)
+    dq, dk, dv, _ = oracle.attention_bwd(q, k[:, :, :1], v[:, :, :1], g, 0.7, False)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-13)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-13)
+    np.testing.assert_allclose(dv[:, :, 0], g.astype(np.float64).sum(axis=2), rtol=1e-13)
+
+
+def test_gqa_equals_repeated_kv():
+    q, k, v = _rand((1, 6, 11, 4), 20), _rand((1, 2, 13, 4), 21), _rand((1, 2, 13, 4), 22)
+    g = _rand((1, 6, 11, 4), 23)
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.4, True)
+    dq2, dk2, dv2, _ = oracle.attention_bwd(q, np.repeat(k, 3, axis=1), np.repeat(v, 3, axis=1), g,
+                                            0.4, True)
+    np.testing.assert_allclose(dq, dq2, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(dk, dk2.reshape(1, 2, 3, 13, 4).sum(axis=2), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(1, 2, 3, 13, 4).sum(axis=2), rtol=1e-12, atol=1e-13)
+
+
+def test_delta_is_dout_dot_output():
+    q, k, v = _rand((1, 2, 15, 8), 24), _rand((1, 2, 15, 8), 25), _rand((1, 2, 15, 8), 26)
+    g = _rand((1, 2, 15, 8), 27)
+    _, _, _, delta = oracle.attention_bwd(q, k, v, g, 0.5, True)
+    o, _ = oracle.attention(q, k, v, 0.5, True)
+    np.testing.assert_allclose(delta, (g.astype(np.float64) * o).sum(-1), rtol=1e-12, atol=1e-13)
