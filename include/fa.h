@@ -72,7 +72,8 @@ enum fa_status {
   FA_ERR_DEVICE_TIMEOUT = 11,      /* (device status) a kernel wait hit its limit  */
   FA_ERR_OVERLAP = 12,             /* o or lse overlaps q, k or v                  */
   FA_ERR_SCRATCH_TOO_SMALL = 13,   /* fa_fwd_noalloc: static scratch too small     */
-  FA_ERR_BAD_WINDOW = 14           /* fa_fwd_window: bound < -1, or causal + right > 0 */
+  FA_ERR_BAD_WINDOW = 14,          /* fa_fwd_window: bound < -1, or causal + right > 0 */
+  FA_ERR_BAD_WORKSPACE = 15        /* fa_bwd: workspace NULL or too small          */
 };
 
 /*
@@ -144,6 +145,37 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *l
                   int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
                   int window_left, int window_right, void *stream, int dtype, void *workspace,
                   size_t workspace_bytes);
+
+/*
+ * Backward pass: the gradients of the attention above for an upstream gradient
+ * dout (the pages mention only that training keeps gradients -- hwcomputing.
+ * csdn.net page, section on standard attention; the operation is taken as the
+ * exact gradient of O = softmax(scale Q K^T) V):
+ *   P = exp(scale Q K^T - LSE), dV = P^T dO, dP = dO V^T, Delta = rowsum(dO * O),
+ *   dS = P * (dP - Delta), dQ = scale dS K, dK = scale dS^T Q
+ * (causal: keys j <= i as in the forward pass; GQA: dK, dV sum over the query
+ * heads of each group).  P is recomputed from q, k and the forward pass's lse,
+ * never stored.
+ *   q, k, v, o  the forward pass's inputs and output (layout as fa_fwd);
+ *   dout        [B, Hq, Nq, D] upstream gradient, same dtype;
+ *   lse         [B, Hq, Nq] float32 from the forward pass (natural log);
+ *   dq          [B, Hq, Nq, D];  dk, dv  [B, Hkv, Nk, D]  outputs, same dtype;
+ *   workspace   device scratch of at least fa_bwd_workspace_size(B, Hq, Nq)
+ *               bytes, 256-byte aligned, caller-owned (Delta and lse * log2 e,
+ *               padded to 128-row blocks; no zero-fill needed); else
+ *               FA_ERR_BAD_WORKSPACE / FA_ERR_MISALIGNED.
+ * D must be 64 or 128 (else FA_ERR_UNSUPPORTED_HEAD_DIM).  Outputs and the
+ * workspace may not overlap any input or each other (FA_ERR_OVERLAP).  Three
+ * kernels on `stream` (Delta, dK and dV, dQ); asynchronous; deterministic (no
+ * atomics).  Other errors as fa_fwd.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk,
+           int D, float scale, int causal, void *stream, int dtype, void *workspace,
+           size_t workspace_bytes);
+
+/* Workspace bytes fa_bwd needs: 8 * B * Hq * (Nq rounded up to 128); 0 for bad sizes. */
+size_t fa_bwd_workspace_size(int B, int Hq, int Nq);
 
 /*
  * fa_fwd_ws for callers that cannot allocate device memory.  The pages have no

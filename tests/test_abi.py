@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 15):
+    for code in range(0, 16):
         s = fa.status_string(code)
         assert s and s != "unknown status", code
     assert fa.status_string(99) == "unknown status"

@@ -1,0 +1,98 @@
+"""GPU parity of the backward pass (fa_bwd) against the float64 gradient oracle.
+
+The forward pass runs on the GPU first (its O and LSE feed fa_bwd, as in
+training); the oracle computes the exact gradients from Q, K, V and dO alone.
+Tolerance (no stated bound for gradients): P and dS are rounded to the input
+dtype before their MMAs and each output is rounded once, each a relative error
+of about one unit roundoff u of the dtype (fp16 2^-11, bf16 2^-8) against the
+gradient's scale, so max |got - ref| <= 4 u G per tensor, where G is the larger
+of that tensor's max |ref| and dV's (dQ and dK can cancel to exactly zero --
+one key -- while the terms they sum keep the scale of dV).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tiled_attention_15_b200 as fa
+from fa_inputs import Workload, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+U = {"fp16": 2.0 ** -11, "bf16": 2.0 ** -8}
+
+
+def _dout(w):
+    g = np.random.default_rng(w.seed + 1000).standard_normal((w.B, w.Hq, w.Nq, w.D)).astype(np.float32)
+    return torch.from_numpy(g).to(torch.float16 if w.dtype == "fp16" else torch.bfloat16)
+
+
+def _run(w, dev):
+    q, k, v = make_qkv(w)
+    g = _dout(w)
+    qd, kd, vd, gd = (x.to(dev) for x in (q, k, v, g))
+    o, lse = fa.fa_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal)
+    dq, dk, dv = fa.fa_bwd(qd, kd, vd, o, lse, gd, scale=w.softmax_scale, causal=w.causal)
+    torch.cuda.synchronize()
+    assert fa.device_status(reset=True) == 0
+    return (q, k, v, g), (dq, dk, dv)
+
+
+def _check(w, got, ref, tag=""):
+    report = os.environ.get("FA_PARITY_REPORT")
+    rows = {}
+    for name, a, b in zip(("dQ", "dK", "dV"), got, ref):
+        a = a.float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(a).all(), name
+        scale = np.abs(b).max()
+        err = np.abs(a - b).max()
+        rows[name] = (err, scale)
+    if report:
+        with open(report, "a") as f:
+            f.write(json.dumps({"case": "bwd " + w.name + tag, "dtype": w.dtype,
+                                **{f"max_abs_d{n}": float(e) for n, (e, _) in rows.items()},
+                                **{f"max_ref_{n}": float(s) for n, (_, s) in rows.items()}}) + "\n")
+    for name, (err, scale) in rows.items():
+        g = max(scale, rows["dV"][1])
+        assert err <= 4 * U[w.dtype] * g, f"{w.name} {name}: {err:.3e} > 4u * {g:.3e}"
+
+
+CASES = [
+    Workload("bwd tiny D64 fp16", 1, 2, 2, 256, 256, 64, "fp16", False, seed=91),
+    Workload("bwd D128 fp16 causal ragged GQA", 1, 4, 2, 700, 700, 128, "fp16", True, seed=92),
+    Workload("bwd D128 bf16 Nq<Nk GQA 4", 1, 8, 2, 300, 1000, 128, "bf16", False, seed=93),
+    Workload("bwd D64 bf16 causal Nk<Nq", 2, 2, 1, 1000, 600, 64, "bf16", True, seed=94),
+    Workload("bwd D128 fp16 causal Nk>Nq", 1, 2, 2, 300, 1000, 128, "fp16", True, seed=95),
+    Workload("bwd single row and key", 1, 3, 1, 1, 1, 128, "fp16", False, seed=96),
+    Workload("bwd D64 fp16 odd sizes", 2, 3, 3, 129, 255, 64, "fp16", False, seed=97),
+    Workload("bwd D128 fp16 N2048 causal", 1, 4, 4, 2048, 2048, 128, "fp16", True, seed=98),
+    Workload("bwd D128 bf16 N2048", 1, 4, 4, 2048, 2048, 128, "bf16", False, seed=99),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_bwd_parity(cuda_dev, w):
+    (q, k, v, g), got = _run(w, cuda_dev)
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, w.softmax_scale, w.causal)
+    _check(w, got, (dq, dk, dv))
+
+
+def test_bwd_deterministic(cuda_dev):
+    w = Workload("bwd det", 1, 4, 2, 500, 640, 128, "bf16", True, seed=100)
+    _, a = _run(w, cuda_dev)
+    _, b = _run(w, cuda_dev)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_bwd_sum_invariants_on_device(cuda_dev):
+    # the key-sum of dK vanishes and the key-sum of dV is the query-sum of dO
+    w = Workload("bwd sums", 1, 2, 2, 512, 512, 64, "fp16", False, seed=101)
+    (q, k, v, g), (dq, dk, dv) = _run(w, cuda_dev)
+    s_dv = dv.double().sum(dim=2).cpu().numpy()
+    want = g.double().sum(dim=2).numpy()
+    np.testing.assert_allclose(s_dv, want, rtol=0, atol=0.05 * np.abs(want).max())
+    assert np.abs(dk.double().sum(dim=2).cpu().numpy()).max() <= 0.02 * np.abs(dk.double().cpu().numpy()).sum(2).max()

@@ -22,10 +22,11 @@ FA_FP16, FA_BF16 = 0, 1
 FA_OK = 0
 FA_ERR_DEVICE_TIMEOUT = 11
 FA_ERR_BAD_WINDOW = 14
+FA_ERR_BAD_WORKSPACE = 15
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
-            "fa_fwd_window",
+            "fa_fwd_window", "fa_bwd", "fa_bwd_workspace_size",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
             "fa_status_string", "fa_device_status", "fa_device_timeout_site",
             "fa_debug_exp2_fma", "fa_debug_wait_timeout", "fa_fwd_num_tiles")
@@ -60,6 +61,10 @@ def load_library() -> ctypes.CDLL:
     lib.fa_fwd_ws.restype = i
     lib.fa_fwd_window.argtypes = fwd_args[:13] + [i, i, vp, i, vp, ctypes.c_size_t]
     lib.fa_fwd_window.restype = i
+    lib.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, vp, i, vp, ctypes.c_size_t]
+    lib.fa_bwd.restype = i
+    lib.fa_bwd_workspace_size.argtypes = [i, i, i]
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_fwd_noalloc.argtypes = fwd_args + [i]
     lib.fa_fwd_noalloc.restype = i
     lib.fa_fwd_noalloc_scratch_bytes.argtypes = []
@@ -210,3 +215,53 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd")
     return o, lse
+
+
+def fa_bwd(q, k, v, o, lse, dout, scale: Optional[float] = None, causal: bool = False,
+           dq=None, dk=None, dv=None, stream=None, workspace=None):
+    """Gradients of the attention forward pass (three kernels on the current stream).
+
+    q, o, dout: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] contiguous CUDA tensors of
+    one dtype (fp16 or bf16); lse: float32 [B, Hq, Nq] from fa_fwd.  D must be
+    64 or 128.  Optional outputs dq (like q), dk, dv (like k); optional
+    workspace: a uint8 CUDA tensor of at least fa_bwd_workspace_size bytes
+    (allocated here when None).  Returns (dq, dk, dv).
+    """
+    import torch
+
+    lib = load_library()
+    if q.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("q, k, v must be float16 or bfloat16")
+    for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} must have the dtype of q")
+    if lse.dtype != torch.float32:
+        raise TypeError("lse must be float32")
+    B, Hq, Nq, D = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if o.shape != q.shape or dout.shape != q.shape or v.shape != k.shape or \
+            tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("expected q, o, dout [B,Hq,Nq,D], k, v [B,Hkv,Nk,D], lse [B,Hq,Nq]")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("lse", lse)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = int(lib.fa_bwd_workspace_size(B, Hq, Nq))
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    elif hasattr(stream, "cuda_stream"):
+        stream = stream.cuda_stream
+    dtype = FA_BF16 if q.dtype == torch.bfloat16 else FA_FP16
+    rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq,
+                    Nk, D, ctypes.c_float(scale), 1 if causal else 0, stream or None, dtype,
+                    workspace.data_ptr(), workspace.numel())
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd")
+    return dq, dk, dv

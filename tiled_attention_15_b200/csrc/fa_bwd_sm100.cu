@@ -1,0 +1,873 @@
+// fa_bwd_sm100.cu -- backward pass of the fused attention for B200 (sm_100a).
+//
+// The pages only say that training has to keep gradients (hwcomputing.csdn.net
+// page, section "标准Attention：一次摊开整本词典"); the operation here is the
+// exact gradient of the forward pass O = softmax(scale * Q K^T) V for an
+// upstream gradient dO, computed the way the forward pass is: tile by tile,
+// without materialising the score matrix.  The softmax is recomputed from Q, K
+// and the forward pass's row log-sum-exp (LSE):
+//
+//   P_ij  = exp(scale q_i.k_j - LSE_i)            Delta_i = dO_i . O_i
+//   dP_ij = dO_i . v_j                            dS_ij   = P_ij (dP_ij - Delta_i)
+//   dV_j  = sum_i P_ij dO_i     dK_j = scale sum_i dS_ij q_i     dQ_i = scale sum_j dS_ij k_j
+//
+// Three kernels, all with tcgen05 tensor-core MMAs accumulating in tensor
+// memory (TMEM) and TMA loads with 128-byte swizzle:
+//   * bwd_prep_kernel: Delta = rowsum(dO * O) and LSE * log2(e), into two planes
+//     padded to whole 128-row blocks (+inf / 0 in the padding, which zeroes P
+//     there without a mask);
+//   * bwd_dkdv_kernel: one 128-key tile per CTA; loops over the query blocks of
+//     every query head of its GQA group: S^T = K Q^T, dP^T = V dO^T,
+//     P^T and dS^T (16-bit, written back over S^T and dP^T), dV += P^T dO,
+//     dK += dS^T Q;
+//   * bwd_dq_kernel: one 128-query tile per CTA; loops over the key blocks:
+//     S = Q K^T, dP = dO V^T, dS, dQ += dS K.
+// dQ is computed in its own pass (S and dP recomputed: two extra MMAs per block
+// pair) instead of being accumulated across key tiles with atomics: no atomic
+// traffic, and the result does not depend on the order CTAs finish in.
+//
+// Warp roles (384 threads, one CTA per SM): warps 0-7 two compute warpgroups
+// that split each block's 128 columns into halves (warp w reads TMEM lanes
+// 32 (w % 4) .. +31), warp 8 issues the MMAs (one thread), warp 9 issues the
+// TMA loads (one thread), warps 10-11 idle.  Every mbarrier wait is bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa.h"
+#include "sm100_ptx.cuh"
+
+namespace fab {
+using namespace fa;
+
+constexpr int kBM = 128;  // query rows per block
+constexpr int kBN = 128;  // keys per block
+constexpr int kThreads = 384;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ unsigned int g_bwd_status = 0;
+__device__ unsigned long long g_bwd_site = 0;
+
+// 1-D bulk copy global -> shared, completion counted on `bar` in bytes (both
+// addresses 16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity,
+                                         volatile uint32_t* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      const uint32_t site =
+          0x80000000u | ((threadIdx.x >> 5) << 24) | ((bar & 0x3FFFFu) << 1) | parity;
+      atomicCAS(const_cast<uint32_t*>(abort_flag), 0u, site);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void publish_abort(uint32_t flag) {
+  if (flag == 0u) return;
+  if (atomicCAS(&g_bwd_status, 0u, static_cast<unsigned>(FA_ERR_DEVICE_TIMEOUT)) == 0u)
+    g_bwd_site = (static_cast<unsigned long long>(blockIdx.x) << 48) |
+                 (static_cast<unsigned long long>((flag >> 24) & 0x3Fu) << 40) |
+                 (static_cast<unsigned long long>((flag >> 1) & 0x3FFFFu) << 8) | (flag & 1u);
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b, bool bf16) {
+  if (bf16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 unpack2(uint32_t w, bool bf16) {
+  if (bf16) return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w));
+  return __half22float2(*reinterpret_cast<__half2*>(&w));
+}
+
+struct BwdParams {
+  void* dq;
+  void* dk;
+  void* dv;
+  const float* lse2;   // [B*Hq][Nq_pad] LSE * log2(e); +inf in the padding
+  const float* delta;  // [B*Hq][Nq_pad] rowsum(dO * O); 0 in the padding
+  int B, Hq, Hkv, Nq, Nk, Nq_pad, group, causal;
+  float c;      // scale * log2(e)
+  float scale;
+  int nqt, nkt;  // query / key blocks per head
+};
+
+// ------------------------------------------------------------------ Delta, LSE2
+// D / 8 threads per row, 8 elements (16 bytes) each; rows in the padding get
+// (+inf, 0).  Rows are taken warp by warp so that every lane of a warp reaches
+// the shuffles.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o,
+                                                       const uint16_t* __restrict__ dout,
+                                                       const float* __restrict__ lse,
+                                                       float* __restrict__ lse2,
+                                                       float* __restrict__ delta, int BH, int Nq,
+                                                       int Nq_pad) {
+  constexpr int TPR = D / 8;      // threads per row
+  constexpr int RPW = 32 / TPR;   // rows per warp
+  const long long total = static_cast<long long>(BH) * Nq_pad;
+  const int lane = threadIdx.x & 31, sub = lane % TPR;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long base = warp * RPW; base < total; base += n_warps * RPW) {
+    const long long row = base + lane / TPR;
+    const long long bh = row / Nq_pad;
+    const int i = static_cast<int>(row - bh * Nq_pad);
+    const bool live = row < total && i < Nq;
+    float acc = 0.f;
+    if (live) {
+      const size_t off = (static_cast<size_t>(bh) * Nq + i) * D + sub * 8;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + off));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + off));
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const float2 fa2 = unpack2(aw[x], BF16), fb2 = unpack2(bw[x], BF16);
+        acc = fmaf(fa2.x, fb2.x, acc);
+        acc = fmaf(fa2.y, fb2.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (sub == 0 && row < total) {
+      delta[row] = live ? acc : 0.f;
+      lse2[row] = live ? lse[bh * Nq + i] * kLog2e : INFINITY;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ shared pieces
+struct Ctx {
+  uint32_t sbase;
+  uint32_t tmem;
+  volatile uint32_t* abort_flag;
+  __device__ uint32_t bar(int i, int off_bar) const { return sbase + off_bar + 8u * i; }
+};
+
+// S-type MMA over one 128 x D by 128 x D pair of K-major SW128 tiles:
+// D[128 x 128] = A B^T.
+template <int D>
+__device__ __forceinline__ void mma_nt(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                       int chunk_a, int chunk_b) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off_a = ((kk >> 2) * chunk_a + (kk & 3) * 32) >> 4;
+    const uint32_t off_b = ((kk >> 2) * chunk_b + (kk & 3) * 32) >> 4;
+    mma_ss(d, a0 + off_a, b0 + off_b, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// Accumulating MMA with A (16-bit, 128 rows x 128 columns of K) in tensor
+// memory and B an MN-major SW128 tile (128 rows of K, D columns).  The packed A
+// of K index k sits at column acol(k / 16) + (k % 16) / 2.
+template <int D, typename ACol>
+__device__ __forceinline__ void mma_tn(uint32_t d, uint32_t a, uint64_t b0, uint32_t idesc,
+                                       bool acc, ACol acol) {
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk)
+    mma_ts(d, a + acol(kk), b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+           (acc || kk > 0) ? 1u : 0u);
+}
+
+// ================================================================== dK, dV
+template <int D>
+struct GeoKV {
+  static constexpr int DCH = D / 64;
+  static constexpr int T_BYTES = 128 * D * 2;  // one 128-row tile
+  static constexpr int CHUNK = 128 * 128;      // one 64-column chunk of a tile
+  static constexpr int NST = D == 64 ? 4 : 2;  // query-block stages (Q, dO, lse2, delta)
+  static constexpr int OFF_K = 0, OFF_V = T_BYTES, OFF_ST = 2 * T_BYTES;
+  static constexpr int ST_BYTES = 2 * T_BYTES + 2 * 512;
+  static constexpr int OFF_BAR = OFF_ST + NST * ST_BYTES;
+  // barriers
+  static constexpr int B_KV = 0, B_QF = 1, B_QE = 1 + NST, B_SF = 1 + 2 * NST, B_DPF = B_SF + 1,
+                       B_PF = B_SF + 2, B_DSF = B_SF + 3, B_ACC = B_SF + 4, NBAR = B_SF + 5;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // TMEM columns: S^T 0..127 (P^T over it), dP^T 128..255 (dS^T over it), dV, dK
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(256 + 2 * D <= 512, "tensor memory budget");
+};
+
+struct KVTile {
+  int bkv;  // b * Hkv + kv head
+  int kt;   // key block
+  int i0;   // first query block
+  int nb;   // blocks: group heads x query blocks
+};
+
+__device__ __forceinline__ KVTile kv_tile(const BwdParams& p) {
+  KVTile T;
+  const int BK = p.B * p.Hkv;
+  const int t = blockIdx.x;
+  if (p.causal) {  // small key blocks see the most query blocks: run them first
+    T.kt = t / BK;
+    T.bkv = t % BK;
+  } else {
+    T.bkv = t / p.nkt;
+    T.kt = t % p.nkt;
+  }
+  T.i0 = p.causal ? T.kt : 0;  // causal: query q sees keys <= q (top-left aligned)
+  T.nb = T.i0 < p.nqt ? p.group * (p.nqt - T.i0) : 0;
+  return T;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const BwdParams p) {
+  using G = GeoKV<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(gbase + G::OFF_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Ctx cx;
+  cx.sbase = sbase;
+  cx.abort_flag = misc + 1;
+  auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
+  const KVTile T = kv_tile(p);
+
+  if (threadIdx.x == 0) {
+    mbar_init(B(G::B_KV), 1);
+    for (int s = 0; s < G::NST; ++s) {
+      mbar_init(B(G::B_QF + s), 1);
+      mbar_init(B(G::B_QE + s), 1);
+    }
+    mbar_init(B(G::B_SF), 1);
+    mbar_init(B(G::B_DPF), 1);
+    mbar_init(B(G::B_PF), 8);
+    mbar_init(B(G::B_DSF), 8);
+    mbar_init(B(G::B_ACC), 1);
+    misc[1] = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(misc), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cx.tmem = misc[0];
+
+  // Registers: 208 for the two compute warpgroups, 88 for the rest (2 x 128 x
+  // 208 + 128 x 88 = 384 x 168); each role branch sets its own limit.
+  const int kv_row0 = T.kt * kBN;
+  if (warp >= 8) setmaxnreg_dec<88>();
+  if (warp == 9 && lane == 0 && T.nb > 0) {
+    // ---- TMA: K and V tiles once, then (Q, dO, lse2, delta) per query block
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_do);
+    const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
+    mbar_arrive_expect_tx(B(G::B_KV), 2 * G::T_BYTES);
+#pragma unroll
+    for (int c = 0; c < G::DCH; ++c) {
+      tma_load_3d(sbase + G::OFF_K + c * G::CHUNK, &tm_k, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
+      tma_load_3d(sbase + G::OFF_V + c * G::CHUNK, &tm_v, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
+    }
+    const int nqb = p.nqt - T.i0;
+    for (int n = 0; n < T.nb; ++n) {
+      const int st = n % G::NST;
+      if (n >= G::NST && !wait_bar(B(G::B_QE + st), ((n / G::NST) - 1) & 1u, cx.abort_flag)) break;
+      const int h = n / nqb, i = T.i0 + n % nqb;
+      const int bh = (T.bkv / p.Hkv) * p.Hq + (T.bkv % p.Hkv) * p.group + h;
+      const uint32_t sb = sbase + G::OFF_ST + st * G::ST_BYTES;
+      mbar_arrive_expect_tx(B(G::B_QF + st), 2 * G::T_BYTES + 1024);
+#pragma unroll
+      for (int c = 0; c < G::DCH; ++c) {
+        tma_load_3d(sb + c * G::CHUNK, &tm_q, B(G::B_QF + st), c * 64, i * kBM, bh, pol_last);
+        tma_load_3d(sb + G::T_BYTES + c * G::CHUNK, &tm_do, B(G::B_QF + st), c * 64, i * kBM, bh,
+                    pol_last);
+      }
+      const size_t row = static_cast<size_t>(bh) * p.Nq_pad + static_cast<size_t>(i) * kBM;
+      bulk_load(sb + 2 * G::T_BYTES, p.lse2 + row, 512, B(G::B_QF + st));
+      bulk_load(sb + 2 * G::T_BYTES + 512, p.delta + row, 512, B(G::B_QF + st));
+    }
+  } else if (warp == 8 && lane == 0 && T.nb > 0) {
+    // ---- MMA: S(0) dP(0) | dV(n) S(n+1) dK(n) dP(n+1) | ...
+    constexpr uint32_t kIdNT = idesc_f16(128, 128, BF16, false);
+    constexpr uint32_t kIdTN = idesc_f16(128, D, BF16, true);
+    const uint32_t tm = cx.tmem;
+    const uint64_t dk0 = sdesc_sw128(sbase + G::OFF_K, 16, 1024);
+    const uint64_t dv0 = sdesc_sw128(sbase + G::OFF_V, 16, 1024);
+    auto st_desc = [&](int st, int which, bool mn) {  // which: 0 = Q, 1 = dO
+      const uint32_t a = sbase + G::OFF_ST + st * G::ST_BYTES + which * G::T_BYTES;
+      return mn ? sdesc_sw128(a, G::CHUNK, 1024) : sdesc_sw128(a, 16, 1024);
+    };
+    // P^T / dS^T of query column q: warpgroup q / 64 packed its half at its own
+    // first 32 columns -> K step kk (16 queries) at (kk / 4) * 64 + (kk % 4) * 8
+    auto acol = [](int kk) { return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8); };
+    bool ok = wait_bar(B(G::B_KV), 0u, cx.abort_flag);
+    uint32_t qf_ph[G::NST] = {};
+    if (ok) ok = wait_bar(B(G::B_QF + 0), 0u, cx.abort_flag);
+    if (ok) {
+      qf_ph[0] ^= 1u;
+      tc_fence_after();
+      mma_nt<D>(tm + G::T_S, dk0, st_desc(0, 0, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_commit(B(G::B_SF));
+      mma_nt<D>(tm + G::T_DP, dv0, st_desc(0, 1, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_commit(B(G::B_DPF));
+    }
+    for (int n = 0; ok && n < T.nb; ++n) {
+      const int st = n % G::NST, st1 = (n + 1) % G::NST;
+      if (!wait_bar(B(G::B_PF), n & 1u, cx.abort_flag)) break;
+      tc_fence_after();
+      mma_tn<D>(tm + G::T_DV, tm + G::T_S, st_desc(st, 1, true), kIdTN, n > 0, acol);
+      if (n + 1 < T.nb) {
+        if (!wait_bar(B(G::B_QF + st1), qf_ph[st1], cx.abort_flag)) break;
+        qf_ph[st1] ^= 1u;
+        tc_fence_after();
+        mma_nt<D>(tm + G::T_S, dk0, st_desc(st1, 0, false), kIdNT, G::CHUNK, G::CHUNK);
+        mma_commit(B(G::B_SF));
+      }
+      if (!wait_bar(B(G::B_DSF), n & 1u, cx.abort_flag)) break;
+      tc_fence_after();
+      mma_tn<D>(tm + G::T_DK, tm + G::T_DP, st_desc(st, 0, true), kIdTN, n > 0, acol);
+      mma_commit(B(G::B_QE + st));
+      if (n + 1 < T.nb) {
+        mma_nt<D>(tm + G::T_DP, dv0, st_desc(st1, 1, false), kIdNT, G::CHUNK, G::CHUNK);
+        mma_commit(B(G::B_DPF));
+      } else {
+        mma_commit(B(G::B_ACC));
+      }
+    }
+  } else if (warp < 8) {
+    // ---- compute: thread = key row r of the tile, warpgroup h = query columns h*64 .. +63
+    setmaxnreg_inc<208>();
+    const int h = warp >> 2, r = (warp & 3) * 32 + lane;
+    const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const float c = p.c;
+    const int nqb = p.nqt - T.i0;
+    uint32_t qf_ph[G::NST] = {};
+    bool ok = true;
+    for (int n = 0; ok && n < T.nb; ++n) {
+      const int st = n % G::NST;
+      const int i = T.i0 + n % nqb;
+      // lse2 / delta of this block were written by the TMA unit: observe its barrier
+      ok = wait_bar(B(G::B_QF + st), qf_ph[st], cx.abort_flag) &&
+           wait_bar(B(G::B_SF), n & 1u, cx.abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      qf_ph[st] ^= 1u;
+      tc_fence_after();
+      const float* l2 = reinterpret_cast<const float*>(gbase + G::OFF_ST + st * G::ST_BYTES +
+                                                       2 * G::T_BYTES) + h * 64;
+      const float* dl = l2 + 128;
+      uint32_t sr[64];
+      tmem_ld_x64(tm + G::T_S + h * 64, sr);
+      // causal: only the diagonal block masks (key k0 + r > query q0 + col <=> r > col)
+      const bool diag = p.causal && i == T.kt;
+      float pv[64];
+#pragma unroll
+      for (int x = 0; x < 64; x += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(l2 + x);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float e2 = ex2(fmaf(__uint_as_float(sr[x + e]), c, -lv[e]));
+          pv[x + e] = (diag && r > h * 64 + x + e) ? 0.f : e2;
+        }
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x) pk[x] = pack2(pv[2 * x], pv[2 * x + 1], BF16);
+      tmem_st_x32(tm + G::T_S + h * 64, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_PF));
+
+      ok = wait_bar(B(G::B_DPF), n & 1u, cx.abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t dr[64];
+      tmem_ld_x64(tm + G::T_DP + h * 64, dr);
+#pragma unroll
+      for (int x = 0; x < 64; x += 4) {
+        const float4 d4 = *reinterpret_cast<const float4*>(dl + x);
+        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pv[x + e] *= __uint_as_float(dr[x + e]) - dv4[e];
+      }
+#pragma unroll
+      for (int x = 0; x < 32; ++x) pk[x] = pack2(pv[2 * x], pv[2 * x + 1], BF16);
+      tmem_st_x32(tm + G::T_DP + h * 64, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_DSF));
+    }
+    // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale)
+    const int key = kv_row0 + r;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
+                    (static_cast<size_t>(T.bkv) * p.Nk + (key < p.Nk ? key : 0)) * D;
+    const float mul = h == 0 ? 1.f : p.scale;
+    if (T.nb == 0) {  // no query sees these keys: zero gradients
+      if (key < p.Nk)
+        for (int c0 = 0; c0 < D; c0 += 8) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(0, 0, 0, 0);
+    } else if (ok) {
+      ok = wait_bar(B(G::B_ACC), 0u, cx.abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t a[32];
+          tmem_ld_x32(tm + (h == 0 ? G::T_DV : G::T_DK) + c0, a);
+          uint32_t w[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            w[x] = pack2(__uint_as_float(a[2 * x]) * mul, __uint_as_float(a[2 * x + 1]) * mul, BF16);
+          if (key < p.Nk) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*cx.abort_flag) {  // let issued copies and MMAs land before tensor memory is freed
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) {
+    }
+  }
+  if (threadIdx.x == 0) publish_abort(*cx.abort_flag);
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(cx.tmem, 512);
+  }
+}
+
+// ================================================================== dQ
+template <int D>
+struct GeoQ {
+  static constexpr int DCH = D / 64;
+  static constexpr int T_BYTES = 128 * D * 2;
+  static constexpr int CHUNK = 128 * 128;
+  static constexpr int NST = D == 64 ? 4 : 2;  // key-block stages (K, V)
+  static constexpr int OFF_Q = 0, OFF_DO = T_BYTES, OFF_ST = 2 * T_BYTES;
+  static constexpr int ST_BYTES = 2 * T_BYTES;
+  static constexpr int OFF_BAR = OFF_ST + NST * ST_BYTES;
+  static constexpr int B_QF = 0, B_KF = 1, B_KE = 1 + NST, B_SDP = 1 + 2 * NST, B_SFREE = B_SDP + 1,
+                       B_DSF = B_SDP + 2, B_DSE = B_SDP + 3, B_DQF = B_SDP + 4, NBAR = B_SDP + 5;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // TMEM columns: S 0..127, dP 128..255, dS (packed) 256..319, dQ 320..320+D-1
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DS = 256, T_DQ = 320;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(320 + D <= 512, "tensor memory budget");
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const BwdParams p) {
+  using G = GeoQ<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(gbase + G::OFF_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Ctx cx;
+  cx.sbase = sbase;
+  cx.abort_flag = misc + 1;
+  auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
+
+  // tile: (b, hq, query block); causal: the last query blocks (most keys) first
+  const int BH = p.B * p.Hq, t = blockIdx.x;
+  int bh, qt;
+  if (p.causal) {
+    qt = p.nqt - 1 - t / BH;
+    bh = t % BH;
+  } else {
+    bh = t / p.nqt;
+    qt = t % p.nqt;
+  }
+  const int q0 = qt * kBM;
+  const int kvz = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
+  const int nkb = (p.Nk + kBN - 1) / kBN;
+  const int nb = p.causal ? min(nkb, (min(q0 + kBM, p.Nq) - 1) / kBN + 1) : nkb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(B(G::B_QF), 1);
+    for (int s = 0; s < G::NST; ++s) {
+      mbar_init(B(G::B_KF + s), 1);
+      mbar_init(B(G::B_KE + s), 1);
+    }
+    mbar_init(B(G::B_SDP), 1);
+    mbar_init(B(G::B_SFREE), 8);
+    mbar_init(B(G::B_DSF), 8);
+    mbar_init(B(G::B_DSE), 1);
+    mbar_init(B(G::B_DQF), 1);
+    misc[1] = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(misc), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cx.tmem = misc[0];
+
+  if (warp >= 8) setmaxnreg_dec<88>();
+  if (warp == 9 && lane == 0) {
+    // ---- TMA: Q and dO once, then (K_j, V_j) per key block
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
+    mbar_arrive_expect_tx(B(G::B_QF), 2 * G::T_BYTES);
+#pragma unroll
+    for (int c = 0; c < G::DCH; ++c) {
+      tma_load_3d(sbase + G::OFF_Q + c * G::CHUNK, &tm_q, B(G::B_QF), c * 64, q0, bh, pol_first);
+      tma_load_3d(sbase + G::OFF_DO + c * G::CHUNK, &tm_do, B(G::B_QF), c * 64, q0, bh, pol_first);
+    }
+    for (int j = 0; j < nb; ++j) {
+      const int st = j % G::NST;
+      if (j >= G::NST && !wait_bar(B(G::B_KE + st), ((j / G::NST) - 1) & 1u, cx.abort_flag)) break;
+      const uint32_t sb = sbase + G::OFF_ST + st * G::ST_BYTES;
+      mbar_arrive_expect_tx(B(G::B_KF + st), 2 * G::T_BYTES);
+#pragma unroll
+      for (int c = 0; c < G::DCH; ++c) {
+        tma_load_3d(sb + c * G::CHUNK, &tm_k, B(G::B_KF + st), c * 64, j * kBN, kvz, pol_last);
+        tma_load_3d(sb + G::T_BYTES + c * G::CHUNK, &tm_v, B(G::B_KF + st), c * 64, j * kBN, kvz,
+                    pol_last);
+      }
+    }
+  } else if (warp == 8 && lane == 0) {
+    // ---- MMA: S(0) dP(0) | S(j+1) dP(j+1) dQ(j) | ...
+    constexpr uint32_t kIdNT = idesc_f16(128, 128, BF16, false);
+    constexpr uint32_t kIdTN = idesc_f16(128, D, BF16, true);
+    const uint32_t tm = cx.tmem;
+    const uint64_t dq0 = sdesc_sw128(sbase + G::OFF_Q, 16, 1024);
+    const uint64_t ddo0 = sdesc_sw128(sbase + G::OFF_DO, 16, 1024);
+    auto kv_desc = [&](int st, int which, bool mn) {  // which: 0 = K, 1 = V
+      const uint32_t a = sbase + G::OFF_ST + st * G::ST_BYTES + which * G::T_BYTES;
+      return mn ? sdesc_sw128(a, G::CHUNK, 1024) : sdesc_sw128(a, 16, 1024);
+    };
+    // dS of key column k: warpgroup k / 64 packed its half at columns (k / 64) * 32 ..
+    auto acol = [](int kk) { return static_cast<uint32_t>(kk * 8); };
+    uint32_t kf_ph[G::NST] = {};
+    bool ok = wait_bar(B(G::B_QF), 0u, cx.abort_flag);
+    if (ok) ok = wait_bar(B(G::B_KF + 0), 0u, cx.abort_flag);
+    if (ok) {
+      kf_ph[0] ^= 1u;
+      tc_fence_after();
+      mma_nt<D>(tm + G::T_S, dq0, kv_desc(0, 0, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_nt<D>(tm + G::T_DP, ddo0, kv_desc(0, 1, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_commit(B(G::B_SDP));
+    }
+    for (int j = 0; ok && j < nb; ++j) {
+      const int st = j % G::NST, st1 = (j + 1) % G::NST;
+      if (j + 1 < nb) {  // next S and dP once the compute warps have read this block's
+        if (!wait_bar(B(G::B_SFREE), j & 1u, cx.abort_flag)) break;
+        if (!wait_bar(B(G::B_KF + st1), kf_ph[st1], cx.abort_flag)) break;
+        kf_ph[st1] ^= 1u;
+        tc_fence_after();
+        mma_nt<D>(tm + G::T_S, dq0, kv_desc(st1, 0, false), kIdNT, G::CHUNK, G::CHUNK);
+        mma_nt<D>(tm + G::T_DP, ddo0, kv_desc(st1, 1, false), kIdNT, G::CHUNK, G::CHUNK);
+        mma_commit(B(G::B_SDP));
+      }
+      if (!wait_bar(B(G::B_DSF), j & 1u, cx.abort_flag)) break;
+      tc_fence_after();
+      mma_tn<D>(tm + G::T_DQ, tm + G::T_DS, kv_desc(st, 0, true), kIdTN, j > 0, acol);
+      mma_commit(B(G::B_DSE));
+      mma_commit(B(G::B_KE + st));
+      if (j + 1 == nb) mma_commit(B(G::B_DQF));
+    }
+  } else if (warp < 8) {
+    // ---- compute: thread = query row r, warpgroup h = key columns h*64 .. +63
+    setmaxnreg_inc<208>();
+    const int h = warp >> 2, r = (warp & 3) * 32 + lane;
+    const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const float c = p.c;
+    const size_t srow = static_cast<size_t>(bh) * p.Nq_pad + q0 + r;
+    const float lse2 = p.lse2[srow], dlt = p.delta[srow];
+    const int qpos = q0 + r;
+    bool ok = true;
+    for (int j = 0; ok && j < nb; ++j) {
+      ok = wait_bar(B(G::B_SDP), j & 1u, cx.abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t sr[64], dr[64];
+      tmem_ld_x64(tm + G::T_S + h * 64, sr);
+      tmem_ld_x64(tm + G::T_DP + h * 64, dr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_SFREE));
+      // visible keys of this row in the block: [0, lim)
+      const int kbase = j * kBN + h * 64;
+      int lim = p.Nk - kbase;
+      if (p.causal) lim = min(lim, qpos - kbase + 1);
+      uint32_t pk[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x) {
+        float v2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 2 * x + e;
+          const float pe = ex2(fmaf(__uint_as_float(sr[i]), c, -lse2));
+          v2[e] = i < lim ? pe * (__uint_as_float(dr[i]) - dlt) : 0.f;
+        }
+        pk[x] = pack2(v2[0], v2[1], BF16);
+      }
+      if (j > 0) {  // dQ(j-1) has read the previous dS
+        ok = wait_bar(B(G::B_DSE), (j - 1) & 1u, cx.abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+      }
+      tmem_st_x32(tm + G::T_DS + h * 32, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_DSF));
+    }
+    // ---- epilogue: dQ = scale * acc, warpgroup h writes columns h * D/2 .. +D/2
+    if (ok && nb > 0) {
+      ok = wait_bar(B(G::B_DQF), 0u, cx.abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) +
+                        (static_cast<size_t>(bh) * p.Nq + (qpos < p.Nq ? qpos : 0)) * D;
+#pragma unroll 1
+        for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 32) {
+          uint32_t a[32];
+          tmem_ld_x32(tm + G::T_DQ + c0, a);
+          uint32_t w[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            w[x] = pack2(__uint_as_float(a[2 * x]) * p.scale, __uint_as_float(a[2 * x + 1]) * p.scale,
+                         BF16);
+          if (qpos < p.Nq) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*cx.abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) {
+    }
+  }
+  if (threadIdx.x == 0) publish_abort(*cx.abort_flag);
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(cx.tmem, 512);
+  }
+}
+
+}  // namespace fab
+
+// ============================================================================ host side
+namespace {
+
+using EncodeTiledFnB = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFnB encode_fn_b() {
+  static EncodeTiledFnB fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFnB>(f);
+  });
+  return fn;
+}
+
+// [Z][rows][D] 16-bit tensor, 64 x 128 boxes, 128-byte swizzle, zero fill out of range.
+bool map_rows(CUtensorMap* m, const void* ptr, int D, long long rows, long long Z, bool bf16) {
+  EncodeTiledFnB enc = encode_fn_b();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)Z};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  const cuuint32_t box[3] = {64u, 128u, 1u};
+  const cuuint32_t es[3] = {1u, 1u, 1u};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+             const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool overlaps_b(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int nq_pad(int Nq) { return (Nq + 127) / 128 * 128; }
+
+template <int D, bool BF16>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+               int Nk, float scale, int causal, cudaStream_t st, void* ws, int sms) {
+  using GK = fab::GeoKV<D>;
+  using GQ = fab::GeoQ<D>;
+  static std::once_flag once;
+  static bool attr_ok = false;
+  std::call_once(once, [] {
+    attr_ok = cudaFuncSetAttribute(fab::bwd_dkdv_kernel<D, BF16>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   GK::SMEM_BYTES) == cudaSuccess &&
+              cudaFuncSetAttribute(fab::bwd_dq_kernel<D, BF16>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   GQ::SMEM_BYTES) == cudaSuccess;
+  });
+  if (!attr_ok) return FA_ERR_LAUNCH;
+  CUtensorMap tq, tdo, tk, tv;
+  if (!map_rows(&tq, q, D, Nq, (long long)B * Hq, BF16) ||
+      !map_rows(&tdo, dout, D, Nq, (long long)B * Hq, BF16) ||
+      !map_rows(&tk, k, D, Nk, (long long)B * Hkv, BF16) ||
+      !map_rows(&tv, v, D, Nk, (long long)B * Hkv, BF16))
+    return FA_ERR_DRIVER;
+  fab::BwdParams p;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.Nq_pad = nq_pad(Nq);
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.c = scale * fab::kLog2e;
+  p.nqt = p.Nq_pad / 128;
+  p.nkt = (Nk + 127) / 128;
+  float* lse2 = static_cast<float*>(ws);
+  float* delta = lse2 + (size_t)B * Hq * p.Nq_pad;
+  p.lse2 = lse2;
+  p.delta = delta;
+  // 1. Delta and LSE * log2(e), padded
+  const long long rows = (long long)B * Hq * p.Nq_pad;
+  const long long warps_needed = (rows * (D / 8) + 31) / 32;
+  long long blocks = (warps_needed + 7) / 8;
+  if (blocks > 16LL * sms) blocks = 16LL * sms;
+  fab::bwd_prep_kernel<D, BF16><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, lse2, delta,
+      B * Hq, Nq, p.Nq_pad);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  // 2. dK, dV: one CTA per (b, kv head, key block)
+  fab::bwd_dkdv_kernel<D, BF16><<<(unsigned)(B * Hkv * p.nkt), fab::kThreads, GK::SMEM_BYTES, st>>>(
+      tq, tdo, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  // 3. dQ: one CTA per (b, query head, query block)
+  fab::bwd_dq_kernel<D, BF16><<<(unsigned)(B * Hq * p.nqt), fab::kThreads, GQ::SMEM_BYTES, st>>>(
+      tq, tdo, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_bwd_workspace_size(int B, int Hq, int Nq) {
+  if (B < 1 || Hq < 1 || Nq < 1) return 0;
+  return 2ull * (size_t)B * Hq * nq_pad(Nq) * sizeof(float);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+           int D, float scale, int causal, void* stream, int dtype, void* workspace,
+           size_t workspace_bytes) {
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_BAD_SHAPE;
+  if (Hq % Hkv != 0) return FA_ERR_BAD_GROUPING;
+  if ((long long)B * Hq * nq_pad(Nq) >= (1ll << 31) || (long long)B * Hkv * Nk >= (1ll << 31))
+    return FA_ERR_BAD_SHAPE;
+  if (!std::isfinite(scale)) return FA_ERR_BAD_SCALE;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_NULL_POINTER;
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o | (uintptr_t)dout |
+       (uintptr_t)dq | (uintptr_t)dk | (uintptr_t)dv) & 15u)
+    return FA_ERR_MISALIGNED;
+  if ((uintptr_t)lse & 3u) return FA_ERR_MISALIGNED;
+  if (workspace == nullptr || workspace_bytes < fa_bwd_workspace_size(B, Hq, Nq))
+    return FA_ERR_BAD_WORKSPACE;
+  if ((uintptr_t)workspace & 255u) return FA_ERR_MISALIGNED;
+  const size_t qb = (size_t)B * Hq * Nq * D * 2, kb = (size_t)B * Hkv * Nk * D * 2;
+  const size_t lb = (size_t)B * Hq * Nq * 4, wb = fa_bwd_workspace_size(B, Hq, Nq);
+  const void* ins[6] = {q, k, v, o, dout, lse};
+  const size_t in_b[6] = {qb, kb, kb, qb, qb, lb};
+  void* outs[4] = {dq, dk, dv, workspace};
+  const size_t out_b[4] = {qb, kb, kb, wb};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps_b(outs[a], out_b[a], ins[b], in_b[b])) return FA_ERR_OVERLAP;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps_b(outs[a], out_b[a], outs[b], out_b[b])) return FA_ERR_OVERLAP;
+  }
+  int dev = -1, major = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      major != 10 || sms < 1)
+    return FA_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = dtype == FA_BF16;
+#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, st, workspace, sms
+  if (D == 64) return bf ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
+  return bf ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
+#undef FA_BWD_ARGS
+}
+
+// Status word of the backward kernels (read and optionally reset); used by
+// fa_device_status, not part of the public interface.
+__attribute__((visibility("hidden"))) int fa_bwd_device_status_internal(int reset) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fab::g_bwd_status, sizeof(v)) != cudaSuccess) return -1;
+  if (reset) {
+    const unsigned int z = 0;
+    const unsigned long long zz = 0;
+    if (cudaMemcpyToSymbol(fab::g_bwd_status, &z, sizeof(z)) != cudaSuccess ||
+        cudaMemcpyToSymbol(fab::g_bwd_site, &zz, sizeof(zz)) != cudaSuccess)
+      return -1;
+  }
+  return static_cast<int>(v);
+}
+
+}  // extern "C"

@@ -1250,6 +1250,8 @@ const char* fa_status_string(int s) {
     case FA_ERR_SCRATCH_TOO_SMALL:
       return "fa_fwd_noalloc: this problem needs more scratch than the static buffer holds; "
              "use fa_fwd_ws";
+    case FA_ERR_BAD_WORKSPACE:
+      return "fa_bwd: workspace missing or smaller than fa_bwd_workspace_size(B, Hq, Nq)";
     case FA_ERR_BAD_WINDOW:
       return "key window bounds must be >= -1, and a causal launch cannot have window_right > 0";
     default: return "unknown status";
@@ -1403,10 +1405,14 @@ int fa_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse
   return fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, FA_BF16);
 }
 
+int fa_bwd_device_status_internal(int reset);  // fa_bwd_sm100.cu
+
 int fa_device_status(int reset) {
   unsigned int v = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return -1;
   if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(v)) != cudaSuccess) return -1;
+  const int vb = fa_bwd_device_status_internal(reset);  // the backward kernels' word
+  if (vb < 0) return -1;
   if (reset) {
     const unsigned int z = 0;
     const unsigned long long zz = 0;
@@ -1414,7 +1420,7 @@ int fa_device_status(int reset) {
         cudaMemcpyToSymbol(fa::g_timeout_site, &zz, sizeof(zz)) != cudaSuccess)
       return -1;
   }
-  return static_cast<int>(v);
+  return v != 0 ? static_cast<int>(v) : vb;
 }
 
 int fa_debug_wait_timeout(void* stream) {
