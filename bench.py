@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurement")
     ap.add_argument("--no-window", action="store_true",
                     help="skip the sliding-window measurement")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward-pass measurement")
     return ap.parse_args()
 
 
@@ -344,6 +346,36 @@ def main():
             del gq, gk, gv, go, gl
         assert fa.device_status(reset=True) == 0
 
+    # ---- backward pass on the bench workload (LLaMA-7B layer), both passes
+    backward = {}
+    if not args.no_backward:
+        g0 = torch.Generator(device=dev).manual_seed(1)
+        bdo = torch.randn(q.shape, device=dev, dtype=q.dtype, generator=g0)
+        bws = torch.empty(fa.load_library().fa_bwd_workspace_size(*q.shape[:3]), dtype=torch.uint8,
+                          device=dev)
+        bdq, bdk, bdv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        for w in ws:
+            bo, bl = fa.fa_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal, stream=sptr)
+            ts = []
+            for i in range(13):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fa.fa_bwd(q, k, v, bo, bl, bdo, scale=w.softmax_scale, causal=w.causal, dq=bdq,
+                          dk=bdk, dv=bdv, stream=sptr, workspace=bws)
+                b.record(stream)
+                torch.cuda.synchronize()
+                if i >= 3:
+                    ts.append(a.elapsed_time(b))
+            ms = statistics.median(ts)
+            bflops = 2.5 * w.flops()  # five GEMMs against the forward pass's two
+            backward["causal" if w.causal else "noncausal"] = {
+                "ms": round(ms, 4), "tflops": round(bflops / (ms * 1e-3) / 1e12, 1),
+                "frac_of_peak": round(bflops / (ms * 1e-3) / 1e12 / peaks()[0], 3)}
+        backward["flops"] = "2.5 x the forward pass's (five GEMMs); three launches per call"
+        del bdo, bws, bdq, bdk, bdv
+        assert fa.device_status(reset=True) == 0
+
     # ---- sliding-window attention (causal, 1024-key window, 8192 positions, GQA 4)
     window = {}
     if not args.no_window:
@@ -436,6 +468,7 @@ def main():
         "gate_d128": gate,
         "decode": decode,
         "window": window,
+        "backward": backward,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
