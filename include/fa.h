@@ -147,6 +147,28 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *l
                   size_t workspace_bytes);
 
 /*
+ * Attention with an additive score bias (a mask beyond causal: the mask step
+ * the pages place on the vector unit, and the float attn_mask of the
+ * scaled_dot_product_attention call on the mooersco.com page):
+ *     O_i = sum_j softmax_j(scale q_i.k_j + bias[b, hq, i, j]) v_j,
+ * with -inf in the bias removing a key (causal still applies when causal = 1).
+ *   bias       device pointer, same dtype as q (fp16 / bf16), 16-byte aligned;
+ *              element (b, hq, i, j) at bias + b * bias_stride_b +
+ *              hq * bias_stride_h + i * bias_stride_q + j;
+ *   strides    in elements, >= 0, multiples of 8 (else FA_ERR_MISALIGNED);
+ *              a zero stride broadcasts that dimension (e.g. a key-padding
+ *              mask [B, 1, 1, Nk] has bias_stride_h = bias_stride_q = 0).
+ * A query row whose keys are all removed gets O = 0 and LSE = -inf.  LSE
+ * includes the bias.  Bias tiles are staged through shared memory by TMA (one
+ * 128 x 128 tile per key block, read once per query tile).  Other arguments,
+ * layout and errors as fa_fwd; o and lse may not overlap the bias.
+ */
+int fa_fwd_bias(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, const void *bias,
+                long long bias_stride_b, long long bias_stride_h, long long bias_stride_q,
+                void *stream, int dtype);
+
+/*
  * Backward pass: the gradients of the attention above for an upstream gradient
  * dout (the pages mention only that training keeps gradients -- hwcomputing.
  * csdn.net page, section on standard attention; the operation is taken as the

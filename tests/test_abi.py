@@ -115,3 +115,19 @@ def test_window_entry_point_host_checks(lib):
     if not torch.cuda.is_available():
         for wl, wr, causal in ((-1, -1, 0), (0, 0, 0), (16, -1, 1), (16, 0, 1), (3, 7, 0)):
             assert call(wl, wr, causal) == 8  # valid: reaches the device check
+
+
+def test_bias_entry_point_host_checks(lib):
+    import torch
+    a = dict(GOOD)
+
+    def call(bias=9 * A, sb=0, sh=0, sq=64, D=a["D"]):
+        return lib.fa_fwd_bias(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                               a["Nq"], a["Nk"], D, ctypes.c_float(a["scale"]), 0, bias, sb, sh, sq,
+                               None, a["dtype"])
+    assert call(bias=None) == 1
+    assert call(sq=-8) == 3
+    assert call(bias=9 * A + 8) == 2 and call(sq=63) == 2 and call(sh=4) == 2
+    assert call(bias=4 * A + 256) == 12  # overlaps o
+    if not torch.cuda.is_available():
+        assert call() == 8 and call(sb=4096, sh=64 * 64, sq=64) == 8

@@ -1,0 +1,107 @@
+"""GPU parity of attention with an additive score bias (fa_fwd_bias) against the oracle.
+
+The bias is added to the scaled scores (-inf removes a key); rows left with
+no key must come back as O = 0, LSE = -inf.  Tolerances as for the other
+forward parity tests.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tiled_attention_15_b200 as fa
+from fa_inputs import Workload, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp16": (4e-3, 1e-3), "bf16": (1.6e-2, 1e-3)}
+TD = {"fp16": torch.float16, "bf16": torch.bfloat16}
+
+
+def _bias(w, shape, seed, scale=2.0, neg_inf_frac=0.0):
+    rng = np.random.default_rng(seed)
+    b = (scale * rng.standard_normal(shape)).astype(np.float32)
+    if neg_inf_frac > 0:
+        b[rng.random(shape) < neg_inf_frac] = -np.inf
+    return torch.from_numpy(b).to(TD[w.dtype])
+
+
+def _check(w, bias, dev, tag=""):
+    q, k, v = make_qkv(w)
+    o, lse = fa.fa_fwd(q.to(dev), k.to(dev), v.to(dev), scale=w.softmax_scale, causal=w.causal,
+                       bias=bias.to(dev))
+    torch.cuda.synchronize()
+    assert fa.device_status(reset=True) == 0
+    ref_o, ref_l = oracle.attention(q, k, v, w.softmax_scale, w.causal, bias=bias.float())
+    got_o, got_l = o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy()
+    empty = np.isneginf(ref_l)
+    np.testing.assert_array_equal(np.isneginf(got_l), empty)
+    assert np.all(got_o[empty] == 0.0) and np.isfinite(got_o).all()
+    do = np.abs(got_o - ref_o).max()
+    dl = np.abs(got_l[~empty] - ref_l[~empty]).max() if (~empty).any() else 0.0
+    report = os.environ.get("FA_PARITY_REPORT")
+    if report:
+        with open(report, "a") as f:
+            f.write(json.dumps({"case": f"bias {w.name}{tag}", "dtype": w.dtype,
+                                "max_abs_dO": float(do), "max_abs_dLSE": float(dl)}) + "\n")
+    to, tl = TOL[w.dtype]
+    assert do <= to, f"{w.name}: max|dO| = {do:.3e}"
+    assert dl <= tl, f"{w.name}: max|dLSE| = {dl:.3e}"
+    return o, lse
+
+
+def test_full_bias_fp16(cuda_dev):
+    w = Workload("full [B,H,Nq,Nk] D128 fp16", 2, 4, 2, 300, 333, 128, "fp16", False, seed=111)
+    _check(w, _bias(w, (2, 4, 300, 333), 1), cuda_dev)
+
+
+def test_broadcast_bias_causal_bf16(cuda_dev):
+    w = Workload("shared [Nq,Nk] D64 bf16 causal", 2, 3, 3, 700, 700, 64, "bf16", True, seed=112)
+    _check(w, _bias(w, (1, 1, 700, 700), 2), cuda_dev)
+
+
+def test_key_padding_mask(cuda_dev):
+    # [B, 1, 1, Nk]: one bias row for every query (broadcast over queries and heads)
+    w = Workload("key padding [B,1,1,Nk] D128 fp16", 2, 4, 4, 200, 333, 128, "fp16", False, seed=113)
+    b = torch.zeros(2, 1, 1, 333)
+    b[0, :, :, 250:] = -float("inf")
+    b[1, :, :, 100:] = -float("inf")
+    _check(w, b.half(), cuda_dev)
+
+
+def test_per_head_bias_d256(cuda_dev):
+    w = Workload("per head [1,H,Nq,Nk] D256 bf16", 2, 4, 1, 256, 512, 256, "bf16", False, seed=114)
+    _check(w, _bias(w, (1, 4, 256, 512), 3), cuda_dev)
+
+
+def test_bias_removes_whole_rows(cuda_dev):
+    w = Workload("empty rows D64 fp16", 1, 2, 2, 150, 260, 64, "fp16", False, seed=115)
+    b = _bias(w, (1, 2, 150, 260), 4, neg_inf_frac=0.3)
+    b[0, 0, 7, :] = -float("inf")
+    b[0, 1, 140:, :] = -float("inf")
+    _check(w, b, cuda_dev)
+
+
+def test_large_bias_values(cuda_dev):
+    # +-30 bias: the running max moves by large steps between blocks (rescales)
+    w = Workload("large bias D128 bf16", 1, 2, 2, 400, 1000, 128, "bf16", False, seed=116)
+    _check(w, _bias(w, (1, 2, 400, 1000), 5, scale=30.0), cuda_dev)
+
+
+def test_zero_bias_equals_no_bias(cuda_dev):
+    w = Workload("zero bias D128 fp16", 1, 2, 2, 300, 300, 128, "fp16", True, seed=117)
+    o, lse = _check(w, torch.zeros(1, 1, 1, 300, dtype=torch.float16), cuda_dev)
+    q, k, v = (x.to(cuda_dev) for x in make_qkv(w))
+    o2, lse2 = fa.fa_fwd(q, k, v, scale=w.softmax_scale, causal=True, use_workspace=False)
+    torch.cuda.synchronize()
+    assert (o.float() - o2.float()).abs().max().item() <= 2e-3
+    assert (lse - lse2).abs().max().item() <= 1e-5
+
+
+def test_unaligned_key_count_is_padded(cuda_dev):
+    # Nk = 77: the binding copies the bias into rows padded to 80 keys
+    w = Workload("Nk 77 D64 fp16", 1, 2, 2, 90, 77, 64, "fp16", False, seed=118)
+    _check(w, _bias(w, (1, 2, 90, 77), 6), cuda_dev)

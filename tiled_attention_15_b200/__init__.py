@@ -26,7 +26,7 @@ FA_ERR_BAD_WORKSPACE = 15
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
-            "fa_fwd_window", "fa_bwd", "fa_bwd_workspace_size",
+            "fa_fwd_window", "fa_fwd_bias", "fa_bwd", "fa_bwd_workspace_size",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
             "fa_status_string", "fa_device_status", "fa_device_timeout_site",
             "fa_debug_exp2_fma", "fa_debug_wait_timeout", "fa_fwd_num_tiles")
@@ -61,6 +61,9 @@ def load_library() -> ctypes.CDLL:
     lib.fa_fwd_ws.restype = i
     lib.fa_fwd_window.argtypes = fwd_args[:13] + [i, i, vp, i, vp, ctypes.c_size_t]
     lib.fa_fwd_window.restype = i
+    ll = ctypes.c_longlong
+    lib.fa_fwd_bias.argtypes = fwd_args[:13] + [vp, ll, ll, ll, vp, i]
+    lib.fa_fwd_bias.restype = i
     lib.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, vp, i, vp, ctypes.c_size_t]
     lib.fa_bwd.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i]
@@ -161,7 +164,7 @@ def fa_fwd_raw(q: int, k: int, v: int, o: int, lse: Optional[int], B: int, Hq: i
 
 def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False,
            return_lse: bool = True, stream=None, use_workspace: bool = True,
-           window: Tuple[int, int] = (-1, -1)) -> Tuple[object, Optional[object]]:
+           window: Tuple[int, int] = (-1, -1), bias=None) -> Tuple[object, Optional[object]]:
     """Fused attention forward on the current CUDA stream.
 
     q: [B, Hq, Nq, D], k/v: [B, Hkv, Nk, D] contiguous CUDA tensors, fp16 or bf16.
@@ -169,6 +172,8 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
     scale defaults to 1/sqrt(D).  use_workspace: call fa_fwd_ws with a cached
     per-(device, stream) workspace (load balance), else fa_fwd.  window:
     (left, right) key window, -1 = unbounded (fa_fwd_window when either is set).
+    bias: additive score bias (fa_fwd_bias), a CUDA tensor of q's dtype that
+    broadcasts to [B, Hq, Nq, Nk] (size-1 dims broadcast).
     Returns (o, lse or None).
     """
     import torch
@@ -202,6 +207,14 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
             lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, D,
             ctypes.c_float(scale), 1 if causal else 0, stream or None, dtype)
     wl, wr = (int(x) for x in window)
+    if bias is not None:
+        if (wl, wr) != (-1, -1):
+            raise ValueError("a bias and a key window cannot be combined")
+        bt, sb, sh, sq = _bias_view(bias, q.dtype, B, Hq, Nq, Nk)
+        rc = lib.fa_fwd_bias(*args[:13], bt.data_ptr(), sb, sh, sq, args[13], dtype)
+        if rc != FA_OK:
+            raise FaError(rc, "fa_fwd_bias")
+        return o, lse
     if (wl, wr) != (-1, -1):
         ws = workspace(q.device, stream) if use_workspace else None
         rc = lib.fa_fwd_window(*args[:13], wl, wr, args[13], dtype,
@@ -265,3 +278,29 @@ def fa_bwd(q, k, v, o, lse, dout, scale: Optional[float] = None, causal: bool = 
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
     return dq, dk, dv
+
+
+def _bias_view(bias, dtype, B, Hq, Nq, Nk):
+    """(tensor, stride_b, stride_h, stride_q) in elements for fa_fwd_bias.
+
+    Broadcast (size-1) dims get stride 0.  Keys must be contiguous and the other
+    strides multiples of 8 elements (16 bytes); otherwise the bias is copied
+    into a buffer whose rows are padded to a multiple of 8 keys.
+    """
+    import torch
+
+    if bias.dtype != dtype or not bias.is_cuda:
+        raise TypeError("bias must be a CUDA tensor with the dtype of q")
+    while bias.dim() < 4:
+        bias = bias.unsqueeze(0)
+    full = (B, Hq, Nq, Nk)
+    if bias.dim() != 4 or any(n not in (1, f) for n, f in zip(bias.shape, full)) or bias.shape[3] != Nk:
+        raise ValueError("bias must broadcast to [B, Hq, Nq, Nk] with last dim Nk")
+    st = [0 if bias.shape[d] == 1 else bias.stride(d) for d in range(3)]
+    if bias.stride(3) != 1 or any(x % 8 for x in st) or bias.data_ptr() % 16:
+        nk_pad = (Nk + 7) // 8 * 8
+        padded = torch.zeros(tuple(bias.shape[:3]) + (nk_pad,), dtype=dtype, device=bias.device)
+        padded[..., :Nk] = bias
+        bias = padded[..., :Nk]
+        st = [0 if bias.shape[d] == 1 else bias.stride(d) for d in range(3)]
+    return bias, st[0], st[1], st[2]

@@ -60,9 +60,10 @@ constexpr int kThreads = 384;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
 constexpr float kRescaleThreshold = 8.0f;         // log2 units: P <= 2^8 between rescales
 constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
 constexpr int kTileRing = 4;  // units the TMA thread may hand out ahead of the consumers
 
-template <int D, int NQ>
+template <int D, int NQ, bool BIAS = false>
 struct Geometry {
   static constexpr int DCH = D / 64;  // 128-byte (64-element) column chunks per row
   static constexpr int Q_BYTES = kBM * D * 2;
@@ -71,15 +72,21 @@ struct Geometry {
   static constexpr int CHUNK_KV = kBN * 128;  // one 64-column chunk of a K/V block
   // K/V stages: what the shared memory left by the Q tiles holds (one query
   // tile leaves room for deeper staging, which decode-like launches need)
-  static constexpr int NST = NQ == 2 ? (D == 64 ? 8 : 4) : (D == 64 ? 12 : (D == 128 ? 6 : 2));
+  static constexpr int NST = BIAS ? (D == 64 ? 8 : (D == 128 ? 4 : 2))
+                                  : NQ == 2 ? (D == 64 ? 8 : 4) : (D == 64 ? 12 : (D == 128 ? 6 : 2));
+  // score-bias tiles (bias launches: one query tile): [2 boxes][128 rows][64 keys], 16-bit
+  static constexpr int NBS = BIAS ? (D == 256 ? 1 : 2) : 0;
+  static constexpr int BIAS_BYTES = 128 * 128 * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = NQ * Q_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NST * KV_BYTES;
+  static constexpr int OFF_BIAS = OFF_KV + NST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_BIAS + NBS * BIAS_BYTES;
   // mbarrier indices
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NST,
                        B_SFULL = 4 + 2 * NST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
                        B_OEMPTY = B_OFULL + 2, B_PVDONE = B_OEMPTY + 2, B_TFULL = B_PVDONE + 1,
-                       B_TEMPTY = B_TFULL + kTileRing, NBAR = B_TEMPTY + kTileRing;
+                       B_TEMPTY = B_TFULL + kTileRing, B_BFULL = B_TEMPTY + kTileRing,
+                       B_BEMPTY = B_BFULL + NBS, NBAR = B_BEMPTY + NBS;
   // tmem base (u32), abort flag (u32), then the ring of unit indices (kTileRing x s32)
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // ... then this CTA's stream-K unit range (2 x s32)
@@ -312,11 +319,11 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
 // way it publishes every index -- or -1 at the end -- in a shared-memory ring
 // (t_full: written; t_empty: read by the MMA thread and every softmax warp, 4
 // per query tile).
-template <int D, int NQ>
+template <int D, int NQ, bool BIAS = false>
 __device__ __forceinline__ bool produce_unit(const Ctx& cx, const FwdParams& p, TileIter& it,
                                              uint32_t& n, int& u) {
   if (!p.use_ring) return it.next(u);
-  using G = Geometry<D, NQ>;
+  using G = Geometry<D, NQ, BIAS>;
   int end = p.n_units;
   if (p.sk_w > 0) {  // stream-K: this CTA's fixed range, left by the prologue after the ring
     const volatile int* sk = cx.ring + kTileRing;
@@ -336,11 +343,11 @@ __device__ __forceinline__ bool produce_unit(const Ctx& cx, const FwdParams& p, 
   return pub >= 0;
 }
 // Consumer side; `lane` < 0 for the single MMA thread, else the softmax warp's lane.
-template <int D, int NQ>
+template <int D, int NQ, bool BIAS = false>
 __device__ __forceinline__ bool consume_unit(const Ctx& cx, const FwdParams& p, TileIter& it,
                                              uint32_t& n, int& u, int lane) {
   if (!p.use_ring) return it.next(u);
-  using G = Geometry<D, NQ>;
+  using G = Geometry<D, NQ, BIAS>;
   const int k = n % kTileRing;
   bool ok = wait_bar(cx.bar(G::B_TFULL + k, G::OFF_BAR), (n / kTileRing) & 1u, cx.abort_flag);
   if (lane >= 0) ok = __all_sync(0xffffffffu, ok);
@@ -363,11 +370,16 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, bool bf16) {
 }
 
 // ---------------------------------------------------------------- TMA producer
-template <int D, int NQ>
+// Score-bias mode bits (bias launches): 1 = one bias row for every query
+// (broadcast over queries), 2 = a bias per query head, 4 = a bias per batch.
+constexpr int kBiasRowBcast = 1, kBiasPerHead = 2, kBiasPerBatch = 4;
+
+template <int D, int NQ, bool BIAS = false>
 __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, const CUtensorMap* tq,
                                           const CUtensorMap* tq4, const CUtensorMap* tk,
-                                          const CUtensorMap* tv) {
-  using G = Geometry<D, NQ>;
+                                          const CUtensorMap* tv, const CUtensorMap* tb,
+                                          int bias_mode) {
+  using G = Geometry<D, NQ, BIAS>;
   prefetch_tmap(p.pack_g > 1 ? tq4 : tq);
   prefetch_tmap(tk);
   prefetch_tmap(tv);
@@ -411,10 +423,32 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
     ++kv_it;
     return true;
   };
+  // Bias launches: the [128 query rows x 128 keys] bias tile of block j, as two
+  // 64-key boxes with 128-byte swizzle (one row when broadcast over queries).
+  uint32_t b_it = 0;
+  auto load_bias = [&](const Tile& T, int j) -> bool {
+    if constexpr (BIAS) {
+      const int bs = b_it % G::NBS;
+      if (b_it >= (uint32_t)G::NBS &&
+          !wait_bar(cx.bar(G::B_BEMPTY + bs, G::OFF_BAR), ((b_it / G::NBS) - 1) & 1u, cx.abort_flag))
+        return false;
+      const int rows = (bias_mode & kBiasRowBcast) ? 1 : kBM;
+      mbar_arrive_expect_tx(cx.bar(G::B_BFULL + bs, G::OFF_BAR), 2 * rows * 128);
+      const int hq = T.bh % p.Hq, b = T.bh / p.Hq;
+#pragma unroll
+      for (int box = 0; box < 2; ++box)
+        tma_load_4d(cx.sbase + G::OFF_BIAS + bs * G::BIAS_BYTES + box * (G::BIAS_BYTES / 2), tb,
+                    cx.bar(G::B_BFULL + bs, G::OFF_BAR), (T.jb + j) * kBN + box * 64,
+                    (bias_mode & kBiasRowBcast) ? 0 : T.row0, (bias_mode & kBiasPerHead) ? hq : 0,
+                    (bias_mode & kBiasPerBatch) ? b : 0, pol_kv);
+      ++b_it;
+    }
+    return true;
+  };
   TileIter it(p.n_units);
   uint32_t n_units_seen = 0;
   int t;
-  while (ok && produce_unit<D, NQ>(cx, p, it, n_units_seen, t)) {
+  while (ok && produce_unit<D, NQ, BIAS>(cx, p, it, n_units_seen, t)) {
     const Tile T = get_tile<NQ>(p, t);
     // Q0, then K0 (the first S MMA of the tile needs only these), then Q1 -- each
     // Q tile waits only for the last S MMA that read its previous contents.
@@ -422,6 +456,7 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
     //   NQ = 2: K0, V0, K1, V1, ...      NQ = 1: K0, K1, V0, K2, V1, ...
     if (T.nblk[0] > 0 && !load_q(T, 0)) { ok = false; break; }
     if (!load_kv(T, tk, 0)) { ok = false; break; }
+    if (BIAS && !load_bias(T, 0)) { ok = false; break; }
     if (NQ == 2 && T.nblk[1] > 0 && !load_q(T, 1)) { ok = false; break; }
     for (int s = 1; s < 2 * T.nb && ok; ++s) {
       int j;
@@ -432,6 +467,7 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
         else { is_k = (s & 1) == 1; j = is_k ? (s + 1) / 2 : s / 2 - 1; }
       }
       if (!load_kv(T, is_k ? tk : tv, j)) ok = false;
+      if (BIAS && ok && is_k && !load_bias(T, j)) ok = false;
     }
   }
   if (!ok) {  // abort: let this CTA's own loads land before the CTA exits
@@ -439,13 +475,16 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
       drain_bar(cx.bar(G::B_KVFULL + n % G::NST, G::OFF_BAR), (n / G::NST) & 1u);
     for (int q = 0; q < 2; ++q)
       if (q_issued[q]) drain_bar(cx.bar(G::B_QFULL + q, G::OFF_BAR), (q_issued[q] - 1) & 1u);
+    if constexpr (BIAS)
+      for (uint32_t n = (b_it > (uint32_t)G::NBS ? b_it - G::NBS : 0); n < b_it; ++n)
+        drain_bar(cx.bar(G::B_BFULL + n % G::NBS, G::OFF_BAR), (n / G::NBS) & 1u);
   }
 }
 
 // ---------------------------------------------------------------- MMA issuer
-template <int D, int NQ, bool BF16>
+template <int D, int NQ, bool BF16, bool BIAS = false>
 __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
-  using G = Geometry<D, NQ>;
+  using G = Geometry<D, NQ, BIAS>;
   constexpr uint32_t kIdS = idesc_f16(kBM, kBN, BF16, false);  // Q, K both K-major
   constexpr uint32_t kIdPV = idesc_f16(kBM, D, BF16, true);    // V is N(=D)-major
   uint32_t kv_it = 0, q_phase[2] = {0u, 0u}, p_phase[2] = {0u, 0u}, oe_phase[2] = {0u, 0u};
@@ -510,7 +549,7 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
   TileIter it(p.n_units);
   uint32_t n_units_seen = 0;
   int t;
-  while (consume_unit<D, NQ>(cx, p, it, n_units_seen, t, -1)) {
+  while (consume_unit<D, NQ, BIAS>(cx, p, it, n_units_seen, t, -1)) {
     const Tile T = get_tile<NQ>(p, t);
     const int nb = T.nb;
     int kst;
@@ -710,22 +749,23 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
-template <int D, int NQ, bool BF16>
+template <int D, int NQ, bool BF16, bool BIAS = false>
 __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, int wg, int sub,
-                                             int lane) {
-  using G = Geometry<D, NQ>;
+                                             int lane, int bias_mode) {
+  using G = Geometry<D, NQ, BIAS>;
   const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
   const uint32_t tm = cx.tmem + lane_off;
   auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
   const float c = p.c;
   constexpr bool kWin = NQ == 1;  // key windows: one-query-tile kernels only
   uint32_t s_phase[2] = {0u, 0u}, of_phase = 0u, pv_seen = 0u;
+  uint32_t b_cnt = 0, b_phase = 0u;  // bias tiles consumed; parity bit per stage
   const int q = (NQ == 2) ? wg : 0;
 
   TileIter it(p.n_units);
   uint32_t n_units_seen = 0;
   int t;
-  while (consume_unit<D, NQ>(cx, p, it, n_units_seen, t, lane)) {
+  while (consume_unit<D, NQ, BIAS>(cx, p, it, n_units_seen, t, lane)) {
     // Only what the key loop needs stays live across it; the epilogue decodes
     // the unit again (registers are the softmax warps' tightest resource).
     int nblk, rfirst, jb;
@@ -749,15 +789,47 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
       tmem_ld_x128(tm + sb * 128, sr);
 
       const int kbase = (jb + j) * kBN;
-      // (key windows exist in the one-query-tile kernels only)
+      // (key windows exist in the one-query-tile kernels only; a score bias
+      // enters the row max, so bias launches take the masked path every block)
       const bool masked =
-          kWin ? (kbase + kBN > p.Nk) || (p.wr >= 0 && kbase + kBN - 1 > rfirst + p.wr) ||
-                     (p.wl >= 0 && kbase < rfirst + kBM - 1 - p.wl)
-               : (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst);
+          BIAS || (kWin ? (kbase + kBN > p.Nk) || (p.wr >= 0 && kbase + kBN - 1 > rfirst + p.wr) ||
+                              (p.wl >= 0 && kbase < rfirst + kBM - 1 - p.wl)
+                        : (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst));
       float m_blk;
       if (masked) {  // scaled scores, -inf where the key is outside the window or past Nk
         int lim = p.Nk - kbase;  // keys [lo, lim) of the block are visible to this row
-        if (kWin) {
+        if constexpr (BIAS) {
+          // scaled score + bias * log2(e); the tile holds this row's 128 bias
+          // values as 16 swizzled 16-byte units (one row for every query when
+          // broadcast over queries)
+          if (p.causal) lim = min(lim, row - kbase + 1);
+          const int bs = b_cnt % G::NBS;
+          ok = wait_bar(B(G::B_BFULL + bs), (b_phase >> bs) & 1u, cx.abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) return;
+          b_phase ^= 1u << bs;
+          ++b_cnt;
+          const uint32_t brow = (bias_mode & kBiasRowBcast) ? 0u : static_cast<uint32_t>(sub * 32 + lane);
+          const uint32_t bbase = cx.sbase + G::OFF_BIAS + bs * G::BIAS_BYTES + brow * 128u;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(bbase + (u >> 3) * (G::BIAS_BYTES / 2) +
+                               ((static_cast<uint32_t>(u & 7) ^ (brow & 7u)) << 4)));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int i = u * 8 + e;
+              const uint32_t h16 = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xffffu);
+              const float bv = BF16 ? __uint_as_float(h16 << 16)
+                                    : __half2float(__ushort_as_half(static_cast<unsigned short>(h16)));
+              sr[i] = __float_as_uint(i < lim ? fmaf(__uint_as_float(sr[i]), c, bv * kLog2e)
+                                              : -INFINITY);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(B(G::B_BEMPTY + bs));
+        } else if (kWin) {
           if (p.wr >= 0) lim = min(lim, row + p.wr - kbase + 1);
           const int lo = p.wl >= 0 ? row - p.wl - kbase : 0;
           const uint32_t span = static_cast<uint32_t>(max(lim - lo, 0));
@@ -885,12 +957,12 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   }
 }
 
-template <int D, int NQ, bool BF16>
+template <int D, int NQ, bool BF16, bool BIAS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q4,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const FwdParams p) {
-  using G = Geometry<D, NQ>;
+                  const FwdParams p, const __grid_constant__ CUtensorMap tm_b, const int bias_mode) {
+  using G = Geometry<D, NQ, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -923,6 +995,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(B(G::B_TFULL + k), 1);
       mbar_init(B(G::B_TEMPTY + k), 1 + 4 * NQ);  // the MMA thread and the softmax warps
     }
+    for (int k = 0; k < G::NBS; ++k) {
+      mbar_init(B(G::B_BFULL + k), 1);
+      mbar_init(B(G::B_BEMPTY + k), 4);  // the four softmax warps
+    }
     misc[1] = 0u;
     if (p.sk_w > 0) {  // stream-K: the units c + t, t over the tiles this CTA's range touches
       const int c = blockIdx.x, C = gridDim.x, W = p.sk_w;
@@ -952,11 +1028,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) setmaxnreg_inc<kSoftmaxRegs>();
   else setmaxnreg_dec<kOtherRegs>();
   if (warp < 8) {
-    if (NQ == 2 || warp < 4) role_softmax<D, NQ, BF16>(cx, p, warp >> 2, warp & 3, lane);
+    if (NQ == 2 || warp < 4) role_softmax<D, NQ, BF16, BIAS>(cx, p, warp >> 2, warp & 3, lane, bias_mode);
   } else if (warp == 8) {
-    if (lane == 0) role_mma<D, NQ, BF16>(cx, p);
+    if (lane == 0) role_mma<D, NQ, BF16, BIAS>(cx, p);
   } else if (warp == 9) {
-    if (lane == 0) role_load<D, NQ>(cx, p, &tm_q, &tm_q4, &tm_k, &tm_v);
+    if (lane == 0) role_load<D, NQ, BIAS>(cx, p, &tm_q, &tm_q4, &tm_k, &tm_v, &tm_b, bias_mode);
   }
   __syncwarp();
   tc_fence_before();
@@ -1099,17 +1175,44 @@ WsLayout ws_layout(int D, int rows, int n_split, int nsplit) {
 // arrival counters are cleared on the stream before the kernel).
 enum class Scratch { kCaller, kStatic };
 
-template <int D, int NQ, bool BF16>
+// A score bias [B][H][Nq][Nk] (16-bit, keys contiguous) given by element strides;
+// a zero stride broadcasts that dimension.
+struct BiasArg {
+  const void* ptr;
+  long long sb, sh, sq;
+};
+
+// 4-D map over the bias with 64-key x `rows`-query boxes, 128-byte swizzle; a
+// broadcast dimension has extent 1 (its coordinate is always 0).
+bool make_bias_map(CUtensorMap* m, const BiasArg& a, int B, int H, int Nq, int Nk, bool bf16) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)Nk, (cuuint64_t)(a.sq ? Nq : 1), (cuuint64_t)(a.sh ? H : 1),
+                              (cuuint64_t)(a.sb ? B : 1)};
+  // strides of extent-1 dimensions are never used; keep them valid and increasing
+  const cuuint64_t s1 = a.sq ? (cuuint64_t)a.sq * 2 : (cuuint64_t)((Nk * 2 + 15) / 16 * 16);
+  const cuuint64_t s2 = a.sh ? (cuuint64_t)a.sh * 2 : s1 * dims[1];
+  const cuuint64_t s3 = a.sb ? (cuuint64_t)a.sb * 2 : s2 * dims[2];
+  const cuuint64_t strides[3] = {s1, s2, s3};
+  const cuuint32_t box[4] = {64u, a.sq ? 128u : 1u, 1u, 1u};
+  const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+             const_cast<void*>(a.ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int NQ, bool BF16, bool BIAS = false>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
            int Hkv, int Nq, int Nk, float scale, int causal, int wl, int wr, cudaStream_t stream,
-           int dev, void* ws, size_t ws_bytes, Scratch mode) {
-  using G = fa::Geometry<D, NQ>;
+           int dev, void* ws, size_t ws_bytes, Scratch mode, const BiasArg* bias = nullptr) {
+  using G = fa::Geometry<D, NQ, BIAS>;
   static bool attr_done[kMaxDevices] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     if (!attr_done[dev]) {
-      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, NQ, BF16>,
+      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, NQ, BF16, BIAS>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                G::SMEM_BYTES) != cudaSuccess)
         return FA_ERR_LAUNCH;
@@ -1118,7 +1221,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   }
   const int g = Hq / Hkv;
   const bool windowed = wl >= 0 || wr >= 0;
-  const bool pack = !windowed && pack_heads(Hq, Hkv, Nq, causal);
+  const bool pack = !BIAS && !windowed && pack_heads(Hq, Hkv, Nq, causal);
   CUtensorMap tq, tq4, tk, tv;
   if (!make_map(&tq, q, D, Nq, (long long)B * Hq, fa::kBM, BF16) ||
       !make_map(&tk, k, D, Nk, (long long)B * Hkv, fa::kBN, BF16) ||
@@ -1155,7 +1258,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
                                                    : NQ * fa::kBM);
   int n_split = 0, nsplit = 1;
   int sk_w = 0, sk_grid = 0;
-  if (ws != nullptr && !causal && !windowed) {
+  if (ws != nullptr && !causal && !windowed && !BIAS) {
     if (p.n_tiles < ctas && p.n_tiles <= kMaxSplit) {
       // Stream-K: fewer tiles than CTAs (decode-like shapes).  The key blocks of
       // all tiles are shared out evenly over C CTAs, each with at least
@@ -1219,7 +1322,15 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
       p.n_units > grid)
     p.sched = reinterpret_cast<int*>(static_cast<char*>(ws) + kMaxSplit * 2 * 4 * sizeof(int));
   p.use_ring = (p.sched != nullptr || sk_w > 0) ? 1 : 0;
-  fa::fa_fwd_kernel<D, NQ, BF16><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(tq, tq4, tk, tv, p);
+  CUtensorMap tb = tk;  // (unused without a bias)
+  int bias_mode = 0;
+  if (BIAS) {
+    if (!make_bias_map(&tb, *bias, B, Hq, Nq, Nk, BF16)) return FA_ERR_DRIVER;
+    bias_mode = (bias->sq ? 0 : fa::kBiasRowBcast) | (bias->sh ? fa::kBiasPerHead : 0) |
+                (bias->sb ? fa::kBiasPerBatch : 0);
+  }
+  fa::fa_fwd_kernel<D, NQ, BF16, BIAS><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(
+      tq, tq4, tk, tv, p, tb, bias_mode);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -1267,7 +1378,7 @@ long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D) {
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                     int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype,
                     void* ws, size_t ws_bytes, Scratch mode = Scratch::kCaller, int wl = -1,
-                    int wr = -1) {
+                    int wr = -1, const BiasArg* bias = nullptr) {
   // ---- argument checks: host only, before any CUDA call
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
   if (wl < -1 || wr < -1 || (causal && wr > 0)) return FA_ERR_BAD_WINDOW;
@@ -1308,6 +1419,16 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   // A work tile of at most 128 rows (short queries, or a packed GQA group) runs
   // the one-query-tile kernel: its two S buffers let the softmax of key block j
   // overlap the S MMA of block j + 1, and its K/V staging is deeper.
+  if (bias != nullptr) {  // score bias: the one-query-tile kernels with bias staging
+#define FA_BARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, -1, -1, st, dev, nullptr, 0, \
+                 Scratch::kCaller, bias
+    switch (D) {
+      case 64: return bf ? launch<64, 1, true, true>(FA_BARGS) : launch<64, 1, false, true>(FA_BARGS);
+      case 128: return bf ? launch<128, 1, true, true>(FA_BARGS) : launch<128, 1, false, true>(FA_BARGS);
+      default: return bf ? launch<256, 1, true, true>(FA_BARGS) : launch<256, 1, false, true>(FA_BARGS);
+    }
+#undef FA_BARGS
+  }
   // Windowed launches too: each tile gets its own key block range.
   const bool windowed = wl >= 0 || wr >= 0;
   const bool one_tile =
@@ -1340,6 +1461,27 @@ int fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* l
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype,
                   workspace, workspace != nullptr ? workspace_bytes : 0, Scratch::kCaller,
                   window_left, window_right);
+}
+
+int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, const void* bias,
+                long long bias_stride_b, long long bias_stride_h, long long bias_stride_q,
+                void* stream, int dtype) {
+  if (bias == nullptr) return FA_ERR_NULL_POINTER;
+  if (bias_stride_b < 0 || bias_stride_h < 0 || bias_stride_q < 0) return FA_ERR_BAD_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(bias) & 15u) || (bias_stride_b & 7) || (bias_stride_h & 7) ||
+      (bias_stride_q & 7))
+    return FA_ERR_MISALIGNED;
+  if (B >= 1 && Hq >= 1 && Nq >= 1 && Nk >= 1 && o != nullptr) {  // o, lse must not overlap the bias
+    const size_t extent = 2 * static_cast<size_t>((B - 1) * bias_stride_b + (Hq - 1) * bias_stride_h +
+                                                  (Nq - 1) * bias_stride_q + Nk);
+    if (overlaps(o, (size_t)B * Hq * Nq * D * 2, bias, extent) ||
+        (lse && overlaps(lse, (size_t)B * Hq * Nq * 4, bias, extent)))
+      return FA_ERR_OVERLAP;
+  }
+  const BiasArg a{bias, bias_stride_b, bias_stride_h, bias_stride_q};
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, nullptr, 0,
+                  Scratch::kCaller, -1, -1, &a);
 }
 
 size_t fa_fwd_workspace_size(int D) {
