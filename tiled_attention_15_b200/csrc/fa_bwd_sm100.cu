@@ -198,13 +198,17 @@ struct GeoKV {
   static constexpr int DCH = D / 64;
   static constexpr int T_BYTES = 128 * D * 2;  // one 128-row tile
   static constexpr int CHUNK = 128 * 128;      // one 64-column chunk of a tile
-  static constexpr int NST = D == 64 ? 4 : 2;  // query-block stages (Q, dO, lse2, delta)
-  static constexpr int OFF_K = 0, OFF_V = T_BYTES, OFF_ST = 2 * T_BYTES;
-  static constexpr int ST_BYTES = 2 * T_BYTES + 2 * 512;
-  static constexpr int OFF_BAR = OFF_ST + NST * ST_BYTES;
+  // Q and dO tiles stream through a ring of single-tile slots in the order
+  // Q0 dO0 Q1 dO1 ...; a slot holding Q_n also holds that block's lse2 and
+  // delta (1 KB side buffer).  dO_n is freed after dV(n), Q_n after dK(n).
+  static constexpr int NSLOT = D == 64 ? 8 : 4;
+  static constexpr int SLOT_BYTES = T_BYTES + 1024;
+  static constexpr int OFF_K = 0, OFF_V = T_BYTES, OFF_SL = 2 * T_BYTES;
+  static constexpr int OFF_BAR = OFF_SL + NSLOT * SLOT_BYTES;
   // barriers
-  static constexpr int B_KV = 0, B_QF = 1, B_QE = 1 + NST, B_SF = 1 + 2 * NST, B_DPF = B_SF + 1,
-                       B_PF = B_SF + 2, B_DSF = B_SF + 3, B_ACC = B_SF + 4, NBAR = B_SF + 5;
+  static constexpr int B_KV = 0, B_SLF = 1, B_SLE = 1 + NSLOT, B_SF = 1 + 2 * NSLOT,
+                       B_DPF = B_SF + 1, B_PF = B_SF + 2, B_DSF = B_SF + 3, B_ACC = B_SF + 4,
+                       NBAR = B_SF + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // TMEM columns: S^T 0..127 (P^T over it), dP^T 128..255 (dS^T over it), dV, dK
@@ -256,9 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(B(G::B_KV), 1);
-    for (int s = 0; s < G::NST; ++s) {
-      mbar_init(B(G::B_QF + s), 1);
-      mbar_init(B(G::B_QE + s), 1);
+    for (int s = 0; s < G::NSLOT; ++s) {
+      mbar_init(B(G::B_SLF + s), 1);
+      mbar_init(B(G::B_SLE + s), 1);
     }
     mbar_init(B(G::B_SF), 1);
     mbar_init(B(G::B_DPF), 1);
@@ -293,22 +297,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sbase + G::OFF_V + c * G::CHUNK, &tm_v, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
     }
     const int nqb = p.nqt - T.i0;
-    for (int n = 0; n < T.nb; ++n) {
-      const int st = n % G::NST;
-      if (n >= G::NST && !wait_bar(B(G::B_QE + st), ((n / G::NST) - 1) & 1u, cx.abort_flag)) break;
+    for (int m = 0; m < 2 * T.nb; ++m) {  // item m: Q (even, + lse2, delta) or dO (odd) of block m / 2
+      const int sl = m % G::NSLOT, n = m >> 1;
+      if (m >= G::NSLOT && !wait_bar(B(G::B_SLE + sl), ((m / G::NSLOT) - 1) & 1u, cx.abort_flag))
+        break;
       const int h = n / nqb, i = T.i0 + n % nqb;
       const int bh = (T.bkv / p.Hkv) * p.Hq + (T.bkv % p.Hkv) * p.group + h;
-      const uint32_t sb = sbase + G::OFF_ST + st * G::ST_BYTES;
-      mbar_arrive_expect_tx(B(G::B_QF + st), 2 * G::T_BYTES + 1024);
+      const uint32_t sb = sbase + G::OFF_SL + sl * G::SLOT_BYTES;
+      mbar_arrive_expect_tx(B(G::B_SLF + sl), G::T_BYTES + ((m & 1) ? 0 : 1024));
 #pragma unroll
-      for (int c = 0; c < G::DCH; ++c) {
-        tma_load_3d(sb + c * G::CHUNK, &tm_q, B(G::B_QF + st), c * 64, i * kBM, bh, pol_last);
-        tma_load_3d(sb + G::T_BYTES + c * G::CHUNK, &tm_do, B(G::B_QF + st), c * 64, i * kBM, bh,
-                    pol_last);
+      for (int c = 0; c < G::DCH; ++c)
+        tma_load_3d(sb + c * G::CHUNK, (m & 1) ? &tm_do : &tm_q, B(G::B_SLF + sl), c * 64, i * kBM,
+                    bh, pol_last);
+      if ((m & 1) == 0) {
+        const size_t row = static_cast<size_t>(bh) * p.Nq_pad + static_cast<size_t>(i) * kBM;
+        bulk_load(sb + G::T_BYTES, p.lse2 + row, 512, B(G::B_SLF + sl));
+        bulk_load(sb + G::T_BYTES + 512, p.delta + row, 512, B(G::B_SLF + sl));
       }
-      const size_t row = static_cast<size_t>(bh) * p.Nq_pad + static_cast<size_t>(i) * kBM;
-      bulk_load(sb + 2 * G::T_BYTES, p.lse2 + row, 512, B(G::B_QF + st));
-      bulk_load(sb + 2 * G::T_BYTES + 512, p.delta + row, 512, B(G::B_QF + st));
     }
   } else if (warp == 8 && lane == 0 && T.nb > 0) {
     // ---- MMA: S(0) dP(0) | dV(n) S(n+1) dK(n) dP(n+1) | ...
@@ -317,42 +322,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm = cx.tmem;
     const uint64_t dk0 = sdesc_sw128(sbase + G::OFF_K, 16, 1024);
     const uint64_t dv0 = sdesc_sw128(sbase + G::OFF_V, 16, 1024);
-    auto st_desc = [&](int st, int which, bool mn) {  // which: 0 = Q, 1 = dO
-      const uint32_t a = sbase + G::OFF_ST + st * G::ST_BYTES + which * G::T_BYTES;
+    auto st_desc = [&](int m, bool mn) {  // ring item m: Q_{m/2} (even) or dO_{m/2} (odd)
+      const uint32_t a = sbase + G::OFF_SL + (m % G::NSLOT) * G::SLOT_BYTES;
       return mn ? sdesc_sw128(a, G::CHUNK, 1024) : sdesc_sw128(a, 16, 1024);
+    };
+    auto wait_item = [&](int m) {
+      return wait_bar(B(G::B_SLF + m % G::NSLOT), (m / G::NSLOT) & 1u, cx.abort_flag);
     };
     // P^T / dS^T of query column q: warpgroup q / 64 packed its half at its own
     // first 32 columns -> K step kk (16 queries) at (kk / 4) * 64 + (kk % 4) * 8
     auto acol = [](int kk) { return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8); };
-    bool ok = wait_bar(B(G::B_KV), 0u, cx.abort_flag);
-    uint32_t qf_ph[G::NST] = {};
-    if (ok) ok = wait_bar(B(G::B_QF + 0), 0u, cx.abort_flag);
+    bool ok = wait_bar(B(G::B_KV), 0u, cx.abort_flag) && wait_item(0) && wait_item(1);
     if (ok) {
-      qf_ph[0] ^= 1u;
       tc_fence_after();
-      mma_nt<D>(tm + G::T_S, dk0, st_desc(0, 0, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_nt<D>(tm + G::T_S, dk0, st_desc(0, false), kIdNT, G::CHUNK, G::CHUNK);
       mma_commit(B(G::B_SF));
-      mma_nt<D>(tm + G::T_DP, dv0, st_desc(0, 1, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_nt<D>(tm + G::T_DP, dv0, st_desc(1, false), kIdNT, G::CHUNK, G::CHUNK);
       mma_commit(B(G::B_DPF));
     }
     for (int n = 0; ok && n < T.nb; ++n) {
-      const int st = n % G::NST, st1 = (n + 1) % G::NST;
       if (!wait_bar(B(G::B_PF), n & 1u, cx.abort_flag)) break;
       tc_fence_after();
-      mma_tn<D>(tm + G::T_DV, tm + G::T_S, st_desc(st, 1, true), kIdTN, n > 0, acol);
+      mma_tn<D>(tm + G::T_DV, tm + G::T_S, st_desc(2 * n + 1, true), kIdTN, n > 0, acol);
+      mma_commit(B(G::B_SLE + (2 * n + 1) % G::NSLOT));  // dO_n's slot
       if (n + 1 < T.nb) {
-        if (!wait_bar(B(G::B_QF + st1), qf_ph[st1], cx.abort_flag)) break;
-        qf_ph[st1] ^= 1u;
+        if (!wait_item(2 * n + 2)) break;
         tc_fence_after();
-        mma_nt<D>(tm + G::T_S, dk0, st_desc(st1, 0, false), kIdNT, G::CHUNK, G::CHUNK);
+        mma_nt<D>(tm + G::T_S, dk0, st_desc(2 * n + 2, false), kIdNT, G::CHUNK, G::CHUNK);
         mma_commit(B(G::B_SF));
       }
       if (!wait_bar(B(G::B_DSF), n & 1u, cx.abort_flag)) break;
       tc_fence_after();
-      mma_tn<D>(tm + G::T_DK, tm + G::T_DP, st_desc(st, 0, true), kIdTN, n > 0, acol);
-      mma_commit(B(G::B_QE + st));
+      mma_tn<D>(tm + G::T_DK, tm + G::T_DP, st_desc(2 * n, true), kIdTN, n > 0, acol);
+      mma_commit(B(G::B_SLE + (2 * n) % G::NSLOT));  // Q_n's slot (and its lse2, delta)
       if (n + 1 < T.nb) {
-        mma_nt<D>(tm + G::T_DP, dv0, st_desc(st1, 1, false), kIdNT, G::CHUNK, G::CHUNK);
+        if (!wait_item(2 * n + 3)) break;
+        tc_fence_after();
+        mma_nt<D>(tm + G::T_DP, dv0, st_desc(2 * n + 3, false), kIdNT, G::CHUNK, G::CHUNK);
         mma_commit(B(G::B_DPF));
       } else {
         mma_commit(B(G::B_ACC));
@@ -365,19 +371,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.c;
     const int nqb = p.nqt - T.i0;
-    uint32_t qf_ph[G::NST] = {};
     bool ok = true;
     for (int n = 0; ok && n < T.nb; ++n) {
-      const int st = n % G::NST;
+      const int sl = (2 * n) % G::NSLOT;  // the slot of Q_n, with lse2 and delta
       const int i = T.i0 + n % nqb;
       // lse2 / delta of this block were written by the TMA unit: observe its barrier
-      ok = wait_bar(B(G::B_QF + st), qf_ph[st], cx.abort_flag) &&
+      ok = wait_bar(B(G::B_SLF + sl), ((2 * n) / G::NSLOT) & 1u, cx.abort_flag) &&
            wait_bar(B(G::B_SF), n & 1u, cx.abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
-      qf_ph[st] ^= 1u;
       tc_fence_after();
-      const float* l2 = reinterpret_cast<const float*>(gbase + G::OFF_ST + st * G::ST_BYTES +
-                                                       2 * G::T_BYTES) + h * 64;
+      const float* l2 = reinterpret_cast<const float*>(gbase + G::OFF_SL + sl * G::SLOT_BYTES +
+                                                       G::T_BYTES) + h * 64;
       const float* dl = l2 + 128;
       uint32_t sr[64];
       tmem_ld_x64(tm + G::T_S + h * 64, sr);
@@ -473,12 +477,21 @@ struct GeoQ {
   static constexpr int DCH = D / 64;
   static constexpr int T_BYTES = 128 * D * 2;
   static constexpr int CHUNK = 128 * 128;
-  static constexpr int NST = D == 64 ? 4 : 2;  // key-block stages (K, V)
-  static constexpr int OFF_Q = 0, OFF_DO = T_BYTES, OFF_ST = 2 * T_BYTES;
-  static constexpr int ST_BYTES = 2 * T_BYTES;
-  static constexpr int OFF_BAR = OFF_ST + NST * ST_BYTES;
-  static constexpr int B_QF = 0, B_KF = 1, B_KE = 1 + NST, B_SDP = 1 + 2 * NST, B_SFREE = B_SDP + 1,
-                       B_DSF = B_SDP + 2, B_DSE = B_SDP + 3, B_DQF = B_SDP + 4, NBAR = B_SDP + 5;
+  // K and V tiles stream through single-tile slots, loaded in the order
+  // K0 V0 K1 V1 ...: NKS slots take K_j in turn, NVS slots V_j.  V_j is freed
+  // after dP(j), early; K_j only after dQ(j), late -- separate slot sets let
+  // V_{j+2} reuse V_j's slot instead of waiting for K_j's.
+  static constexpr int NSLOT = D == 64 ? 10 : 5;
+  static constexpr int NVS = D == 64 ? 4 : 2, NKS = NSLOT - NVS;
+  // item m (K_{m/2} for even m, V_{m/2} for odd m): its slot, and how many
+  // items used that slot before it
+  __device__ static int slot(int m) { return (m & 1) ? NKS + (m >> 1) % NVS : (m >> 1) % NKS; }
+  __device__ static int use(int m) { return (m & 1) ? (m >> 1) / NVS : (m >> 1) / NKS; }
+  static constexpr int OFF_Q = 0, OFF_DO = T_BYTES, OFF_SL = 2 * T_BYTES;
+  static constexpr int OFF_BAR = OFF_SL + NSLOT * T_BYTES;
+  static constexpr int B_QF = 0, B_SLF = 1, B_SLE = 1 + NSLOT, B_SDP = 1 + 2 * NSLOT,
+                       B_SFREE = B_SDP + 1, B_DSF = B_SDP + 2, B_DSE = B_SDP + 3, B_DQF = B_SDP + 4,
+                       NBAR = B_SDP + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // TMEM columns: S 0..127, dP 128..255, dS (packed) 256..319, dQ 320..320+D-1
@@ -521,9 +534,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(B(G::B_QF), 1);
-    for (int s = 0; s < G::NST; ++s) {
-      mbar_init(B(G::B_KF + s), 1);
-      mbar_init(B(G::B_KE + s), 1);
+    for (int s = 0; s < G::NSLOT; ++s) {
+      mbar_init(B(G::B_SLF + s), 1);
+      mbar_init(B(G::B_SLE + s), 1);
     }
     mbar_init(B(G::B_SDP), 1);
     mbar_init(B(G::B_SFREE), 8);
@@ -554,17 +567,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sbase + G::OFF_Q + c * G::CHUNK, &tm_q, B(G::B_QF), c * 64, q0, bh, pol_first);
       tma_load_3d(sbase + G::OFF_DO + c * G::CHUNK, &tm_do, B(G::B_QF), c * 64, q0, bh, pol_first);
     }
-    for (int j = 0; j < nb; ++j) {
-      const int st = j % G::NST;
-      if (j >= G::NST && !wait_bar(B(G::B_KE + st), ((j / G::NST) - 1) & 1u, cx.abort_flag)) break;
-      const uint32_t sb = sbase + G::OFF_ST + st * G::ST_BYTES;
-      mbar_arrive_expect_tx(B(G::B_KF + st), 2 * G::T_BYTES);
+    for (int m = 0; m < 2 * nb; ++m) {  // item m: K (even) or V (odd) of block m / 2
+      const int sl = G::slot(m), u = G::use(m);
+      if (u > 0 && !wait_bar(B(G::B_SLE + sl), (u - 1) & 1u, cx.abort_flag)) break;
+      mbar_arrive_expect_tx(B(G::B_SLF + sl), G::T_BYTES);
 #pragma unroll
-      for (int c = 0; c < G::DCH; ++c) {
-        tma_load_3d(sb + c * G::CHUNK, &tm_k, B(G::B_KF + st), c * 64, j * kBN, kvz, pol_last);
-        tma_load_3d(sb + G::T_BYTES + c * G::CHUNK, &tm_v, B(G::B_KF + st), c * 64, j * kBN, kvz,
-                    pol_last);
-      }
+      for (int c = 0; c < G::DCH; ++c)
+        tma_load_3d(sbase + G::OFF_SL + sl * G::T_BYTES + c * G::CHUNK, (m & 1) ? &tm_v : &tm_k,
+                    B(G::B_SLF + sl), c * 64, (m >> 1) * kBN, kvz, pol_last);
     }
   } else if (warp == 8 && lane == 0) {
     // ---- MMA: S(0) dP(0) | S(j+1) dP(j+1) dQ(j) | ...
@@ -573,38 +583,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm = cx.tmem;
     const uint64_t dq0 = sdesc_sw128(sbase + G::OFF_Q, 16, 1024);
     const uint64_t ddo0 = sdesc_sw128(sbase + G::OFF_DO, 16, 1024);
-    auto kv_desc = [&](int st, int which, bool mn) {  // which: 0 = K, 1 = V
-      const uint32_t a = sbase + G::OFF_ST + st * G::ST_BYTES + which * G::T_BYTES;
+    // ring item m (K_{m/2} or V_{m/2}): its slot, and the parity of its fill
+    auto kv_desc = [&](int m, bool mn) {
+      const uint32_t a = sbase + G::OFF_SL + G::slot(m) * G::T_BYTES;
       return mn ? sdesc_sw128(a, G::CHUNK, 1024) : sdesc_sw128(a, 16, 1024);
+    };
+    auto wait_item = [&](int m) {
+      return wait_bar(B(G::B_SLF + G::slot(m)), G::use(m) & 1u, cx.abort_flag);
+    };
+    // S(j) and dP(j); V_j's slot is free once dP(j) completes
+    auto issue_sdp = [&](int j) {
+      mma_nt<D>(tm + G::T_S, dq0, kv_desc(2 * j, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_nt<D>(tm + G::T_DP, ddo0, kv_desc(2 * j + 1, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_commit(B(G::B_SDP));
+      mma_commit(B(G::B_SLE + G::slot(2 * j + 1)));
     };
     // dS of key column k: warpgroup k / 64 packed its half at columns (k / 64) * 32 ..
     auto acol = [](int kk) { return static_cast<uint32_t>(kk * 8); };
-    uint32_t kf_ph[G::NST] = {};
-    bool ok = wait_bar(B(G::B_QF), 0u, cx.abort_flag);
-    if (ok) ok = wait_bar(B(G::B_KF + 0), 0u, cx.abort_flag);
+    bool ok = wait_bar(B(G::B_QF), 0u, cx.abort_flag) && wait_item(0) && wait_item(1);
     if (ok) {
-      kf_ph[0] ^= 1u;
       tc_fence_after();
-      mma_nt<D>(tm + G::T_S, dq0, kv_desc(0, 0, false), kIdNT, G::CHUNK, G::CHUNK);
-      mma_nt<D>(tm + G::T_DP, ddo0, kv_desc(0, 1, false), kIdNT, G::CHUNK, G::CHUNK);
-      mma_commit(B(G::B_SDP));
+      issue_sdp(0);
     }
     for (int j = 0; ok && j < nb; ++j) {
-      const int st = j % G::NST, st1 = (j + 1) % G::NST;
       if (j + 1 < nb) {  // next S and dP once the compute warps have read this block's
         if (!wait_bar(B(G::B_SFREE), j & 1u, cx.abort_flag)) break;
-        if (!wait_bar(B(G::B_KF + st1), kf_ph[st1], cx.abort_flag)) break;
-        kf_ph[st1] ^= 1u;
+        if (!wait_item(2 * j + 2) || !wait_item(2 * j + 3)) break;
         tc_fence_after();
-        mma_nt<D>(tm + G::T_S, dq0, kv_desc(st1, 0, false), kIdNT, G::CHUNK, G::CHUNK);
-        mma_nt<D>(tm + G::T_DP, ddo0, kv_desc(st1, 1, false), kIdNT, G::CHUNK, G::CHUNK);
-        mma_commit(B(G::B_SDP));
+        issue_sdp(j + 1);
       }
       if (!wait_bar(B(G::B_DSF), j & 1u, cx.abort_flag)) break;
       tc_fence_after();
-      mma_tn<D>(tm + G::T_DQ, tm + G::T_DS, kv_desc(st, 0, true), kIdTN, j > 0, acol);
+      mma_tn<D>(tm + G::T_DQ, tm + G::T_DS, kv_desc(2 * j, true), kIdTN, j > 0, acol);
       mma_commit(B(G::B_DSE));
-      mma_commit(B(G::B_KE + st));
+      mma_commit(B(G::B_SLE + G::slot(2 * j)));  // K_j's slot
       if (j + 1 == nb) mma_commit(B(G::B_DQF));
     }
   } else if (warp < 8) {
