@@ -141,6 +141,7 @@ struct Tile {
   int row0;   // first query row of the work tile
   int kvz;    // b * Hkv + kv head
   int nblk[2];
+  int j0[2];  // key windows, two query tiles: query tile q uses blocks j0[q] .. j0[q] + nblk[q] - 1
   int nb;
   int jb;     // first key block of this unit
   int slot;    // split-tile index, or -1 for a whole tile
@@ -149,7 +150,7 @@ struct Tile {
   int store0;  // workspace index of part 0 (parts are stored consecutively)
 };
 
-template <int NQ>
+template <int NQ, bool WIN = false>
 __device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
   Tile T;
   int t = u;
@@ -200,6 +201,26 @@ __device__ __forceinline__ Tile get_tile(const FwdParams& p, int u) {
   }
   T.row0 = qt * NQ * kBM;
   const int rows = p.pack_g > 1 ? p.pack_g * p.Nq : p.Nq;  // rows of the (packed) tile space
+  T.j0[0] = T.j0[1] = 0;
+  if constexpr (WIN) {  // key windows, two query tiles: each its own range in the union
+    int lo[2] = {0, 0}, hi[2] = {0, 0};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int rf = T.row0 + q * kBM;
+      const int rl = min(rf + kBM - 1, p.Nq - 1);
+      const int hk = p.wr >= 0 ? min(p.Nk - 1, rl + p.wr) : p.Nk - 1;
+      const int lk = p.wl >= 0 ? max(0, rf - p.wl) : 0;
+      lo[q] = min(lk / kBN, p.nkb - 1);
+      hi[q] = max(lo[q], hk / kBN);  // at least one block (rows with no key: O = 0, LSE = -inf)
+    }
+    const bool two = T.row0 + kBM < rows;
+    T.jb = lo[0];
+    T.nb = (two ? hi[1] : hi[0]) - lo[0] + 1;
+    T.nblk[0] = hi[0] - lo[0] + 1;
+    T.nblk[1] = two ? hi[1] - lo[1] + 1 : 0;
+    T.j0[1] = two ? lo[1] - lo[0] : 0;
+    return T;
+  }
   T.jb = kb0;
   T.nb = 0;
 #pragma unroll
@@ -374,7 +395,7 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, bool bf16) {
 // (broadcast over queries), 2 = a bias per query head, 4 = a bias per batch.
 constexpr int kBiasRowBcast = 1, kBiasPerHead = 2, kBiasPerBatch = 4;
 
-template <int D, int NQ, bool BIAS = false>
+template <int D, int NQ, bool BIAS = false, bool WIN = false>
 __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, const CUtensorMap* tq,
                                           const CUtensorMap* tq4, const CUtensorMap* tk,
                                           const CUtensorMap* tv, const CUtensorMap* tb,
@@ -449,7 +470,7 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
   uint32_t n_units_seen = 0;
   int t;
   while (ok && produce_unit<D, NQ, BIAS>(cx, p, it, n_units_seen, t)) {
-    const Tile T = get_tile<NQ>(p, t);
+    const Tile T = get_tile<NQ, WIN>(p, t);
     // Q0, then K0 (the first S MMA of the tile needs only these), then Q1 -- each
     // Q tile waits only for the last S MMA that read its previous contents.
     // K/V block order matches the MMA warp's consumption order:
@@ -482,7 +503,7 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
 }
 
 // ---------------------------------------------------------------- MMA issuer
-template <int D, int NQ, bool BF16, bool BIAS = false>
+template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false>
 __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
   using G = Geometry<D, NQ, BIAS>;
   constexpr uint32_t kIdS = idesc_f16(kBM, kBN, BF16, false);  // Q, K both K-major
@@ -550,11 +571,64 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
   uint32_t n_units_seen = 0;
   int t;
   while (consume_unit<D, NQ, BIAS>(cx, p, it, n_units_seen, t, -1)) {
-    const Tile T = get_tile<NQ>(p, t);
+    const Tile T = get_tile<NQ, WIN>(p, t);
     const int nb = T.nb;
     int kst;
     if (!consume(kst)) return;
-    if (NQ == 2) {
+    if (NQ == 2 && WIN) {
+      // key windows: the same stream, query tile q taking part in blocks
+      // j0[q] <= j < j0[q] + nblk[q] of the unit (j0[0] = 0)
+      const int s1 = T.j0[1], e0 = T.nblk[0], e1 = T.j0[1] + T.nblk[1];
+      auto in1 = [&](int j) { return j >= s1 && j < e1; };
+      if (e0 > 0) {
+        if (!q_ready(0)) return;
+        issue_S(0, 0, kst);
+        mma_commit(B(G::B_SFULL + 0));
+        if (e0 == 1) mma_commit(B(G::B_QEMPTY + 0));
+      }
+      if (in1(0)) {
+        if (!q_ready(1)) return;
+        issue_S(1, 1, kst);
+        mma_commit(B(G::B_SFULL + 1));
+        if (e1 == 1) mma_commit(B(G::B_QEMPTY + 1));
+      }
+      mma_commit(B(G::B_KVEMPTY + kst));
+      for (int j = 0; j < nb; ++j) {
+        int vst;
+        if (!consume(vst)) return;
+        if (j < e0) {
+          if (j == 0 && !o_ready(0)) return;
+          if (!p_ready(0)) return;
+          issue_PV(0, 0, vst, j > 0);
+          if (j == e0 - 1) { mma_commit(B(G::B_OFULL + 0)); o_pending[0] = true; }
+        }
+        int kst2 = -1;
+        if (j + 1 < nb) {
+          if (!consume(kst2)) return;
+          if (j + 1 < e0) {
+            issue_S(0, 0, kst2);
+            mma_commit(B(G::B_SFULL + 0));
+            if (j + 1 == e0 - 1) mma_commit(B(G::B_QEMPTY + 0));
+          }
+        }
+        if (in1(j)) {
+          if (j == s1 && !o_ready(1)) return;
+          if (!p_ready(1)) return;
+          issue_PV(1, 1, vst, j > s1);
+          if (j == e1 - 1) { mma_commit(B(G::B_OFULL + 1)); o_pending[1] = true; }
+        }
+        mma_commit(B(G::B_KVEMPTY + vst));
+        if (kst2 >= 0) {
+          if (in1(j + 1)) {
+            if (j + 1 == s1 && !q_ready(1)) return;
+            issue_S(1, 1, kst2);
+            mma_commit(B(G::B_SFULL + 1));
+            if (j + 1 == e1 - 1) mma_commit(B(G::B_QEMPTY + 1));
+          }
+          mma_commit(B(G::B_KVEMPTY + kst2));
+        }
+      }
+    } else if (NQ == 2) {
       // stream: S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
       // q_empty[q] is committed right after the last S MMA that reads Q_q.
       if (T.nblk[0] > 0) {
@@ -749,7 +823,7 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
-template <int D, int NQ, bool BF16, bool BIAS = false>
+template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false>
 __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, int wg, int sub,
                                              int lane, int bias_mode) {
   using G = Geometry<D, NQ, BIAS>;
@@ -757,7 +831,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   const uint32_t tm = cx.tmem + lane_off;
   auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
   const float c = p.c;
-  constexpr bool kWin = NQ == 1;  // key windows: one-query-tile kernels only
+  constexpr bool kWin = NQ == 1 || WIN;  // kernels that take key windows
   uint32_t s_phase[2] = {0u, 0u}, of_phase = 0u, pv_seen = 0u;
   uint32_t b_cnt = 0, b_phase = 0u;  // bias tiles consumed; parity bit per stage
   const int q = (NQ == 2) ? wg : 0;
@@ -770,10 +844,10 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     // the unit again (registers are the softmax warps' tightest resource).
     int nblk, rfirst, jb;
     {
-      const Tile T0 = get_tile<NQ>(p, t);
+      const Tile T0 = get_tile<NQ, WIN>(p, t);
       nblk = T0.nblk[q];
       rfirst = T0.row0 + q * kBM;
-      jb = T0.jb;
+      jb = WIN ? T0.jb + T0.j0[q] : T0.jb;
     }
     if (nblk == 0) continue;
     // query position of this thread's row (causal mask; packing is non-causal only)
@@ -921,7 +995,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     tc_fence_after();
     int t_again;  // opaque copy: the compiler must not keep the first decode live
     asm volatile("mov.b32 %0, %1;" : "=r"(t_again) : "r"(t));
-    const Tile T = get_tile<NQ>(p, t_again);
+    const Tile T = get_tile<NQ, WIN>(p, t_again);
     const RowInfo ri = row_info(p, T, q, sub * 32 + lane);
     const bool live = ri.live;
     const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
@@ -957,7 +1031,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   }
 }
 
-template <int D, int NQ, bool BF16, bool BIAS = false>
+template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q4,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -1028,11 +1102,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) setmaxnreg_inc<kSoftmaxRegs>();
   else setmaxnreg_dec<kOtherRegs>();
   if (warp < 8) {
-    if (NQ == 2 || warp < 4) role_softmax<D, NQ, BF16, BIAS>(cx, p, warp >> 2, warp & 3, lane, bias_mode);
+    if (NQ == 2 || warp < 4)
+      role_softmax<D, NQ, BF16, BIAS, WIN>(cx, p, warp >> 2, warp & 3, lane, bias_mode);
   } else if (warp == 8) {
-    if (lane == 0) role_mma<D, NQ, BF16, BIAS>(cx, p);
+    if (lane == 0) role_mma<D, NQ, BF16, BIAS, WIN>(cx, p);
   } else if (warp == 9) {
-    if (lane == 0) role_load<D, NQ, BIAS>(cx, p, &tm_q, &tm_q4, &tm_k, &tm_v, &tm_b, bias_mode);
+    if (lane == 0) role_load<D, NQ, BIAS, WIN>(cx, p, &tm_q, &tm_q4, &tm_k, &tm_v, &tm_b, bias_mode);
   }
   __syncwarp();
   tc_fence_before();
@@ -1202,7 +1277,7 @@ bool make_bias_map(CUtensorMap* m, const BiasArg& a, int B, int H, int Nq, int N
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int NQ, bool BF16, bool BIAS = false>
+template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
            int Hkv, int Nq, int Nk, float scale, int causal, int wl, int wr, cudaStream_t stream,
            int dev, void* ws, size_t ws_bytes, Scratch mode, const BiasArg* bias = nullptr) {
@@ -1212,7 +1287,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   {
     std::lock_guard<std::mutex> lk(mu);
     if (!attr_done[dev]) {
-      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, NQ, BF16, BIAS>,
+      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, NQ, BF16, BIAS, WIN>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                G::SMEM_BYTES) != cudaSuccess)
         return FA_ERR_LAUNCH;
@@ -1329,7 +1404,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     bias_mode = (bias->sq ? 0 : fa::kBiasRowBcast) | (bias->sh ? fa::kBiasPerHead : 0) |
                 (bias->sb ? fa::kBiasPerBatch : 0);
   }
-  fa::fa_fwd_kernel<D, NQ, BF16, BIAS><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(
+  fa::fa_fwd_kernel<D, NQ, BF16, BIAS, WIN><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(
       tq, tq4, tk, tv, p, tb, bias_mode);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
@@ -1429,8 +1504,16 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
     }
 #undef FA_BARGS
   }
-  // Windowed launches too: each tile gets its own key block range.
+  // Windowed launches: each query tile gets its own key block range; tiles of
+  // 256 rows (D <= 128) run the two-query-tile kernel's windowed variant.
   const bool windowed = wl >= 0 || wr >= 0;
+  if (windowed && D <= 128 && Nq > fa::kBM) {
+#define FA_WARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, wl, wr, st, dev, ws, ws_bytes, mode
+    if (D == 64)
+      return bf ? launch<64, 2, true, false, true>(FA_WARGS) : launch<64, 2, false, false, true>(FA_WARGS);
+    return bf ? launch<128, 2, true, false, true>(FA_WARGS) : launch<128, 2, false, false, true>(FA_WARGS);
+#undef FA_WARGS
+  }
   const bool one_tile =
       windowed || (pack_heads(Hq, Hkv, Nq, causal) ? (Hq / Hkv) * Nq : Nq) <= fa::kBM;
 #define FA_ARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, wl, wr, st, dev, ws, ws_bytes, mode
