@@ -51,6 +51,7 @@ def parse():
                     help="skip the sliding-window measurement")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward-pass measurement")
+    ap.add_argument("--no-bias", action="store_true", help="skip the score-bias measurement")
     return ap.parse_args()
 
 
@@ -376,6 +377,30 @@ def main():
         del bdo, bws, bdq, bdk, bdv
         assert fa.device_status(reset=True) == 0
 
+    # ---- additive score bias on the bench workload: one [N, N] bias shared by all heads
+    bias_line = {}
+    if not args.no_bias:
+        w = ws[0]  # non-causal pass
+        g1 = torch.Generator(device=dev).manual_seed(2)
+        bb = torch.randn((1, 1, w.Nq, w.Nk), device=dev, dtype=q.dtype, generator=g1)
+        bo, bl = torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        ts = []
+        for i in range(13):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fa.fa_fwd(q, k, v, o=bo, lse=bl, scale=w.softmax_scale, bias=bb, stream=sptr)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        ms = statistics.median(ts)
+        bias_line = {"workload": "LLaMA-7B layer non-causal + shared [N, N] fp16 bias",
+                     "ms": round(ms, 4), "tflops": round(w.flops() / (ms * 1e-3) / 1e12, 1),
+                     "frac_of_peak": round(w.flops() / (ms * 1e-3) / 1e12 / peaks()[0], 3)}
+        del bb, bo, bl
+        assert fa.device_status(reset=True) == 0
+
     # ---- sliding-window attention (causal, 1024-key window, 8192 positions, GQA 4)
     window = {}
     if not args.no_window:
@@ -469,6 +494,7 @@ def main():
         "decode": decode,
         "window": window,
         "backward": backward,
+        "bias": bias_line,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
