@@ -57,6 +57,9 @@ def _load():
             ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
             ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
             ctypes.c_int64, ctypes.c_int]
+        lib.oracle_attention_bwd_ex.restype = ctypes.c_int
+        lib.oracle_attention_bwd_ex.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64] * 6 + [
+            ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
         lib.oracle_attention_bwd.restype = ctypes.c_int
         lib.oracle_attention_bwd.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64] * 6 + [
             ctypes.c_double, ctypes.c_int, ctypes.c_int]
@@ -134,10 +137,13 @@ def attention(q, k, v, scale: float, causal: bool, rows: Optional[np.ndarray] = 
     return o, lse
 
 
-def attention_bwd(q, k, v, dout, scale: float, causal: bool, nthreads: int = 0):
+def attention_bwd(q, k, v, dout, scale: float, causal: bool, nthreads: int = 0,
+                  window: Tuple[int, int] = (-1, -1)):
     """Gradients of attention in float64 for the upstream gradient dout.
 
     q, dout: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] (torch tensors or numpy arrays).
+    window: (left, right) key window as in attention(); rows with no visible
+    key contribute nothing.
     Returns (dQ [B, Hq, Nq, D], dK [B, Hkv, Nk, D], dV [B, Hkv, Nk, D],
     Delta [B, Hq, Nq]) as float64 numpy arrays; Delta_i = dO_i . O_i.
     """
@@ -151,10 +157,11 @@ def attention_bwd(q, k, v, dout, scale: float, causal: bool, nthreads: int = 0):
     dk = np.empty((B, Hkv, Nk, D), dtype=np.float64)
     dv = np.empty((B, Hkv, Nk, D), dtype=np.float64)
     delta = np.empty((B, Hq, Nq), dtype=np.float64)
-    rc = lib.oracle_attention_bwd(qf.ctypes.data, kf.ctypes.data, vf.ctypes.data, gf.ctypes.data,
-                                  dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, delta.ctypes.data,
-                                  B, Hq, Hkv, Nq, Nk, D, float(scale), int(bool(causal)),
-                                  int(nthreads))
+    wl, wr = (int(x) for x in window)
+    rc = lib.oracle_attention_bwd_ex(qf.ctypes.data, kf.ctypes.data, vf.ctypes.data,
+                                     gf.ctypes.data, dq.ctypes.data, dk.ctypes.data,
+                                     dv.ctypes.data, delta.ctypes.data, B, Hq, Hkv, Nq, Nk, D,
+                                     float(scale), int(bool(causal)), wl, wr, int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_attention_bwd rejected its arguments (code {rc})")
     return dq, dk, dv, delta

@@ -179,15 +179,19 @@ int oracle_attention(const float *q, const int64_t *q_pos, int64_t R, const floa
  *   dK_j  += scale * dS_ij q_i
  *
  * GQA: dK and dV of a key/value head sum over the query heads of its group.
+ * Key windows (oracle_attention_bwd_ex; same reading as the forward pass):
+ * the sums run over the keys i - window_left .. i + window_right only; a row
+ * with no such key has O = 0, so it contributes nothing (dQ_i = 0, Delta_i = 0).
  * All arrays are float32 inputs (rounded values) and float64 outputs:
  * q, dout [B, Hq, Nq, D]; k, v [B, Hkv, Nk, D]; dq [B, Hq, Nq, D];
  * dk, dv [B, Hkv, Nk, D]; delta [B, Hq, Nq] (may be NULL).
  * Returns 0, or a negative number for invalid arguments.
  */
-int oracle_attention_bwd(const float *q, const float *k, const float *v, const float *dout,
-                         double *dq, double *dk, double *dv, double *delta, int64_t B,
-                         int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
-                         double scale, int causal, int nthreads) {
+int oracle_attention_bwd_ex(const float *q, const float *k, const float *v, const float *dout,
+                            double *dq, double *dk, double *dv, double *delta, int64_t B,
+                            int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
+                            double scale, int causal, int64_t window_left,
+                            int64_t window_right, int nthreads) {
     if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
     if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || D < 1) return -2;
     if (Hq % Hkv != 0) return -3;
@@ -222,24 +226,34 @@ int oracle_attention_bwd(const float *q, const float *k, const float *v, const f
                     const float *qi = q + (bh * Nq + i) * D;
                     const float *gi = dout + (bh * Nq + i) * D;
                     double *dqi = dq + (bh * Nq + i) * D;
-                    const int64_t n_vis = causal ? (i + 1 < Nk ? i + 1 : Nk) : Nk;
+                    /* visible keys j0 .. j1 (inclusive) */
+                    int64_t j0 = 0, j1 = Nk - 1;
+                    if (causal && i < j1) j1 = i;
+                    if (window_right >= 0 && i + window_right < j1) j1 = i + window_right;
+                    if (window_left >= 0 && i - window_left > j0) j0 = i - window_left;
+                    double *dqi0 = dq + (bh * Nq + i) * D;
+                    if (j1 < j0) { /* no visible key: O = 0, nothing to propagate */
+                        for (int64_t d = 0; d < D; ++d) dqi0[d] = 0.0;
+                        if (delta) delta[bh * Nq + i] = 0.0;
+                        continue;
+                    }
                     /* forward softmax of the row */
                     double M = -INFINITY;
-                    for (int64_t j = 0; j < n_vis; ++j) {
+                    for (int64_t j = j0; j <= j1; ++j) {
                         double acc = 0.0;
                         for (int64_t d = 0; d < D; ++d) acc += (double)qi[d] * (double)kb[j * D + d];
                         p[j] = scale * acc;
                         if (p[j] > M) M = p[j];
                     }
                     double Z = 0.0;
-                    for (int64_t j = 0; j < n_vis; ++j) {
+                    for (int64_t j = j0; j <= j1; ++j) {
                         p[j] = exp(p[j] - M);
                         Z += p[j];
                     }
-                    for (int64_t j = 0; j < n_vis; ++j) p[j] /= Z;
+                    for (int64_t j = j0; j <= j1; ++j) p[j] /= Z;
                     /* dP, Delta */
                     double dl = 0.0;
-                    for (int64_t j = 0; j < n_vis; ++j) {
+                    for (int64_t j = j0; j <= j1; ++j) {
                         double acc = 0.0;
                         for (int64_t d = 0; d < D; ++d) acc += (double)gi[d] * (double)vb[j * D + d];
                         dp[j] = acc;
@@ -248,7 +262,7 @@ int oracle_attention_bwd(const float *q, const float *k, const float *v, const f
                     if (delta) delta[bh * Nq + i] = dl;
                     /* dS, then the three gradients */
                     for (int64_t d = 0; d < D; ++d) dqi[d] = 0.0;
-                    for (int64_t j = 0; j < n_vis; ++j) {
+                    for (int64_t j = j0; j <= j1; ++j) {
                         const double ds = p[j] * (dp[j] - dl);
                         for (int64_t d = 0; d < D; ++d) {
                             dqi[d] += scale * ds * (double)kb[j * D + d];
@@ -263,6 +277,15 @@ int oracle_attention_bwd(const float *q, const float *k, const float *v, const f
         free(dp);
     }
     return err;
+}
+
+/* The unwindowed gradients (causal or not). */
+int oracle_attention_bwd(const float *q, const float *k, const float *v, const float *dout,
+                         double *dq, double *dk, double *dv, double *delta, int64_t B,
+                         int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
+                         double scale, int causal, int nthreads) {
+    return oracle_attention_bwd_ex(q, k, v, dout, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk, D, scale,
+                                   causal, -1, -1, nthreads);
 }
 
 int oracle_max_threads(void) {

@@ -129,3 +129,92 @@ def test_delta_is_dout_dot_output():
     _, _, _, delta = oracle.attention_bwd(q, k, v, g, 0.5, True)
     o, _ = oracle.attention(q, k, v, 0.5, True)
     np.testing.assert_allclose(delta, (g.astype(np.float64) * o).sum(-1), rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- key windows
+def _forward64_window(q, k, v, scale, causal, wl, wr):
+    """Windowed softmax(scale q k^T) v in float64; rows with no visible key give 0."""
+    g = q.shape[1] // k.shape[1]
+    kr, vr = np.repeat(k, g, axis=1), np.repeat(v, g, axis=1)
+    s = scale * np.einsum("bhid,bhjd->bhij", q, kr)
+    i, j = np.meshgrid(np.arange(q.shape[2]), np.arange(k.shape[2]), indexing="ij")
+    keep = np.ones_like(i, dtype=bool)
+    if causal:
+        keep &= j <= i
+    if wl >= 0:
+        keep &= j >= i - wl
+    if wr >= 0:
+        keep &= j <= i + wr
+    s = np.where(keep, s, -np.inf)
+    m = s.max(axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    p = np.exp(s - m)
+    z = p.sum(axis=-1, keepdims=True)
+    p = np.divide(p, z, out=np.zeros_like(p), where=z > 0)
+    return np.einsum("bhij,bhjd->bhid", p, vr)
+
+
+@pytest.mark.parametrize("causal,wl,wr,nq,nk", [(False, 2, 1, 6, 7), (True, 3, -1, 7, 7),
+                                                 (False, 1, 2, 9, 5)])  # the last: rows 7, 8 see no key
+def test_window_finite_differences(causal, wl, wr, nq, nk):
+    q, k, v = _rand((1, 2, nq, 3), 40), _rand((1, 1, nk, 3), 41), _rand((1, 1, nk, 3), 42)
+    g = _rand((1, 2, nq, 3), 43)
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.8, causal, window=(wl, wr))
+    x = [q.astype(np.float64), k.astype(np.float64), v.astype(np.float64)]
+    o_or, _ = oracle.attention(q, k, v, 0.8, causal, window=(wl, wr))
+    np.testing.assert_allclose(_forward64_window(*x, 0.8, causal, wl, wr), o_or, rtol=1e-12, atol=1e-13)
+    h = 1e-5
+
+    def loss(xs):
+        return float(np.sum(g.astype(np.float64) * _forward64_window(*xs, 0.8, causal, wl, wr)))
+
+    for which, grad in enumerate((dq, dk, dv)):
+        fd = np.zeros_like(grad)
+        for idx in np.ndindex(*grad.shape):
+            xp = [a.copy() for a in x]
+            xm = [a.copy() for a in x]
+            xp[which][idx] += h
+            xm[which][idx] -= h
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * h)
+        np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal,wl,wr", [(False, 8, 4), (True, 16, -1), (False, -1, 10)])
+def test_window_against_torch_autograd(causal, wl, wr):
+    q, k, v = _rand((2, 4, 40, 8), 44), _rand((2, 2, 40, 8), 45), _rand((2, 2, 40, 8), 46)
+    g = _rand((2, 4, 40, 8), 47)
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.4, causal, window=(wl, wr))
+    i, j = np.meshgrid(np.arange(40), np.arange(40), indexing="ij")
+    keep = np.ones((40, 40), dtype=bool)
+    if causal:
+        keep &= j <= i
+    if wl >= 0:
+        keep &= j >= i - wl
+    if wr >= 0:
+        keep &= j <= i + wr
+    qt, kt, vt = (torch.from_numpy(a).double().requires_grad_() for a in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt.repeat_interleave(2, dim=1), vt.repeat_interleave(2, dim=1),
+        attn_mask=torch.from_numpy(keep), scale=0.4)
+    o.backward(torch.from_numpy(g).double())
+    np.testing.assert_allclose(dq, qt.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_window_special_cases():
+    q, k, v = _rand((1, 2, 12, 4), 48), _rand((1, 2, 12, 4), 49), _rand((1, 2, 12, 4), 50)
+    g = _rand((1, 2, 12, 4), 51)
+    a = oracle.attention_bwd(q, k, v, g, 0.5, False, window=(-1, 0))
+    b = oracle.attention_bwd(q, k, v, g, 0.5, True)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+    a = oracle.attention_bwd(q, k, v, g, 0.5, False, window=(50, 50))
+    b = oracle.attention_bwd(q, k, v, g, 0.5, False)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+    # (0, 0): O_i = v_i, so dV = dO and dQ = dK = 0
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.5, False, window=(0, 0))
+    np.testing.assert_array_equal(dq, 0.0)
+    np.testing.assert_array_equal(dk, 0.0)
+    np.testing.assert_array_equal(dv, g.astype(np.float64))
