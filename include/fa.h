@@ -196,6 +196,19 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const voi
            int D, float scale, int causal, void *stream, int dtype, void *workspace,
            size_t workspace_bytes);
 
+/*
+ * fa_bwd with a key window (the gradient of fa_fwd_window's operation): query
+ * i sees keys i - window_left .. i + window_right (-1: no bound; causal = 1 is
+ * window_right = 0, which must then be -1 or 0, else FA_ERR_BAD_WINDOW).  A
+ * row that saw no key (its lse is -inf) contributes nothing: its dQ row is 0.
+ * Key/query blocks wholly outside the windows are skipped.  Other arguments
+ * and errors as fa_bwd; window_left = window_right = -1 is fa_bwd.
+ */
+int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                  const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq,
+                  int Nk, int D, float scale, int causal, int window_left, int window_right,
+                  void *stream, int dtype, void *workspace, size_t workspace_bytes);
+
 /* Workspace bytes fa_bwd needs: 8 * B * Hq * (Nq rounded up to 128); 0 for bad sizes. */
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq);
 

@@ -131,3 +131,16 @@ def test_bias_entry_point_host_checks(lib):
     assert call(bias=4 * A + 256) == 12  # overlaps o
     if not torch.cuda.is_available():
         assert call() == 8 and call(sb=4096, sh=64 * 64, sq=64) == 8
+
+
+
+def test_bwd_window_host_checks(lib):
+    a = dict(GOOD)
+
+    def call(wl, wr, causal=0):
+        return lib.fa_bwd_window(a["q"], a["k"], a["v"], 6 * A, 7 * A, 8 * A, 9 * A, 10 * A, 11 * A,
+                                 a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], a["D"],
+                                 ctypes.c_float(a["scale"]), causal, wl, wr, None, a["dtype"],
+                                 12 * A, 1 << 20)
+    assert call(-2, 0) == fa.FA_ERR_BAD_WINDOW and call(3, -5) == fa.FA_ERR_BAD_WINDOW
+    assert call(8, 2, causal=1) == fa.FA_ERR_BAD_WINDOW

@@ -30,12 +30,13 @@ def _dout(w):
     return torch.from_numpy(g).to(torch.float16 if w.dtype == "fp16" else torch.bfloat16)
 
 
-def _run(w, dev):
+def _run(w, dev, window=(-1, -1)):
     q, k, v = make_qkv(w)
     g = _dout(w)
     qd, kd, vd, gd = (x.to(dev) for x in (q, k, v, g))
-    o, lse = fa.fa_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal)
-    dq, dk, dv = fa.fa_bwd(qd, kd, vd, o, lse, gd, scale=w.softmax_scale, causal=w.causal)
+    o, lse = fa.fa_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal, window=window)
+    dq, dk, dv = fa.fa_bwd(qd, kd, vd, o, lse, gd, scale=w.softmax_scale, causal=w.causal,
+                           window=window)
     torch.cuda.synchronize()
     assert fa.device_status(reset=True) == 0
     return (q, k, v, g), (dq, dk, dv)
@@ -96,3 +97,22 @@ def test_bwd_sum_invariants_on_device(cuda_dev):
     want = g.double().sum(dim=2).numpy()
     np.testing.assert_allclose(s_dv, want, rtol=0, atol=0.05 * np.abs(want).max())
     assert np.abs(dk.double().sum(dim=2).cpu().numpy()).max() <= 0.02 * np.abs(dk.double().cpu().numpy()).sum(2).max()
+
+
+# key windows (the gradient of fa_fwd_window's operation)
+WINDOW_CASES = [
+    (Workload("bwd sliding causal 255 D128 fp16", 1, 4, 2, 1000, 1000, 128, "fp16", True, seed=131), (255, -1)),
+    (Workload("bwd local 100/50 D64 bf16", 2, 2, 2, 777, 777, 64, "bf16", False, seed=132), (100, 50)),
+    (Workload("bwd narrow 5/3 D128 fp16", 1, 2, 2, 600, 600, 128, "fp16", False, seed=133), (5, 3)),
+    # queries 410.. see no key (Nq > Nk + left): their dQ rows are 0
+    (Workload("bwd empty rows D64 fp16", 1, 2, 2, 700, 300, 64, "fp16", False, seed=134), (110, 10)),
+    (Workload("bwd right only 64 D128 bf16 GQA", 1, 4, 2, 500, 600, 128, "bf16", False, seed=135), (-1, 64)),
+    (Workload("bwd causal window 128 D128 fp16 Nk>Nq", 1, 2, 2, 300, 900, 128, "fp16", True, seed=136), (128, 0)),
+]
+
+
+@pytest.mark.parametrize("w,window", WINDOW_CASES, ids=lambda c: c.name if hasattr(c, "name") else str(c))
+def test_bwd_window_parity(cuda_dev, w, window):
+    (q, k, v, g), got = _run(w, cuda_dev, window)
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, w.softmax_scale, w.causal, window=window)
+    _check(w, got, (dq, dk, dv), f" window {window}")

@@ -26,7 +26,8 @@ FA_ERR_BAD_WORKSPACE = 15
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
-            "fa_fwd_window", "fa_fwd_bias", "fa_bwd", "fa_bwd_workspace_size",
+            "fa_fwd_window", "fa_fwd_bias", "fa_bwd", "fa_bwd_window",
+            "fa_bwd_workspace_size",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
             "fa_status_string", "fa_device_status", "fa_device_timeout_site",
             "fa_debug_exp2_fma", "fa_debug_wait_timeout", "fa_fwd_num_tiles")
@@ -66,6 +67,8 @@ def load_library() -> ctypes.CDLL:
     lib.fa_fwd_bias.restype = i
     lib.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, vp, i, vp, ctypes.c_size_t]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_window.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, i, i, vp, i, vp, ctypes.c_size_t]
+    lib.fa_bwd_window.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i]
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_fwd_noalloc.argtypes = fwd_args + [i]
@@ -231,14 +234,16 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
 
 
 def fa_bwd(q, k, v, o, lse, dout, scale: Optional[float] = None, causal: bool = False,
-           dq=None, dk=None, dv=None, stream=None, workspace=None):
+           dq=None, dk=None, dv=None, stream=None, workspace=None,
+           window: Tuple[int, int] = (-1, -1)):
     """Gradients of the attention forward pass (three kernels on the current stream).
 
     q, o, dout: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] contiguous CUDA tensors of
     one dtype (fp16 or bf16); lse: float32 [B, Hq, Nq] from fa_fwd.  D must be
     64 or 128.  Optional outputs dq (like q), dk, dv (like k); optional
     workspace: a uint8 CUDA tensor of at least fa_bwd_workspace_size bytes
-    (allocated here when None).  Returns (dq, dk, dv).
+    (allocated here when None).  window: (left, right) key window of the
+    forward pass (fa_bwd_window), -1 = unbounded.  Returns (dq, dk, dv).
     """
     import torch
 
@@ -271,10 +276,11 @@ def fa_bwd(q, k, v, o, lse, dout, scale: Optional[float] = None, causal: bool = 
     elif hasattr(stream, "cuda_stream"):
         stream = stream.cuda_stream
     dtype = FA_BF16 if q.dtype == torch.bfloat16 else FA_FP16
-    rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
-                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq,
-                    Nk, D, ctypes.c_float(scale), 1 if causal else 0, stream or None, dtype,
-                    workspace.data_ptr(), workspace.numel())
+    wl, wr = (int(x) for x in window)
+    rc = lib.fa_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                           lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv,
+                           Nq, Nk, D, ctypes.c_float(scale), 1 if causal else 0, wl, wr,
+                           stream or None, dtype, workspace.data_ptr(), workspace.numel())
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
     return dq, dk, dv

@@ -110,6 +110,8 @@ struct BwdParams {
   const float* lse2;   // [B*Hq][Nq_pad] LSE * log2(e); +inf in the padding
   const float* delta;  // [B*Hq][Nq_pad] rowsum(dO * O); 0 in the padding
   int B, Hq, Hkv, Nq, Nk, Nq_pad, group, causal;
+  // key window: query i sees keys i - wl .. i + wr (-1: no bound); wr is 0 when causal
+  int wl, wr;
   float c;      // scale * log2(e)
   float scale;
   int nqt, nkt;  // query / key blocks per head
@@ -154,7 +156,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (sub == 0 && row < total) {
       delta[row] = live ? acc : 0.f;
-      lse2[row] = live ? lse[bh * Nq + i] * kLog2e : INFINITY;
+      // a row that saw no key (LSE = -inf, key windows) gets +inf: P = 0 there
+      const float L = live ? lse[bh * Nq + i] : -INFINITY;
+      lse2[row] = L == -INFINITY ? INFINITY : L * kLog2e;
     }
   }
 }
@@ -221,6 +225,7 @@ struct KVTile {
   int bkv;  // b * Hkv + kv head
   int kt;   // key block
   int i0;   // first query block
+  int nqb;  // query blocks per head
   int nb;   // blocks: group heads x query blocks
 };
 
@@ -235,8 +240,13 @@ __device__ __forceinline__ KVTile kv_tile(const BwdParams& p) {
     T.bkv = t / p.nkt;
     T.kt = t % p.nkt;
   }
-  T.i0 = p.causal ? T.kt : 0;  // causal: query q sees keys <= q (top-left aligned)
-  T.nb = T.i0 < p.nqt ? p.group * (p.nqt - T.i0) : 0;
+  // query blocks that see a key of this tile: q >= k0 - wr and q <= k0 + 127 + wl
+  // (causal: wr = 0, so from the diagonal block on; top-left aligned)
+  const int k0 = T.kt * kBN;
+  T.i0 = p.wr >= 0 ? max(0, k0 - p.wr) / kBM : 0;
+  const int i1 = p.wl >= 0 ? min(p.nqt - 1, (k0 + kBN - 1 + p.wl) / kBM) : p.nqt - 1;
+  T.nqb = i1 >= T.i0 ? i1 - T.i0 + 1 : 0;
+  T.nb = p.group * T.nqb;
   return T;
 }
 
@@ -296,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sbase + G::OFF_K + c * G::CHUNK, &tm_k, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
       tma_load_3d(sbase + G::OFF_V + c * G::CHUNK, &tm_v, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
     }
-    const int nqb = p.nqt - T.i0;
+    const int nqb = T.nqb;
     for (int m = 0; m < 2 * T.nb; ++m) {  // item m: Q (even, + lse2, delta) or dO (odd) of block m / 2
       const int sl = m % G::NSLOT, n = m >> 1;
       if (m >= G::NSLOT && !wait_bar(B(G::B_SLE + sl), ((m / G::NSLOT) - 1) & 1u, cx.abort_flag))
@@ -370,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2, r = (warp & 3) * 32 + lane;
     const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.c;
-    const int nqb = p.nqt - T.i0;
+    const int nqb = T.nqb;
     bool ok = true;
     for (int n = 0; ok && n < T.nb; ++n) {
       const int sl = (2 * n) % G::NSLOT;  // the slot of Q_n, with lse2 and delta
@@ -385,8 +395,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* dl = l2 + 128;
       uint32_t sr[64];
       tmem_ld_x64(tm + G::T_S + h * 64, sr);
-      // causal: only the diagonal block masks (key k0 + r > query q0 + col <=> r > col)
-      const bool diag = p.causal && i == T.kt;
+      // visible query columns of this key row: [lo_c, lo_c + span) -- key k0 + r
+      // is seen by query q0 + col iff k0 + r <= q0 + col + wr and k0 + r >= q0 + col - wl
+      const int dqk = kv_row0 + r - i * kBM;  // key minus query offset of column 0
+      const bool msk = (p.wr >= 0 && kv_row0 + kBN - 1 - p.wr > i * kBM) ||
+                       (p.wl >= 0 && kv_row0 + p.wl < i * kBM + kBM - 1);
+      const int lo_c = p.wr >= 0 ? dqk - p.wr : -kBM;
+      const int hi_c = p.wl >= 0 ? dqk + p.wl : 2 * kBM;
+      const uint32_t span = static_cast<uint32_t>(max(hi_c - lo_c + 1, 0));
       float pv[64];
 #pragma unroll
       for (int x = 0; x < 64; x += 4) {
@@ -395,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float e2 = ex2(fmaf(__uint_as_float(sr[x + e]), c, -lv[e]));
-          pv[x + e] = (diag && r > h * 64 + x + e) ? 0.f : e2;
+          pv[x + e] = (msk && static_cast<uint32_t>(h * 64 + x + e - lo_c) >= span) ? 0.f : e2;
         }
       }
       uint32_t pk[32];
@@ -530,7 +546,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = qt * kBM;
   const int kvz = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
   const int nkb = (p.Nk + kBN - 1) / kBN;
-  const int nb = p.causal ? min(nkb, (min(q0 + kBM, p.Nq) - 1) / kBN + 1) : nkb;
+  // key blocks this tile's rows see: keys q - wl .. q + wr (causal: wr = 0)
+  const int qlast = min(q0 + kBM, p.Nq) - 1;
+  const int jb0 = p.wl >= 0 ? min(max(0, q0 - p.wl) / kBN, nkb) : 0;
+  const int jb1 = p.wr >= 0 ? min(nkb - 1, (qlast + p.wr) / kBN) : nkb - 1;
+  const int nb = jb1 >= jb0 ? jb1 - jb0 + 1 : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(B(G::B_QF), 1);
@@ -556,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   cx.tmem = misc[0];
 
   if (warp >= 8) setmaxnreg_dec<88>();
-  if (warp == 9 && lane == 0) {
+  if (warp == 9 && lane == 0 && nb > 0) {
     // ---- TMA: Q and dO once, then (K_j, V_j) per key block
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -574,9 +594,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < G::DCH; ++c)
         tma_load_3d(sbase + G::OFF_SL + sl * G::T_BYTES + c * G::CHUNK, (m & 1) ? &tm_v : &tm_k,
-                    B(G::B_SLF + sl), c * 64, (m >> 1) * kBN, kvz, pol_last);
+                    B(G::B_SLF + sl), c * 64, (jb0 + (m >> 1)) * kBN, kvz, pol_last);
     }
-  } else if (warp == 8 && lane == 0) {
+  } else if (warp == 8 && lane == 0 && nb > 0) {
     // ---- MMA: S(0) dP(0) | S(j+1) dP(j+1) dQ(j) | ...
     constexpr uint32_t kIdNT = idesc_f16(128, 128, BF16, false);
     constexpr uint32_t kIdTN = idesc_f16(128, D, BF16, true);
@@ -640,9 +660,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(B(G::B_SFREE));
       // visible keys of this row in the block: [0, lim)
-      const int kbase = j * kBN + h * 64;
-      int lim = p.Nk - kbase;
-      if (p.causal) lim = min(lim, qpos - kbase + 1);
+      const int kbase = (jb0 + j) * kBN + h * 64;
+      int lim = p.Nk - kbase;  // keys [lo, lim) of this half block are visible to the row
+      if (p.wr >= 0) lim = min(lim, qpos + p.wr - kbase + 1);
+      const int lo = p.wl >= 0 ? qpos - p.wl - kbase : 0;
+      const uint32_t span = static_cast<uint32_t>(max(lim - lo, 0));
       uint32_t pk[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
@@ -651,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 2; ++e) {
           const int i = 2 * x + e;
           const float pe = ex2(fmaf(__uint_as_float(sr[i]), c, -lse2));
-          v2[e] = i < lim ? pe * (__uint_as_float(dr[i]) - dlt) : 0.f;
+          v2[e] = static_cast<uint32_t>(i - lo) < span ? pe * (__uint_as_float(dr[i]) - dlt) : 0.f;
         }
         pk[x] = pack2(v2[0], v2[1], BF16);
       }
@@ -667,6 +689,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(B(G::B_DSF));
     }
     // ---- epilogue: dQ = scale * acc, warpgroup h writes columns h * D/2 .. +D/2
+    if (nb == 0 && qpos < p.Nq) {  // no key seen by this tile's rows (key windows): dQ = 0
+      uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) + (static_cast<size_t>(bh) * p.Nq + qpos) * D;
+      for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 8)
+        *reinterpret_cast<uint4*>(dst + c0) = make_uint4(0, 0, 0, 0);
+    }
     if (ok && nb > 0) {
       ok = wait_bar(B(G::B_DQF), 0u, cx.abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
@@ -754,7 +781,8 @@ int nq_pad(int Nq) { return (Nq + 127) / 128 * 128; }
 template <int D, bool BF16>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
-               int Nk, float scale, int causal, cudaStream_t st, void* ws, int sms) {
+               int Nk, float scale, int causal, int wl, int wr, cudaStream_t st, void* ws,
+               int sms) {
   using GK = fab::GeoKV<D>;
   using GQ = fab::GeoQ<D>;
   static std::once_flag once;
@@ -786,6 +814,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.Nq_pad = nq_pad(Nq);
   p.group = Hq / Hkv;
   p.causal = causal ? 1 : 0;
+  p.wl = wl;
+  p.wr = causal ? 0 : wr;
   p.scale = scale;
   p.c = scale * fab::kLog2e;
   p.nqt = p.Nq_pad / 128;
@@ -822,11 +852,12 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Nq) {
   return 2ull * (size_t)B * Hq * nq_pad(Nq) * sizeof(float);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-           const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
-           int D, float scale, int causal, void* stream, int dtype, void* workspace,
-           size_t workspace_bytes) {
+int fa_bwd_window(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                  int Nk, int D, float scale, int causal, int window_left, int window_right,
+                  void* stream, int dtype, void* workspace, size_t workspace_bytes) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
+  if (window_left < -1 || window_right < -1 || (causal && window_right > 0)) return FA_ERR_BAD_WINDOW;
   if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_BAD_SHAPE;
   if (Hq % Hkv != 0) return FA_ERR_BAD_GROUPING;
@@ -861,10 +892,19 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
     return FA_ERR_NO_DEVICE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA_BF16;
-#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, st, workspace, sms
+#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, \
+                    window_right, st, workspace, sms
   if (D == 64) return bf ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
   return bf ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
 #undef FA_BWD_ARGS
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+           int D, float scale, int causal, void* stream, int dtype, void* workspace,
+           size_t workspace_bytes) {
+  return fa_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, D, scale, causal, -1,
+                       -1, stream, dtype, workspace, workspace_bytes);
 }
 
 // Status word of the backward kernels (read and optionally reset); used by
