@@ -144,3 +144,26 @@ def test_bwd_window_host_checks(lib):
                                  12 * A, 1 << 20)
     assert call(-2, 0) == fa.FA_ERR_BAD_WINDOW and call(3, -5) == fa.FA_ERR_BAD_WINDOW
     assert call(8, 2, causal=1) == fa.FA_ERR_BAD_WINDOW
+
+
+def test_python_binding_argument_checks(lib):
+    """The binding's own checks run before any CUDA call (argument marshalling only)."""
+    import torch
+    q = torch.zeros(1, 2, 16, 64, dtype=torch.float16)
+    k = torch.zeros(1, 2, 16, 64, dtype=torch.float16)
+    with pytest.raises(TypeError):
+        fa.fa_fwd(q.float(), k.float(), k.float())
+    with pytest.raises(TypeError):
+        fa.fa_fwd(q, k.bfloat16(), k)
+    with pytest.raises(ValueError):
+        fa.fa_fwd(q[0], k[0], k[0])  # not 4-D
+    with pytest.raises(ValueError):
+        fa.fa_fwd(q, k, k)  # CPU tensors
+    lse = torch.zeros(1, 2, 16)
+    with pytest.raises(ValueError):
+        fa.fa_bwd(q, k, k, q, lse, q)  # CPU tensors
+    with pytest.raises(TypeError):
+        fa.fa_bwd(q, k, k, q, lse.double(), q)  # lse must be float32
+    if not torch.cuda.is_available():
+        with pytest.raises(TypeError):
+            fa._bias_view(torch.zeros(1, 1, 16, 16, dtype=torch.float16), torch.float16, 1, 2, 16, 16)
