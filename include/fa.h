@@ -1,5 +1,6 @@
 /*
- * fa.h -- C ABI of the fused, tiled attention forward pass for NVIDIA B200 (sm_100a).
+ * fa.h -- C ABI of the fused, tiled attention for NVIDIA B200 (sm_100a): the
+ * forward pass (with key windows or an additive score bias) and its gradients.
  *
  * The operation (sources: "FlashAttention 算子" article on mooersco.com, sections
  * "标准 Attention 的瓶颈在哪" and "昇腾NPU上的分块策略"):
@@ -219,8 +220,8 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Nq);
  * interface that hands the library only its inputs and outputs -- there a
  * cudaMalloc would fail, or stall the device while the caller's stream is busy.
  * It takes exactly fa_fwd's arguments and allocates nothing (no cudaMalloc, no
- * cudaFree, no allocating library routine); the split-tail scratch is a
- * file-scope device array of fa_fwd_noalloc_scratch_bytes() bytes (24 MiB) that
+ * cudaFree, no allocating library routine); the scratch of the split tail and
+ * of stream-K decode launches is a file-scope device array of fa_fwd_noalloc_scratch_bytes() bytes (24 MiB) that
  * every GPU loading this library holds until the process exits.
  *   - The first call on each device looks up that array's device address
  *     (cudaGetSymbolAddress) with the device current; make that first call
@@ -229,7 +230,8 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Nq);
  *     kernel; all calls share the one array, so calls whose work overlaps on
  *     the GPU (other streams, other threads) race and must not be issued.
  *   - A problem whose split tail would need more scratch than the array holds
- *     returns FA_ERR_SCRATCH_TOO_SMALL and launches nothing.
+ *     returns FA_ERR_SCRATCH_TOO_SMALL and launches nothing (a stream-K launch
+ *     uses fewer CTAs instead, or none of the split).
  * Results equal fa_fwd_ws's for the same arguments.
  */
 int fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
