@@ -167,3 +167,29 @@ def test_python_binding_argument_checks(lib):
     if not torch.cuda.is_available():
         with pytest.raises(TypeError):
             fa._bias_view(torch.zeros(1, 1, 16, 16, dtype=torch.float16), torch.float16, 1, 2, 16, 16)
+
+
+def test_size_limits_are_rejected_on_the_host(lib):
+    # work-tile counts, row indices and TMA coordinates are 32-bit: sizes whose
+    # B * H * N reaches 2^31 are refused before anything is enqueued
+    assert _call(B=1 << 16, Hq=1 << 8, Hkv=1 << 8, Nq=1 << 8, Nk=64) == 3
+    assert _call(B=1 << 16, Hq=4, Hkv=2, Nq=64, Nk=1 << 15) == 3
+
+
+def test_bwd_host_checks(lib):
+    a = dict(GOOD)
+
+    def call(D=128, ws=12 * A, ws_bytes=1 << 20, dq=9 * A, dtype=a["dtype"], lse=8 * A):
+        return lib.fa_bwd(a["q"], a["k"], a["v"], 6 * A, 7 * A, lse, dq, 10 * A, 11 * A, a["B"],
+                          a["Hq"], a["Hkv"], a["Nq"], a["Nk"], D, ctypes.c_float(a["scale"]), 0,
+                          None, dtype, ws, ws_bytes)
+    assert call(D=256) == 5              # backward: head_dim 64 or 128
+    assert call(dtype=3) == 7
+    assert call(ws=None) == fa.FA_ERR_BAD_WORKSPACE
+    assert call(ws_bytes=16) == fa.FA_ERR_BAD_WORKSPACE
+    assert call(ws=12 * A + 128) == 2   # workspace not 256-byte aligned
+    assert call(lse=8 * A + 2) == 2
+    assert call(dq=1 * A) == 12          # dq overlaps q
+    assert call(lse=None) == 1
+    assert lib.fa_bwd_workspace_size(1, 4, 64) == 2 * 4 * 128 * 4
+    assert lib.fa_bwd_workspace_size(0, 4, 64) == 0
