@@ -108,9 +108,14 @@ def llama7b(causal: bool, peaky: bool = False) -> Workload:
                         + (" peaky" if peaky else ""))
 
 
-def seq_sweep(n: int, causal: bool) -> Workload:
-    seed = {512: 1, 2048: 2, 4096: 3, 8192: 4}[n]
-    return Workload(f"sweep B1 H32 N{n} D128 fp16 {'causal' if causal else 'noncausal'}",
+SWEEP_SEEDS = (1, 2, 3, 4)
+
+
+def seq_sweep(n: int, causal: bool, seed: Optional[int] = None) -> Workload:
+    """Sequence sweep workload; the default seed is the k-th of 1-4 for the k-th length."""
+    if seed is None:
+        seed = {512: 1, 2048: 2, 4096: 3, 8192: 4}[n]
+    return Workload(f"sweep B1 H32 N{n} D128 fp16 {'causal' if causal else 'noncausal'} seed{seed}",
                     1, 32, 32, n, n, 128, "fp16", causal, seed)
 
 

@@ -223,16 +223,21 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Nq);
  * cudaFree, no allocating library routine); the scratch of the split tail and
  * of stream-K decode launches is a file-scope device array of fa_fwd_noalloc_scratch_bytes() bytes (24 MiB) that
  * every GPU loading this library holds until the process exits.
+ *   - Argument errors are returned before any CUDA call, as for fa_fwd.
  *   - The first call on each device looks up that array's device address
  *     (cudaGetSymbolAddress) with the device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  If the lookup fails the call returns
+ *     FA_ERR_LAUNCH and launches nothing; the next call tries again.
  *   - Each call clears the array's arrival counters on `stream` before its
  *     kernel; all calls share the one array, so calls whose work overlaps on
  *     the GPU (other streams, other threads) race and must not be issued.
  *   - A problem whose split tail would need more scratch than the array holds
  *     returns FA_ERR_SCRATCH_TOO_SMALL and launches nothing (a stream-K launch
  *     uses fewer CTAs instead, or none of the split).
- * Results equal fa_fwd_ws's for the same arguments.
+ * Results are bit-identical to fa_fwd_ws's with a workspace of
+ * fa_fwd_workspace_size(D) bytes (the same split and the same fixed merge
+ * order), except for a stream-K launch that one of the two scratch sizes cuts
+ * to fewer CTAs than the other: those agree within rounding.
  */
 int fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream,

@@ -99,6 +99,19 @@ def test_workspace_entry_point_host_checks(lib):
     assert fa.set_max_ctas(0) == 0
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=2), 7), (dict(D=96), 5), (dict(B=0), 3), (dict(Hq=6, Hkv=4), 4),
+    (dict(scale=float("nan")), 6), (dict(q=0), 1), (dict(k=2 * A + 8), 2), (dict(o=1 * A + 64), 12),
+])
+def test_noalloc_entry_point_host_checks(lib, kw, code):
+    """fa_fwd_noalloc rejects bad arguments on the host, before its scratch lookup."""
+    a = dict(GOOD)
+    a.update(kw)
+    assert lib.fa_fwd_noalloc(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                              a["Nq"], a["Nk"], a["D"], ctypes.c_float(a["scale"]), a["causal"],
+                              None, a["dtype"]) == code
+
+
 def test_window_entry_point_host_checks(lib):
     import torch
     a = dict(GOOD)

@@ -1,6 +1,6 @@
 """The FMA-pipe exp2 the softmax uses for part of its exponentials.
 
-CPU: the coefficients in sm100_ptx.cuh are the Remez fit that
+CPU: the coefficients in sm100_ptx.cuh are the linear-programming minimax fit that
 fit_exp2_poly.py produces, and their float32 Horner evaluation meets the
 stated 1.02e-4 relative-error bound against 2^f computed in float64.
 GPU: the kernel-side evaluation (range reduction + polynomial + exponent add)

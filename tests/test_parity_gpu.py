@@ -1,9 +1,11 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
-Small and ragged shapes are compared on every output element; the workloads
-the pages measure on (LLaMA-7B layer, sequence sweep, GQA/MQA and head-dim
-sweep, 128K context) are compared on seeded samples of query rows (every head,
-rows 0 and N-1 always included), plus properties that hold at any size.
+Small and ragged shapes, the LLaMA-7B layer (all four variants) and the
+sequence sweep up to N=4096 (all four seeds) are compared on every output
+element.  The largest workloads -- the sweep at N=8192, the GQA/MQA and
+head-dim sweep at N=8192 and the 128K context -- are compared on seeded
+samples of query rows (every head, rows 0 and N-1 always included), plus
+properties that hold at any size.
 
 Tolerances (max abs difference against the fp64 oracle): fp16 inputs O 4e-3
 and LSE 1e-3; bf16 inputs O 1.6e-2 and LSE 1e-3.
@@ -18,7 +20,8 @@ import torch
 
 import oracle
 import tiled_attention_15_b200 as fa
-from fa_inputs import TINY, LONG, Workload, gqa, llama7b, make_qkv, sample_rows, seq_sweep
+from fa_inputs import (SWEEP_SEEDS, TINY, LONG, Workload, gqa, llama7b, make_qkv, sample_rows,
+                       seq_sweep)
 
 pytestmark = pytest.mark.gpu
 
@@ -243,9 +246,10 @@ def test_side_stream(cuda_dev):
     assert torch.equal(o, ref)
 
 
-# ------------------------------------------------------------ full-size workloads (sampled rows)
+# ------------------------------------------------------------ full-size workloads
 def _full(w, n_rows, cuda_dev):
-    rows = sample_rows(w.Nq, n_rows, w.seed)
+    """Every element when n_rows is None, else a seeded sample of n_rows query rows per head."""
+    rows = None if n_rows is None else sample_rows(w.Nq, n_rows, w.seed)
     o, lse, (q, k, v), do, dl = compare(w, cuda_dev, rows=rows)
     # properties at every row: O is a convex combination of V rows, LSE is finite
     vmax = v.float().abs().amax(dim=(2, 3)).to(cuda_dev)
@@ -259,13 +263,14 @@ def _full(w, n_rows, cuda_dev):
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("peaky", [False, True])
 def test_llama7b_layer(cuda_dev, causal, peaky):
-    _full(llama7b(causal, peaky), 64, cuda_dev)
+    _full(llama7b(causal, peaky), None, cuda_dev)
 
 
+@pytest.mark.parametrize("seed", SWEEP_SEEDS)
 @pytest.mark.parametrize("n", [512, 2048, 4096, 8192])
 @pytest.mark.parametrize("causal", [False, True])
-def test_sequence_sweep(cuda_dev, n, causal):
-    _full(seq_sweep(n, causal), 48, cuda_dev)
+def test_sequence_sweep(cuda_dev, n, causal, seed):
+    _full(seq_sweep(n, causal, seed), None if n <= 4096 else 48, cuda_dev)
 
 
 @pytest.mark.parametrize("hkv,d", [(8, 128), (1, 128), (8, 64), (8, 256)])

@@ -7,7 +7,9 @@ nothing and keeps the split tail's scratch in a file-scope device array.
 
 Each case calls it through the C ABI twice in a row and checks both results
 against the existing workspace entry point (fa_fwd_ws with a caller-allocated
-workspace), within the parity tolerances of the other GPU tests.  The cases
+workspace of fa_fwd_workspace_size bytes): within the parity tolerances of the
+other GPU tests, and in fact bit for bit, since both take the same split and
+merge in the same fixed order.  The cases
 include shapes whose last round of tiles is split and a decode shape split
 stream-K (so the static scratch is really used), and a causal one (no split).  The file name makes pytest collect
 it last, so a failure here leaves every other test already run.
@@ -68,5 +70,6 @@ def test_noalloc_matches_workspace_entry_point(cuda_dev, w, cap):
             assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
             assert (o.float() - o_ref.float()).abs().max().item() <= TOL[w.dtype], call
             assert (lse - l_ref).abs().max().item() <= 1e-3, call
+            assert torch.equal(o, o_ref) and torch.equal(lse, l_ref), call
     finally:
         fa.set_max_ctas(prev)

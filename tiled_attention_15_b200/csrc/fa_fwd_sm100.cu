@@ -1450,11 +1450,10 @@ long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D) {
   return (long long)B * Hq * ((Nq + rows - 1) / rows);
 }
 
-static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                    int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype,
-                    void* ws, size_t ws_bytes, Scratch mode = Scratch::kCaller, int wl = -1,
-                    int wr = -1, const BiasArg* bias = nullptr) {
-  // ---- argument checks: host only, before any CUDA call
+// Argument checks of every forward entry point: host only, before any CUDA call.
+static int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
+                          int dtype, int wl, int wr) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
   if (wl < -1 || wr < -1 || (causal && wr > 0)) return FA_ERR_BAD_WINDOW;
   if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;
@@ -1477,6 +1476,15 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
         overlaps(lse, lb, o, qo_b))
       return FA_ERR_OVERLAP;
   }
+  return FA_OK;
+}
+
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                    int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream, int dtype,
+                    void* ws, size_t ws_bytes, Scratch mode = Scratch::kCaller, int wl = -1,
+                    int wr = -1, const BiasArg* bias = nullptr) {
+  const int bad = check_fwd_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, dtype, wl, wr);
+  if (bad != FA_OK) return bad;
   // ---- device
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_NO_DEVICE;
@@ -1590,26 +1598,38 @@ int fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, 
 // scratch of the split tail lives in this file-scope device array, which every
 // GPU that loads the library holds until the process exits.  In host code the
 // array's name is only a host-side stand-in, so its device address is fetched
-// with cudaGetSymbolAddress once per device, on that device's first call.
+// with cudaGetSymbolAddress, with the device current, by the first call on each
+// device (and kept once that lookup has succeeded).
 constexpr size_t kNoAllocScratchBytes = size_t(24) << 20;  // 24 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-struct NoAllocDevice {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaErrorUnknown;
-};
-NoAllocDevice g_noalloc[kMaxDevices];
+// Device address of the array, per device; kept only once a lookup succeeded,
+// so a lookup that failed (for example inside a stream capture) is retried on
+// the next call.
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
 
 int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int D, float scale, int causal, void* stream,
                    int dtype) {
+  const int bad = check_fwd_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, dtype, -1, -1);
+  if (bad != FA_OK) return bad;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_NO_DEVICE;
-  NoAllocDevice& nd = g_noalloc[dev];
-  std::call_once(nd.once, [&] { nd.err = cudaGetSymbolAddress(&nd.ptr, g_noalloc_scratch); });
-  if (nd.err != cudaSuccess || nd.ptr == nullptr) return FA_ERR_NO_DEVICE;
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, nd.ptr,
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+        cudaGetLastError();  // the failed lookup leaves no sticky error behind
+        return FA_ERR_LAUNCH;
+      }
+      g_noalloc_ptr[dev] = ptr;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, scratch,
                   kNoAllocScratchBytes, Scratch::kStatic);
 }
 
