@@ -7,7 +7,11 @@ attention-layer workload (B=2, Hq=Hkv=32, N=2048, D=128, fp16,
 scale=1/sqrt(128)): the non-causal forward pass and the causal forward pass,
 both through the library's C ABI.  Inputs are synthetic (seeded N(0,1),
 rounded to fp16) and resident in HBM when timing starts; L2 is flushed
-(256 MiB write) between steps because the inputs (~100 MB) fit in L2.
+(256 MiB write, outside the timed events) before every pass because the
+inputs (~100 MB) fit in L2.  Beside the step, every other workload of the
+pages is timed on its own (the tiny check, the sequence sweep, the GQA/MQA and
+head-dim sweep, the 128K context) together with KV-cache decode, key windows,
+a score bias and the backward pass.
 
 metric: attention forward TFLOP/s with FLOPs = 4*B*Hq*Nq*Nk*D (halved for the
 causal pass).  Prints one JSON line on rank 0.  For N > 1 (torchrun) every rank
@@ -36,6 +40,7 @@ if ROOT not in sys.path:
 METRIC = "attn fwd TFLOP/s (4·B·Hq·Nq·Nk·D, ½ if causal) and % of B200 dense FP16 peak"
 SPEC_PEAK_TFLOPS = 2250.0
 FALLBACK_PEAK_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -46,7 +51,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-gate", action="store_true", help="skip the N=4096/8192 gate configs")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload lines (tiny, sweep, GQA/head-dim, 128K)")
     ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurement")
     ap.add_argument("--no-window", action="store_true",
                     help="skip the sliding-window measurement")
@@ -75,6 +81,14 @@ def aggregate_tflops(flops_per_step: float, steps: int, max_ms: float, world: in
 def workloads():
     from fa_inputs import llama7b
     return [llama7b(False), llama7b(True)]
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"])
+    return FALLBACK_HBM_GBS
 
 
 def peaks():
@@ -151,7 +165,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:  # noqa: BLE001
                 pass
-            time.sleep(0.005)
+            time.sleep(0.001)
 
     def __enter__(self):
         if self.ok:
@@ -225,6 +239,50 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------------------- CUDA arm
+def device_qkv(w, dev, seed):
+    """Seeded N(0,1) inputs drawn on the device (the large sweep workloads; same recipe
+    as fa_inputs.make_qkv, including the outlier keys, but torch's generator)."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(seed)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    q = torch.randn((w.B, w.Hq, w.Nq, w.D), device=dev, generator=g) * w.q_mult
+    k = torch.randn((w.B, w.Hkv, w.Nk, w.D), device=dev, generator=g)
+    v = torch.randn((w.B, w.Hkv, w.Nk, w.D), device=dev, generator=g)
+    if w.outlier_frac > 0.0:
+        n_out = int(w.outlier_frac * w.Nk)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                rows = torch.randperm(w.Nk, device=dev, generator=g)[:n_out]
+                k[b, h, rows] *= w.outlier_mult
+    return q.to(dt), k.to(dt), v.to(dt)
+
+
+def time_launches(fn, flush, stream, n=10, warm=3):
+    """Median CUDA-event time (ms) of fn() over n launches, L2 flushed before each."""
+    import torch
+    for _ in range(warm):
+        flush.zero_()
+        fn()
+    ts = []
+    for _ in range(n):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def workload_line(w, ms, peak, hbm, flops=None):
+    flops = w.flops() if flops is None else flops
+    tf = flops / (ms * 1e-3) / 1e12
+    gbs = w.io_bytes() / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 3),
+            "alg_bytes": w.io_bytes(), "alg_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm, 3)}
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -250,6 +308,8 @@ def main():
         if world > 1:
             dist.barrier()
 
+    peak, peak_sus, peak_kind = peaks()
+    hbm = hbm_peak()
     ws = workloads()
     inputs = []
     for w in ws:
@@ -263,95 +323,145 @@ def main():
     stream = torch.cuda.current_stream(dev)
     sptr = stream.cuda_stream
 
-    def step():
-        for w, (o, lse) in zip(ws, outs):
-            fa.fa_fwd(q, k, v, o=o, lse=lse, scale=w.softmax_scale, causal=w.causal, stream=sptr)
+    def run_pass(j, qq=None, kk=None, vv=None, st=None):
+        w, (o, lse) = ws[j], outs[j]
+        fa.fa_fwd(q if qq is None else qq, k if kk is None else kk, v if vv is None else vv,
+                  o=o, lse=lse, scale=w.softmax_scale, causal=w.causal,
+                  stream=sptr if st is None else st)
 
     for _ in range(args.warmup):
-        flush.zero_()
-        step()
+        for j in range(len(ws)):
+            flush.zero_()
+            run_pass(j)
     torch.cuda.synchronize()
     assert fa.device_status(reset=True) == 0
 
+    # ---- the timed step: each pass bracketed by its own events, L2 flushed before it
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ws) + 1)] for _ in range(K)]
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in ws] for _ in range(K)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         for i in range(K):
-            flush.zero_()
-            e = ev[i]
-            e[0].record(stream)
-            for j, (w, (o, lse)) in enumerate(zip(ws, outs)):
-                fa.fa_fwd(q, k, v, o=o, lse=lse, scale=w.softmax_scale, causal=w.causal,
-                          stream=sptr)
-                e[j + 1].record(stream)
+            for j in range(len(ws)):
+                flush.zero_()
+                ev[i][j][0].record(stream)
+                run_pass(j)
+                ev[i][j][1].record(stream)
         torch.cuda.synchronize()
     barrier()
-    per_launch = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)] for j in range(len(ws))]
-    step_ms = [sum(per_launch[j][i] for j in range(len(ws))) for i in range(K)]
-    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    per_pass = [[ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(K)] for j in range(len(ws))]
+    total_ms = max_over_ranks(sum(sum(x) for x in per_pass), world, dev)
     assert fa.device_status(reset=True) == 0
     flops_step = sum(w.flops() for w in ws)
     value = aggregate_tflops(flops_step, K, total_ms, world)
+    pass_lines = {("causal" if w.causal else "non-causal"):
+                  {"median_ms": round(statistics.median(per_pass[j]), 5),
+                   "tflops": round(w.flops() / (statistics.median(per_pass[j]) * 1e-3) / 1e12, 1),
+                   "l2": "flushed before the pass"}
+                  for j, w in enumerate(ws)}
 
-    # ---- end to end: pinned host inputs -> device -> both passes -> O and LSE back to host
+    # ---- end to end through the public API: pinned host inputs -> device -> both
+    # passes -> O and LSE back to pinned host memory, every step.  Copies in and
+    # out run on their own streams with two device buffer sets, so the upload of
+    # step i + 1 and the download of step i - 1 overlap the passes of step i.
     hq, hk, hv = (x.pin_memory() for x in inputs[0][1:])
-    ho = [(torch.empty(q.shape, dtype=q.dtype, pin_memory=True),
-           torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)) for _ in ws]
+    ho = [[(torch.empty(q.shape, dtype=q.dtype, pin_memory=True),
+            torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)) for _ in ws]
+          for _ in range(2)]
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
-    d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in ho)
-    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in ho[0])
+    dbuf = [tuple(torch.empty_like(x) for x in (q, k, v)) for _ in range(2)]
+    dout = [[(torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev))
+             for _ in ws] for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     E = max(10, K // 20)
 
-    def e2e_step():
-        qd.copy_(hq, non_blocking=True)
-        kd.copy_(hk, non_blocking=True)
-        vd.copy_(hv, non_blocking=True)
-        for w, (o, lse), (h_o, h_l) in zip(ws, outs, ho):
-            fa.fa_fwd(qd, kd, vd, o=o, lse=lse, scale=w.softmax_scale, causal=w.causal, stream=sptr)
-            h_o.copy_(o, non_blocking=True)
-            h_l.copy_(lse, non_blocking=True)
+    def e2e_run(n):
+        done_in = [None, None]   # compute of the step that last read buffer b is done
+        done_out = [None, None]  # download of the step that last wrote output set b is done
+        for i in range(n):
+            b = i & 1
+            if done_in[b] is not None:
+                s_in.wait_event(done_in[b])
+            with torch.cuda.stream(s_in):
+                for dst, src in zip(dbuf[b], (hq, hk, hv)):
+                    dst.copy_(src, non_blocking=True)
+            up = torch.cuda.Event()
+            up.record(s_in)
+            stream.wait_event(up)
+            if done_out[b] is not None:
+                stream.wait_event(done_out[b])
+            for j, w in enumerate(ws):
+                o, lse = dout[b][j]
+                fa.fa_fwd(*dbuf[b], o=o, lse=lse, scale=w.softmax_scale, causal=w.causal,
+                          stream=sptr)
+            comp = torch.cuda.Event()
+            comp.record(stream)
+            done_in[b] = comp
+            s_out.wait_event(comp)
+            with torch.cuda.stream(s_out):
+                for (o, lse), (h_o, h_l) in zip(dout[b], ho[b]):
+                    h_o.copy_(o, non_blocking=True)
+                    h_l.copy_(lse, non_blocking=True)
+            down = torch.cuda.Event()
+            down.record(s_out)
+            done_out[b] = down
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
 
-    for _ in range(3):
-        e2e_step()
+    e2e_run(3)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(E):
-        e2e_step()
+    s_in.wait_stream(stream)
+    e2e_run(E)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = aggregate_tflops(flops_step, E, e2e_ms, world)
+    assert fa.device_status(reset=True) == 0
+    del dbuf, dout
 
-    # ---- gate configs (N = 4096 / 8192, D = 128), a few launches each, L2 flushed
-    gate = {}
-    if not args.no_gate:
-        from fa_inputs import seq_sweep
-        for n in (4096, 8192):
-            w0 = seq_sweep(n, False)
-            gq, gk, gv = (x.to(dev) for x in make_qkv(w0))
-            go, gl = torch.empty_like(gq), torch.empty(gq.shape[:3], dtype=torch.float32, device=dev)
+    # ---- every other workload the pages measure on, one line each (10 launches,
+    # L2 flushed before each; the median)
+    from fa_inputs import TINY, LONG, gqa, seq_sweep
+    configs = {}
+    if not args.no_configs:
+        cases = [("tiny B1 H1 N256 D64 fp16", TINY, None)]
+        for n in (512, 2048, 4096, 8192):
             for causal in (False, True):
-                w = seq_sweep(n, causal)
-                ts = []
-                for i in range(13):
-                    flush.zero_()
-                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    a.record(stream)
-                    fa.fa_fwd(gq, gk, gv, o=go, lse=gl, scale=w.softmax_scale, causal=causal,
-                              stream=sptr)
-                    b.record(stream)
-                    torch.cuda.synchronize()
-                    if i >= 3:
-                        ts.append(a.elapsed_time(b))
-                ms = statistics.median(ts)
-                gate[f"N{n}_{'causal' if causal else 'noncausal'}"] = {
-                    "ms": round(ms, 4), "tflops": round(w.flops() / (ms * 1e-3) / 1e12, 1)}
-            del gq, gk, gv, go, gl
+                cases.append((f"sweep B1 H32 N{n} D128 fp16 {'causal' if causal else 'non-causal'}",
+                              seq_sweep(n, causal), None))
+        for hkv, d in ((8, 128), (1, 128), (8, 64), (8, 256)):
+            cases.append((f"gqa B4 Hq32 Hkv{hkv} N8192 D{d} bf16 causal", gqa(hkv, d), 11))
+        cases.append(("long B1 Hq32 Hkv8 N131072 D128 bf16 causal, 1% outlier keys", LONG, 12))
+        for name, w, dseed in cases:
+            if dseed is None:
+                cq, ck, cv = (x.to(dev) for x in make_qkv(w))
+            else:
+                cq, ck, cv = device_qkv(w, dev, dseed)
+            co = torch.empty_like(cq)
+            cl = torch.empty(cq.shape[:3], dtype=torch.float32, device=dev)
+            n_launch = 3 if w.Nq > 65536 else 10
+            ms = time_launches(lambda: fa.fa_fwd(cq, ck, cv, o=co, lse=cl, scale=w.softmax_scale,
+                                                 causal=w.causal, stream=sptr),
+                               flush, stream, n=n_launch, warm=2)
+            configs[name] = workload_line(w, ms, peak, hbm)
+            del cq, ck, cv, co, cl
+        configs["note"] = ("ms: median CUDA-event time of one launch, L2 flushed before each; "
+                           "alg_gbs: algorithmic bytes (read Q, K, V once, write O and LSE once) "
+                           "per second, frac_of_hbm against the measured copy bandwidth")
         assert fa.device_status(reset=True) == 0
+    gate = {}
+    for n in (4096, 8192):
+        for cz in ("non-causal", "causal"):
+            c = configs.get(f"sweep B1 H32 N{n} D128 fp16 {cz}")
+            if c:
+                gate[f"N{n}_{cz.replace('-', '')}"] = {"ms": c["ms"], "tflops": c["tflops"],
+                                                       "frac_of_peak": c["frac_of_peak"]}
 
     # ---- backward pass on the bench workload (LLaMA-7B layer), both passes
     backward = {}
@@ -363,22 +473,13 @@ def main():
         bdq, bdk, bdv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         for w in ws:
             bo, bl = fa.fa_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal, stream=sptr)
-            ts = []
-            for i in range(13):
-                flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fa.fa_bwd(q, k, v, bo, bl, bdo, scale=w.softmax_scale, causal=w.causal, dq=bdq,
-                          dk=bdk, dv=bdv, stream=sptr, workspace=bws)
-                b.record(stream)
-                torch.cuda.synchronize()
-                if i >= 3:
-                    ts.append(a.elapsed_time(b))
-            ms = statistics.median(ts)
+            ms = time_launches(lambda: fa.fa_bwd(q, k, v, bo, bl, bdo, scale=w.softmax_scale,
+                                                 causal=w.causal, dq=bdq, dk=bdk, dv=bdv,
+                                                 stream=sptr, workspace=bws), flush, stream)
             bflops = 2.5 * w.flops()  # five GEMMs against the forward pass's two
             backward["causal" if w.causal else "noncausal"] = {
                 "ms": round(ms, 4), "tflops": round(bflops / (ms * 1e-3) / 1e12, 1),
-                "frac_of_peak": round(bflops / (ms * 1e-3) / 1e12 / peaks()[0], 3)}
+                "frac_of_peak": round(bflops / (ms * 1e-3) / 1e12 / peak, 3)}
         backward["flops"] = "2.5 x the forward pass's (five GEMMs); three launches per call"
         del bdo, bws, bdq, bdk, bdv
         assert fa.device_status(reset=True) == 0
@@ -390,20 +491,10 @@ def main():
         g1 = torch.Generator(device=dev).manual_seed(2)
         bb = torch.randn((1, 1, w.Nq, w.Nk), device=dev, dtype=q.dtype, generator=g1)
         bo, bl = torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-        ts = []
-        for i in range(13):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fa.fa_fwd(q, k, v, o=bo, lse=bl, scale=w.softmax_scale, bias=bb, stream=sptr)
-            b.record(stream)
-            torch.cuda.synchronize()
-            if i >= 3:
-                ts.append(a.elapsed_time(b))
-        ms = statistics.median(ts)
+        ms = time_launches(lambda: fa.fa_fwd(q, k, v, o=bo, lse=bl, scale=w.softmax_scale, bias=bb,
+                                             stream=sptr), flush, stream)
         bias_line = {"workload": "LLaMA-7B layer non-causal + shared [N, N] fp16 bias",
-                     "ms": round(ms, 4), "tflops": round(w.flops() / (ms * 1e-3) / 1e12, 1),
-                     "frac_of_peak": round(w.flops() / (ms * 1e-3) / 1e12 / peaks()[0], 3)}
+                     **workload_line(w, ms, peak, hbm)}
         del bb, bo, bl
         assert fa.device_status(reset=True) == 0
 
@@ -416,61 +507,52 @@ def main():
         W = 1024
         wq, wk, wv = (x.to(dev) for x in make_qkv(ww))
         wo, wl_ = torch.empty_like(wq), torch.empty(wq.shape[:3], dtype=torch.float32, device=dev)
-        ts = []
-        for i in range(13):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fa.fa_fwd(wq, wk, wv, o=wo, lse=wl_, scale=ww.softmax_scale, causal=True,
-                      window=(W - 1, -1), stream=sptr)
-            b.record(stream)
-            torch.cuda.synchronize()
-            if i >= 3:
-                ts.append(a.elapsed_time(b))
-        ms = statistics.median(ts)
+        ms = time_launches(lambda: fa.fa_fwd(wq, wk, wv, o=wo, lse=wl_, scale=ww.softmax_scale,
+                                             causal=True, window=(W - 1, -1), stream=sptr),
+                           flush, stream)
         # visible (query, key) pairs per head: query i sees min(i + 1, W) keys
         pairs = W * (W + 1) // 2 + (ww.Nq - W) * W
         wflops = 4 * ww.B * ww.Hq * ww.D * pairs
-        window = {"workload": ww.name, "ms": round(ms, 4), "visible_pairs_per_head": pairs,
-                  "tflops": round(wflops / (ms * 1e-3) / 1e12, 1),
-                  "frac_of_peak": round(wflops / (ms * 1e-3) / 1e12 / peaks()[0], 3)}
+        window = {"workload": ww.name, "visible_pairs_per_head": pairs,
+                  **workload_line(ww, ms, peak, hbm, flops=wflops)}
         del wq, wk, wv, wo, wl_
         assert fa.device_status(reset=True) == 0
 
-    # ---- KV-cache decode (one query row per head, 32K-token cache, GQA 4): HBM-bound
+    # ---- KV-cache decode (one query row per head, long cache, GQA 4): HBM-bound
     decode = {}
     if not args.no_decode:
         from fa_inputs import Workload
-        wd = Workload("decode B8 Hq32 Hkv8 Nq1 Nk32768 D128 fp16", 8, 32, 8, 1, 32768, 128, "fp16",
-                      False, seed=0)
-        dq, dk, dv = (x.to(dev) for x in make_qkv(wd))
-        do_, dl_ = torch.empty_like(dq), torch.empty(dq.shape[:3], dtype=torch.float32, device=dev)
-        # The K/V cache (1.07 GB) is 8x the L2, so launches run back to back (no
-        # flush): a serving loop's view, with no host time between launches.
-        for _ in range(3):
-            fa.fa_fwd(dq, dk, dv, o=do_, lse=dl_, scale=wd.softmax_scale, stream=sptr)
-        ts = []
-        for i in range(5):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(10):
+        for wd in (Workload("decode B8 Hq32 Hkv8 Nq1 Nk32768 D128 fp16", 8, 32, 8, 1, 32768, 128,
+                            "fp16", False, seed=0),
+                   Workload("decode B1 Hq32 Hkv8 Nq1 Nk131072 D128 fp16", 1, 32, 8, 1, 131072,
+                            128, "fp16", False, seed=0)):
+            dq, dk, dv = (x.to(dev) for x in make_qkv(wd))
+            do_, dl_ = torch.empty_like(dq), torch.empty(dq.shape[:3], dtype=torch.float32,
+                                                         device=dev)
+            # The K/V cache (>= 268 MB) is larger than L2, so launches run back to
+            # back (no flush): a serving loop's view, with no host time between launches.
+            for _ in range(3):
                 fa.fa_fwd(dq, dk, dv, o=do_, lse=dl_, scale=wd.softmax_scale, stream=sptr)
-            b.record(stream)
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b) / 10)
-        ms = statistics.median(ts)
-        nbytes = wd.io_bytes()
-        hbm = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"] \
-            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 6650.0
-        decode = {"workload": wd.name, "ms": round(ms, 4), "bytes": nbytes,
-                  "l2": "inputs larger than L2 (1.07 GB K/V), 10 launches back to back per event pair",
-                  "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
-                  "frac_of_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 3),
-                  "tflops": round(wd.flops() / (ms * 1e-3) / 1e12, 2)}
-        del dq, dk, dv, do_, dl_
+            ts = []
+            for i in range(5):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(10):
+                    fa.fa_fwd(dq, dk, dv, o=do_, lse=dl_, scale=wd.softmax_scale, stream=sptr)
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b) / 10)
+            ms = statistics.median(ts)
+            nbytes = wd.io_bytes()
+            decode[wd.name] = {
+                "ms": round(ms, 4), "bytes": nbytes,
+                "l2": "K/V larger than L2, 10 launches back to back per event pair",
+                "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                "frac_of_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 3),
+                "tflops": round(wd.flops() / (ms * 1e-3) / 1e12, 2)}
+            del dq, dk, dv, do_, dl_
         assert fa.device_status(reset=True) == 0
 
-    peak, peak_sus, peak_kind = peaks()
     launch_ms = total_ms / world / (K * len(ws)) if world > 1 else total_ms / (K * len(ws))
     achieved = (flops_step / len(ws)) / (launch_ms * 1e-3) / 1e12
     traffic = recorded_traffic()
@@ -482,7 +564,8 @@ def main():
         "config": {"workload": "llama7b-attn B2 Hq32 Hkv32 N2048 D128 fp16, non-causal + causal",
                    "B": 2, "Hq": 32, "Hkv": 32, "N": 2048, "D": 128,
                    "passes_per_step": ["non-causal", "causal"],
-                   "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+                   "l2": "flushed before every pass (256 MiB write, outside the timed events)"},
+        "per_pass": pass_lines,
         "pct_of_peak": {"measured_burst": round(100 * value / world / peak, 1),
                         "measured_sustained": round(100 * value / world / peak_sus, 1),
                         "spec_2250": round(100 * value / world / SPEC_PEAK_TFLOPS, 1),
@@ -493,9 +576,12 @@ def main():
                      "kernel": "fa::fa_fwd_kernel<128, 2, false> (fp16, D=128)",
                      "peak_note": f"{peak_kind} bf16 dense burst (fp16:bf16 nominal ratio 1:1)"},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "note": "copies on their own streams, double-buffered: uploads and downloads "
+                        "overlap the passes of the neighbouring steps"},
         "gpu_launches": K * len(ws),
         "clocks": clk.summary(),
+        "configs": configs,
         "gate_d128": gate,
         "decode": decode,
         "window": window,

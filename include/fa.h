@@ -74,7 +74,8 @@ enum fa_status {
   FA_ERR_OVERLAP = 12,             /* o or lse overlaps q, k or v                  */
   FA_ERR_SCRATCH_TOO_SMALL = 13,   /* fa_fwd_noalloc: static scratch too small     */
   FA_ERR_BAD_WINDOW = 14,          /* fa_fwd_window: bound < -1, or causal + right > 0 */
-  FA_ERR_BAD_WORKSPACE = 15        /* fa_bwd: workspace NULL or too small          */
+  FA_ERR_BAD_WORKSPACE = 15,       /* fa_bwd, fa_fwd_unfused: workspace NULL, too small or misaligned */
+  FA_ERR_LIBRARY = 16              /* fa_fwd_unfused: a cuBLAS call failed          */
 };
 
 /*
@@ -245,6 +246,33 @@ int fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *
 
 /* Size in bytes of fa_fwd_noalloc's static scratch array. */
 size_t fa_fwd_noalloc_scratch_bytes(void);
+
+/*
+ * Standard attention in three steps through device memory -- the comparison
+ * the pages make (mooersco.com article, "标准 Attention 的瓶颈在哪" and the table of
+ * "跟标准 Attention 的性能差距有多大"; gitcode.csdn.net article, section 二): S =
+ * scale Q K^T is written out (fp32), a row-softmax kernel reads it and writes P
+ * (rounded to the input dtype) and the LSE, and O = P V reads P back.  The two
+ * products are cuBLAS batched GEMMs with fp32 accumulation; the softmax is this
+ * library's kernel.  It exists to measure what the fused kernel saves (time,
+ * device memory, DRAM traffic); it is not the fast path.
+ *   Arguments, layout, causal, scale and LSE as fa_fwd; D in {64, 128, 256}.
+ *   workspace  device buffer of at least fa_fwd_unfused_workspace_size(B, Hq, Nq, Nk)
+ *              bytes, 256-byte aligned, caller-owned (holds S and P: 6 bytes per
+ *              score); FA_ERR_BAD_WORKSPACE otherwise.
+ *   Errors     as fa_fwd, plus FA_ERR_LIBRARY if creating the cuBLAS handle (once
+ *              per device, on the first call; it allocates cuBLAS's own device
+ *              memory) or a cuBLAS call fails.
+ *   Results agree with fa_fwd's within the rounding of P (both round P to the
+ *   input dtype, at different points).
+ */
+int fa_fwd_unfused(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int D, float scale, int causal, void *stream,
+                   int dtype, void *workspace, size_t workspace_bytes);
+
+/* Workspace bytes fa_fwd_unfused needs: 256-aligned 4 + 2 bytes per score (B * Hq * Nq * Nk);
+ * 0 for bad sizes. */
+size_t fa_fwd_unfused_workspace_size(int B, int Hq, int Nq, int Nk);
 
 /* Process-wide cap on the CTAs (one per SM) a launch uses; 0, the default, means
  * every SM.  Useful to leave SMs to concurrent work.  Returns the previous cap,

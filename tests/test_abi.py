@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 16):
+    for code in range(0, 17):
         s = fa.status_string(code)
         assert s and s != "unknown status", code
     assert fa.status_string(99) == "unknown status"
@@ -110,6 +110,30 @@ def test_noalloc_entry_point_host_checks(lib, kw, code):
     assert lib.fa_fwd_noalloc(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
                               a["Nq"], a["Nk"], a["D"], ctypes.c_float(a["scale"]), a["causal"],
                               None, a["dtype"]) == code
+
+
+def test_unfused_entry_point_host_checks(lib):
+    a = dict(GOOD)
+    need = int(lib.fa_fwd_unfused_workspace_size(a["B"], a["Hq"], a["Nq"], a["Nk"]))
+    assert need == 256 * ((a["B"] * a["Hq"] * a["Nq"] * a["Nk"] * 4 + 255) // 256) + \
+        256 * ((a["B"] * a["Hq"] * a["Nq"] * a["Nk"] * 2 + 255) // 256)
+    assert lib.fa_fwd_unfused_workspace_size(0, 1, 1, 1) == 0
+
+    def call(ws=7 * A, nbytes=need, **kw):
+        b = dict(a)
+        b.update(kw)
+        return lib.fa_fwd_unfused(b["q"], b["k"], b["v"], b["o"], b["lse"], b["B"], b["Hq"],
+                                  b["Hkv"], b["Nq"], b["Nk"], b["D"], ctypes.c_float(b["scale"]),
+                                  b["causal"], None, b["dtype"], ws, nbytes)
+    bad_ws = fa.FA_ERR_BAD_WORKSPACE
+    assert call(ws=None) == bad_ws
+    assert call(nbytes=need - 1) == bad_ws
+    assert call(ws=7 * A + 16) == bad_ws
+    assert call(D=96) == 5 and call(dtype=2) == 7 and call(Hq=6, Hkv=4) == 4
+    assert call(q=0) == 1 and call(k=2 * A + 8) == 2 and call(o=1 * A + 64) == 12
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == 8  # valid arguments reach the device check
 
 
 def test_window_entry_point_host_checks(lib):

@@ -29,6 +29,7 @@ EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspa
             "fa_fwd_window", "fa_fwd_bias", "fa_bwd", "fa_bwd_window",
             "fa_bwd_workspace_size",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
+            "fa_fwd_unfused", "fa_fwd_unfused_workspace_size",
             "fa_status_string", "fa_device_status", "fa_device_timeout_site",
             "fa_debug_exp2_fma", "fa_debug_wait_timeout", "fa_fwd_num_tiles")
 
@@ -75,6 +76,10 @@ def load_library() -> ctypes.CDLL:
     lib.fa_fwd_noalloc.restype = i
     lib.fa_fwd_noalloc_scratch_bytes.argtypes = []
     lib.fa_fwd_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.fa_fwd_unfused.argtypes = fwd_args + [i, vp, ctypes.c_size_t]
+    lib.fa_fwd_unfused.restype = i
+    lib.fa_fwd_unfused_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_fwd_unfused_workspace_size.restype = ctypes.c_size_t
     lib.fa_fwd_workspace_size.argtypes = [i]
     lib.fa_fwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_set_max_ctas.argtypes = [i]
@@ -230,6 +235,43 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
         rc = lib.fa_fwd(*args)
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd")
+    return o, lse
+
+
+def fa_fwd_unfused(q, k, v, o=None, lse=None, scale: Optional[float] = None,
+                   causal: bool = False, stream=None, workspace=None):
+    """Standard three-step attention (S and P through device memory), for comparison.
+
+    Same tensors and arguments as fa_fwd; workspace: optional uint8 CUDA tensor
+    of at least fa_fwd_unfused_workspace_size bytes (allocated here when None).
+    Returns (o, lse).
+    """
+    import torch
+
+    lib = load_library()
+    if q.dtype not in (torch.float16, torch.bfloat16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype, float16 or bfloat16")
+    B, Hq, Nq, D = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    nbytes = int(lib.fa_fwd_unfused_workspace_size(B, Hq, Nq, Nk))
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    elif hasattr(stream, "cuda_stream"):
+        stream = stream.cuda_stream
+    dtype = FA_BF16 if q.dtype == torch.bfloat16 else FA_FP16
+    rc = lib.fa_fwd_unfused(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                            B, Hq, Hkv, Nq, Nk, D, ctypes.c_float(scale), 1 if causal else 0,
+                            stream or None, dtype, workspace.data_ptr(), workspace.numel())
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_unfused")
     return o, lse
 
 

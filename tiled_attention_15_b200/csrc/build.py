@@ -3,7 +3,8 @@
     python -m tiled_attention_15_b200.csrc.build [--verbose]
 
 nvcc compiles every ``*.cu`` file of this folder into one shared library with
-``-gencode arch=compute_100a,code=sm_100a`` (cross-compiles without a GPU).
+``-gencode arch=compute_100a,code=sm_100a`` (cross-compiles without a GPU),
+linked against cuBLAS (used only by the unfused comparison path).
 """
 from __future__ import annotations
 
@@ -37,7 +38,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
            "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           "-o", tmp] + sources()
+           "-o", tmp] + sources() + ["-lcublas"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)

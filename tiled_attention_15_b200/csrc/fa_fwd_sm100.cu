@@ -115,11 +115,15 @@ struct FwdParams {
   // Each part leaves its un-normalised partial in the workspace and the last one
   // to finish a row group merges (see merge_epilogue).
   int n_whole, n_units, nsplit;
-  int ws_rows;      // partial rows stored per split unit (rows of the tile that exist)
+  int ws_rows;      // partial rows stored per split unit: the rows of the tile that
+                    // exist, rounded up to whole warps (multiple of 32)
   // GQA packing (pack_g > 1): a work tile holds all pack_g query heads of one
   // key/value head, row r = (head r / Nq, query r % Nq), pack_g * Nq <= 128.
   int pack_g;
-  float* ws_o;      // [partial][ws_rows][D] partial O (fp32); a tile's parts are consecutive
+  // partial O (fp32), [partial][ws_rows / 32][D / 4][32 lanes] float4: one warp's
+  // 32 rows interleaved by column quad, so that a warp's stores and loads of a
+  // column quad are one contiguous 512-byte run; a tile's parts are consecutive
+  float4* ws_o;
   float4* ws_ml;    // [partial][ws_rows] (m, l, l_rounded, 0)
   int* ws_cnt;      // [split tile][NQ][4 row groups] arrival counters (left at 0)
   // Dynamic schedule (with a workspace): sched[0] hands out units beyond the
@@ -560,10 +564,12 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
     tc_fence_after();
     return true;
   };
-  auto p_ready = [&](int q) -> bool {
-    if (!wait_bar(B(G::B_PFULL + q), p_phase[q], cx.abort_flag)) return false;
-    p_phase[q] ^= 1u;
+  // P V of one key block, once the softmax has written P into S buffer sb
+  auto pv_block = [&](int ot, int sb, int st, bool acc) -> bool {
+    if (!wait_bar(B(G::B_PFULL + sb), p_phase[sb], cx.abort_flag)) return false;
+    p_phase[sb] ^= 1u;
     tc_fence_after();
+    issue_PV(ot, sb, st, acc);
     return true;
   };
 
@@ -598,8 +604,7 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
         if (!consume(vst)) return;
         if (j < e0) {
           if (j == 0 && !o_ready(0)) return;
-          if (!p_ready(0)) return;
-          issue_PV(0, 0, vst, j > 0);
+          if (!pv_block(0, 0, vst, j > 0)) return;
           if (j == e0 - 1) { mma_commit(B(G::B_OFULL + 0)); o_pending[0] = true; }
         }
         int kst2 = -1;
@@ -613,8 +618,7 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
         }
         if (in1(j)) {
           if (j == s1 && !o_ready(1)) return;
-          if (!p_ready(1)) return;
-          issue_PV(1, 1, vst, j > s1);
+          if (!pv_block(1, 1, vst, j > s1)) return;
           if (j == e1 - 1) { mma_commit(B(G::B_OFULL + 1)); o_pending[1] = true; }
         }
         mma_commit(B(G::B_KVEMPTY + vst));
@@ -649,8 +653,7 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
         if (!consume(vst)) return;
         if (j < T.nblk[0]) {
           if (j == 0 && !o_ready(0)) return;
-          if (!p_ready(0)) return;
-          issue_PV(0, 0, vst, j > 0);
+          if (!pv_block(0, 0, vst, j > 0)) return;
           if (j == T.nblk[0] - 1) { mma_commit(B(G::B_OFULL + 0)); o_pending[0] = true; }
         }
         int kst2 = -1;
@@ -664,8 +667,7 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
         }
         if (j < T.nblk[1]) {
           if (j == 0 && !o_ready(1)) return;
-          if (!p_ready(1)) return;
-          issue_PV(1, 1, vst, j > 0);
+          if (!pv_block(1, 1, vst, j > 0)) return;
           if (j == T.nblk[1] - 1) { mma_commit(B(G::B_OFULL + 1)); o_pending[1] = true; }
         }
         mma_commit(B(G::B_KVEMPTY + vst));
@@ -700,8 +702,7 @@ __device__ __forceinline__ void role_mma(const Ctx& cx, const FwdParams& p) {
         // S(j+1) is already issued here, so a fast softmax warp may finish block j+1
         // before a slow one finishes block j -- one barrier per buffer keeps their
         // arrivals apart (a warp can never get two blocks ahead: S(j+2) follows PV(j)).
-        if (!p_ready(j & 1)) return;
-        issue_PV(0, j & 1, vst, j > 0);
+        if (!pv_block(0, j & 1, vst, j > 0)) return;
         mma_commit(B(G::B_PVDONE));
         mma_commit(B(G::B_KVEMPTY + vst));
         if (j == nb - 1) { mma_commit(B(G::B_OFULL + 0)); o_pending[0] = true; }
@@ -751,23 +752,29 @@ __device__ __forceinline__ F2 unpack_bf16x2(uint32_t w) {
 }
 
 // Epilogue of one key part of a split tile, for the 32 rows of this warp.  Each
-// part stores its un-normalised O row (fp32), its stabiliser m and sums l, l_r;
+// part stores its un-normalised O rows (fp32), its stabiliser m and sums l, l_r;
 // then the warp bumps the counter of its row group.  The warp that arrives last
-// (the nparts-th) reads all parts, in part order, and writes the merged row:
+// (the nparts-th) reads all parts, in part order, and writes the merged rows:
 //   M = max_s m_s,  a_s = 2^(m_s - M),  L = sum_s a_s l_s,
 //   O = sum_s a_s O_s / L,  LSE = (M + log2 L) ln 2,
 // then resets the counter to 0 for the next call.  No part waits for another,
 // so no cross-CTA wait exists, and the result does not depend on which part
-// finished last.
+// finished last.  The partial rows of a warp are stored interleaved by column
+// quad (see FwdParams::ws_o), so every store and load of the partials is a
+// coalesced 512-byte run, and the merge keeps 8 loads per part in flight.
 template <int D, int NQ, bool BF16>
 __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T, int q, int sub,
                                                int lane, const RowInfo& ri, uint32_t ocol,
                                                float m, float l, float l_r) {
-  const int rr = q * kBM + sub * 32 + lane;  // row of the work tile
-  const bool stored = rr < p.ws_rows;         // rows beyond ws_rows do not exist
-  auto idx = [&](int part) { return (static_cast<size_t>(T.store0) + part) * p.ws_rows + rr; };
-  if (stored) p.ws_ml[idx(T.part)] = make_float4(m, l, l_r, 0.f);
-  float4* my_o = reinterpret_cast<float4*>(p.ws_o + idx(stored ? T.part : 0) * D);
+  const int g0 = q * kBM + sub * 32;  // first row of this warp in the work tile
+  const int rr = g0 + lane;
+  // warp-uniform: the warp's rows lie within the stored (padded) rows of the unit
+  const bool stored = g0 < p.ws_rows;
+  auto mlx = [&](int part) { return (static_cast<size_t>(T.store0) + part) * p.ws_rows + rr; };
+  auto ox = [&](int part, int c4) {
+    return ((static_cast<size_t>(T.store0) + part) * p.ws_rows + g0) * (D / 4) + c4 * 32 + lane;
+  };
+  if (stored) p.ws_ml[mlx(T.part)] = make_float4(m, l, l_r, 0.f);
 #pragma unroll 1
   for (int c0 = 0; c0 < D; c0 += 32) {
     uint32_t orr[32];
@@ -775,8 +782,9 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
     if (stored) {
 #pragma unroll
       for (int x = 0; x < 8; ++x)
-        my_o[c0 / 4 + x] = make_float4(__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
-                                       __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3]));
+        p.ws_o[ox(T.part, c0 / 4 + x)] =
+            make_float4(__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
+                        __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3]));
     }
   }
   __threadfence();
@@ -789,10 +797,10 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
   __threadfence();
   if (stored) {
     float M = -INFINITY;
-    for (int s = 0; s < T.nparts; ++s) M = fmaxf(M, __ldcg(p.ws_ml + idx(s)).x);
+    for (int s = 0; s < T.nparts; ++s) M = fmaxf(M, __ldcg(p.ws_ml + mlx(s)).x);
     float L = 0.f, Lr = 0.f;
     for (int s = 0; s < T.nparts; ++s) {
-      const float4 ml = __ldcg(p.ws_ml + idx(s));
+      const float4 ml = __ldcg(p.ws_ml + mlx(s));
       const float a = ex2(ml.x - M);
       L = fmaf(a, ml.y, L);
       Lr = fmaf(a, ml.z, Lr);
@@ -800,21 +808,31 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T
     const float inv = 1.f / (BF16 ? Lr : L);
     uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 8) {
-      float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c4 = 0; c4 < D / 4; c4 += 8) {  // 32 columns per pass
+      float z[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x) z[x] = 0.f;
       for (int s = 0; s < T.nparts; ++s) {
-        const float sc = ex2(__ldcg(p.ws_ml + idx(s)).x - M) * inv;
-        const float4* po = reinterpret_cast<const float4*>(p.ws_o + idx(s) * D + c0);
-        const float4 u0 = __ldcg(po), u1 = __ldcg(po + 1);
-        z[0] = fmaf(u0.x, sc, z[0]); z[1] = fmaf(u0.y, sc, z[1]);
-        z[2] = fmaf(u0.z, sc, z[2]); z[3] = fmaf(u0.w, sc, z[3]);
-        z[4] = fmaf(u1.x, sc, z[4]); z[5] = fmaf(u1.y, sc, z[5]);
-        z[6] = fmaf(u1.z, sc, z[6]); z[7] = fmaf(u1.w, sc, z[7]);
+        const float sc = ex2(__ldcg(p.ws_ml + mlx(s)).x - M) * inv;
+        float4 u[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) u[x] = __ldcg(p.ws_o + ox(s, c4 + x));
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          z[4 * x] = fmaf(u[x].x, sc, z[4 * x]);
+          z[4 * x + 1] = fmaf(u[x].y, sc, z[4 * x + 1]);
+          z[4 * x + 2] = fmaf(u[x].z, sc, z[4 * x + 2]);
+          z[4 * x + 3] = fmaf(u[x].w, sc, z[4 * x + 3]);
+        }
       }
-      if (ri.live)
-        *reinterpret_cast<uint4*>(orow + c0) =
-            make_uint4(pack2(z[0], z[1], BF16), pack2(z[2], z[3], BF16), pack2(z[4], z[5], BF16),
-                       pack2(z[6], z[7], BF16));
+      if (ri.live) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 4);
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+          dst[x] = make_uint4(pack2(z[8 * x], z[8 * x + 1], BF16), pack2(z[8 * x + 2], z[8 * x + 3], BF16),
+                              pack2(z[8 * x + 4], z[8 * x + 5], BF16),
+                              pack2(z[8 * x + 6], z[8 * x + 7], BF16));
+      }
     }
     if (p.lse != nullptr && ri.live) p.lse[ri.out_row] = (M + log2f(L)) * kLn2;
   }
@@ -1228,7 +1246,7 @@ std::atomic<int> g_max_ctas{0};
 // partial results of up to max_split tiles follow.  Offsets are multiples of
 // 256 bytes.
 constexpr int kMaxSplit = 1024;  // >= half the SMs of any device
-constexpr int kMinSplitBlocks = 24;
+constexpr int kMinSplitBlocks = 8;
 constexpr int kMinPartBlocks = 4;  // least key blocks per CTA under stream-K
 struct WsLayout {
   size_t cnt_off, ml_off, o_off, total;
@@ -1328,9 +1346,11 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   int ctas = g_dev[dev].sms;
   const int cap = g_max_ctas.load();
   if (cap > 0 && cap < ctas) ctas = cap;
-  // rows of a work tile that exist (partials are stored for these only)
+  // rows of a work tile that exist, rounded up to whole warps (partials are
+  // stored for these only)
   p.ws_rows = pack ? g * Nq : (p.qt_per_head == 1 ? (Nq < NQ * fa::kBM ? Nq : NQ * fa::kBM)
                                                    : NQ * fa::kBM);
+  p.ws_rows = (p.ws_rows + 31) / 32 * 32;
   int n_split = 0, nsplit = 1;
   int sk_w = 0, sk_grid = 0;
   if (ws != nullptr && !causal && !windowed && !BIAS) {
@@ -1350,9 +1370,9 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     } else {
       // Split tail: if the last round of tiles would keep at most half of the
       // CTAs busy, give each of those tiles to two CTAs, one per half of the key
-      // blocks.  Below kMinSplitBlocks key blocks the halves are too short to pay
-      // for writing and re-reading the fp32 partials (measured on the LLaMA-7B
-      // layer shape).
+      // blocks.  With coalesced partials and a merge that keeps its loads in
+      // flight this pays from 16 key blocks on (the LLaMA-7B layer shape:
+      // +5 %); below kMinSplitBlocks the halves are too short for it.
       const int grid0 = p.n_tiles < ctas ? p.n_tiles : ctas;
       const int rem = p.n_tiles % grid0;
       if (p.nkb >= kMinSplitBlocks && p.n_tiles > grid0 && rem > 0 && 2 * rem <= grid0 &&
@@ -1374,7 +1394,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
           cudaMemsetAsync(ws, 0, L.ml_off, stream) != cudaSuccess)  // the counters start at zero
         return FA_ERR_LAUNCH;
       char* base = static_cast<char*>(ws);
-      p.ws_o = reinterpret_cast<float*>(base + L.o_off);
+      p.ws_o = reinterpret_cast<float4*>(base + L.o_off);
       p.ws_ml = reinterpret_cast<float4*>(base + L.ml_off);
       p.ws_cnt = reinterpret_cast<int*>(base + L.cnt_off);
     }
@@ -1437,7 +1457,8 @@ const char* fa_status_string(int s) {
       return "fa_fwd_noalloc: this problem needs more scratch than the static buffer holds; "
              "use fa_fwd_ws";
     case FA_ERR_BAD_WORKSPACE:
-      return "fa_bwd: workspace missing or smaller than fa_bwd_workspace_size(B, Hq, Nq)";
+      return "workspace missing, misaligned or smaller than the entry point's *_workspace_size()";
+    case FA_ERR_LIBRARY: return "fa_fwd_unfused: a cuBLAS call failed";
     case FA_ERR_BAD_WINDOW:
       return "key window bounds must be >= -1, and a causal launch cannot have window_right > 0";
     default: return "unknown status";
