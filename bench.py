@@ -133,7 +133,12 @@ def recorded_traffic():
 
 
 class ClockSampler:
-    """NVML samples of SM clock and clock-event reasons while the timed region runs."""
+    """NVML samples of SM clock and clock-event reasons while the GPU works.
+
+    Runs from the warm-up to the end of the per-workload lines; summary() gives
+    the median SM clock and the union of throttle reasons over all samples, and
+    how many of them fell inside the timed region of the step (an NVML query
+    takes a few ms, so a short timed region gets only a few)."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -142,7 +147,8 @@ class ClockSampler:
 
     def __init__(self, index: int):
         self.ok = False
-        self.samples, self.reasons = [], set()
+        self.samples = []  # (time, mhz, reason bits)
+        self.window = [None, None]
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -158,14 +164,16 @@ class ClockSampler:
         nv = self.nv
         while not self._stop.is_set():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
+                self.samples.append((time.perf_counter(), mhz, r))
             except Exception:  # noqa: BLE001
                 pass
             time.sleep(0.001)
+
+    def mark(self, i: int):
+        """Mark the start (0) or end (1) of the timed region."""
+        self.window[i] = time.perf_counter()
 
     def __enter__(self):
         if self.ok:
@@ -179,10 +187,19 @@ class ClockSampler:
             self.t.join()
 
     def summary(self):
-        if not self.ok or not self.samples:
+        busy = [x for x in self.samples if not x[2] & 0x1]  # gpu_idle samples left out
+        if not self.ok or not busy:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+        reasons = set()
+        for _, _, r in busy:
+            reasons |= {n for b, n in self.REASONS.items() if r & b}
+        t0, t1 = self.window
+        timed = [m for t, m, _ in busy if t0 is not None and t1 is not None and t0 <= t <= t1]
+        return {"sm_mhz": statistics.median(m for _, m, _ in busy), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(busy),
+                "timed_region_samples": len(timed),
+                "timed_region_sm_mhz": statistics.median(timed) if timed else None,
+                "window": "warm-up through the per-workload lines (GPU busy)"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -329,6 +346,8 @@ def main():
                   o=o, lse=lse, scale=w.softmax_scale, causal=w.causal,
                   stream=sptr if st is None else st)
 
+    clk = ClockSampler(local)
+    clk.__enter__()
     for _ in range(args.warmup):
         for j in range(len(ws)):
             flush.zero_()
@@ -342,14 +361,15 @@ def main():
            for _ in ws] for _ in range(K)]
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(K):
-            for j in range(len(ws)):
-                flush.zero_()
-                ev[i][j][0].record(stream)
-                run_pass(j)
-                ev[i][j][1].record(stream)
-        torch.cuda.synchronize()
+    clk.mark(0)
+    for i in range(K):
+        for j in range(len(ws)):
+            flush.zero_()
+            ev[i][j][0].record(stream)
+            run_pass(j)
+            ev[i][j][1].record(stream)
+    torch.cuda.synchronize()
+    clk.mark(1)
     barrier()
     per_pass = [[ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(K)] for j in range(len(ws))]
     total_ms = max_over_ranks(sum(sum(x) for x in per_pass), world, dev)
@@ -455,6 +475,7 @@ def main():
                            "alg_gbs: algorithmic bytes (read Q, K, V once, write O and LSE once) "
                            "per second, frac_of_hbm against the measured copy bandwidth")
         assert fa.device_status(reset=True) == 0
+    clk.__exit__(None, None, None)
     gate = {}
     for n in (4096, 8192):
         for cz in ("non-causal", "causal"):
