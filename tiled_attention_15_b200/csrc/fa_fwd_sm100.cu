@@ -86,11 +86,13 @@ struct Geometry {
                        B_SFULL = 4 + 2 * NST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
                        B_OEMPTY = B_OFULL + 2, B_PVDONE = B_OEMPTY + 2, B_TFULL = B_PVDONE + 1,
                        B_TEMPTY = B_TFULL + kTileRing, B_BFULL = B_TEMPTY + kTileRing,
-                       B_BEMPTY = B_BFULL + NBS, NBAR = B_BEMPTY + NBS;
+                       B_BEMPTY = B_BFULL + NBS, B_MSTORED = B_BEMPTY + NBS,
+                       B_MLAST = B_MSTORED + 2, NBAR = B_MLAST + 2;
   // tmem base (u32), abort flag (u32), then the ring of unit indices (kTileRing x s32)
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // ... then this CTA's stream-K unit range (2 x s32)
-  static constexpr int SMEM_BYTES = OFF_MISC + 8 + 4 * kTileRing + 8 + 1024;  // + alignment slack
+  // ... then this CTA's stream-K unit range (2 x s32), then per query tile the
+  // split-merge verdict (2 x s32: 1 = this CTA merges the tile)
+  static constexpr int SMEM_BYTES = OFF_MISC + 8 + 4 * kTileRing + 8 + 8 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(NQ == 2 ? (256 + 2 * D <= 512) : (256 + D <= 512), "tensor memory budget");
@@ -125,7 +127,8 @@ struct FwdParams {
   // column quad are one contiguous 512-byte run; a tile's parts are consecutive
   float4* ws_o;
   float4* ws_ml;    // [partial][ws_rows] (m, l, l_rounded, 0)
-  int* ws_cnt;      // [split tile][NQ][4 row groups] arrival counters (left at 0)
+  int* ws_cnt;      // [split tile][NQ][4 row groups] arrival counters (left at 0); one
+                    // query tile per work tile uses [split tile][0][0] only
   // Dynamic schedule (with a workspace): sched[0] hands out units beyond the
   // first gridDim.x, sched[1] counts finished CTAs; the last CTA resets both.
   int* sched;
@@ -751,7 +754,126 @@ __device__ __forceinline__ F2 unpack_bf16x2(uint32_t w) {
   return F2{__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)};
 }
 
-// Epilogue of one key part of a split tile, for the 32 rows of this warp.  Each
+// Epilogue of one key part of a split tile (one query tile: KV-cache decode
+// tiles often have a single row group).  Each warp of the query tile's
+// warpgroup stores its un-normalised O rows (fp32), stabiliser m and sums l,
+// l_r; once all four warps have stored (a bounded mbarrier handshake), warp 0
+// bumps the tile's arrival counter.  The CTA that arrives last (the nparts-th)
+// merges the tile with all four warps -- one 32-row group each, or, when the
+// tile has fewer row groups than warps (KV-cache decode), column slices of
+// them -- reading the parts in part order:
+//   M = max_s m_s,  a_s = 2^(m_s - M),  L = sum_s a_s l_s,
+//   O = sum_s a_s O_s / L,  LSE = (M + log2 L) ln 2,
+// and resets the counter to 0 for the next call.  No part waits for another
+// CTA, and the result does not depend on which part finished last.  The
+// partial rows of a warp are stored interleaved by column quad (see
+// FwdParams::ws_o), so every store and load of the partials is a coalesced
+// 512-byte run.  Returns false if a handshake wait gave up (abort).
+template <int D, int NQ, bool BF16, class G>
+__device__ __forceinline__ bool merge_epilogue(const Ctx& cx, uint32_t& m_phase, const FwdParams& p,
+                                               const Tile& T, int q, int sub, int lane, uint32_t ocol,
+                                               float m, float l, float l_r) {
+  const uint32_t b_stored = cx.bar(G::B_MSTORED + q, G::OFF_BAR), b_last = cx.bar(G::B_MLAST + q, G::OFF_BAR);
+  volatile int* verdict = cx.ring + kTileRing + 2 + q;
+  const int g0 = q * kBM + sub * 32;  // first row of this warp in the work tile
+  const int rr = g0 + lane;
+  // warp-uniform: the warp's rows lie within the stored (padded) rows of the unit
+  const bool stored = g0 < p.ws_rows;
+  auto mlx = [&](int part, int r) { return (static_cast<size_t>(T.store0) + part) * p.ws_rows + r; };
+  auto ox = [&](int part, int gr, int c4) {  // gr: first row of a 32-row group
+    return ((static_cast<size_t>(T.store0) + part) * p.ws_rows + gr) * (D / 4) + c4 * 32 + lane;
+  };
+  if (stored) p.ws_ml[mlx(T.part, rr)] = make_float4(m, l, l_r, 0.f);
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t orr[32];
+    tmem_ld_x32(ocol + c0, orr);  // warp-collective: every lane takes part
+    if (stored) {
+#pragma unroll
+      for (int x = 0; x < 8; ++x)
+        p.ws_o[ox(T.part, g0, c0 / 4 + x)] =
+            make_float4(__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
+                        __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3]));
+    }
+  }
+  __threadfence();
+  __syncwarp();
+  // all four warps have stored -> warp 0 takes the tile's verdict -> all read it
+  if (lane == 0) mbar_arrive(b_stored);
+  bool ok = wait_bar(b_stored, m_phase, cx.abort_flag);
+  if (!__all_sync(0xffffffffu, ok)) return false;
+  int* cnt = p.ws_cnt + (T.slot * NQ + q) * 4;
+  if (sub == 0) {
+    int old = 0;
+    if (lane == 0) {
+      old = atomicAdd(cnt, 1);
+      *verdict = old == T.nparts - 1 ? 1 : 0;
+      mbar_arrive(b_last);
+    }
+  }
+  ok = wait_bar(b_last, m_phase, cx.abort_flag);
+  if (!__all_sync(0xffffffffu, ok)) return false;
+  m_phase ^= 1u;
+  const bool last = *verdict != 0;
+  __syncwarp();
+  if (!last) return true;  // a later part merges this tile
+  __threadfence();
+  // this warp's share: row group gsel, column quads [c4a, c4b)
+  const int rows_q = min(p.ws_rows - q * kBM, kBM);  // stored rows of this query tile (x32)
+  const int ng = rows_q > 0 ? rows_q / 32 : 0;         // its row groups (1..4)
+  if (ng == 0) return true;
+  const int per = 4 / ng;                              // warps per row group (ng = 3: 1)
+  const int gsel = sub / per, slice = sub % per;
+  if (gsel >= ng) return true;
+  const int c4a = slice * (D / 4) / per, c4b = (slice + 1) * (D / 4) / per;
+  const int gr = q * kBM + gsel * 32;
+  const RowInfo ri = row_info(p, T, q, gsel * 32 + lane);
+  float M = -INFINITY;
+  for (int s = 0; s < T.nparts; ++s) M = fmaxf(M, __ldcg(p.ws_ml + mlx(s, gr + lane)).x);
+  float L = 0.f, Lr = 0.f;
+  for (int s = 0; s < T.nparts; ++s) {
+    const float4 ml = __ldcg(p.ws_ml + mlx(s, gr + lane));
+    const float a = ex2(ml.x - M);
+    L = fmaf(a, ml.y, L);
+    Lr = fmaf(a, ml.z, Lr);
+  }
+  const float inv = 1.f / (BF16 ? Lr : L);
+  uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
+#pragma unroll 1
+  for (int c4 = c4a; c4 < c4b; c4 += 4) {  // 16 columns per pass
+    float z[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) z[x] = 0.f;
+    for (int s = 0; s < T.nparts; ++s) {
+      const float sc = ex2(__ldcg(p.ws_ml + mlx(s, gr + lane)).x - M) * inv;
+      float4 u[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) u[x] = __ldcg(p.ws_o + ox(s, gr, c4 + x));
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        z[4 * x] = fmaf(u[x].x, sc, z[4 * x]);
+        z[4 * x + 1] = fmaf(u[x].y, sc, z[4 * x + 1]);
+        z[4 * x + 2] = fmaf(u[x].z, sc, z[4 * x + 2]);
+        z[4 * x + 3] = fmaf(u[x].w, sc, z[4 * x + 3]);
+      }
+    }
+    if (ri.live) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 4);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+        dst[x] = make_uint4(pack2(z[8 * x], z[8 * x + 1], BF16), pack2(z[8 * x + 2], z[8 * x + 3], BF16),
+                            pack2(z[8 * x + 4], z[8 * x + 5], BF16),
+                            pack2(z[8 * x + 6], z[8 * x + 7], BF16));
+    }
+  }
+  if (slice == 0 && p.lse != nullptr && ri.live) p.lse[ri.out_row] = (M + log2f(L)) * kLn2;
+  __syncwarp();
+  if (sub == 0 && lane == 0) *cnt = 0;  // every part has arrived: safe to reset
+  return true;
+}
+
+// Epilogue of one key part of a split tile, for the 32 rows of this warp (two
+// query tiles: each query tile has four row groups, one per warp).  Each
 // part stores its un-normalised O rows (fp32), its stabiliser m and sums l, l_r;
 // then the warp bumps the counter of its row group.  The warp that arrives last
 // (the nparts-th) reads all parts, in part order, and writes the merged rows:
@@ -763,9 +885,9 @@ __device__ __forceinline__ F2 unpack_bf16x2(uint32_t w) {
 // quad (see FwdParams::ws_o), so every store and load of the partials is a
 // coalesced 512-byte run, and the merge keeps 8 loads per part in flight.
 template <int D, int NQ, bool BF16>
-__device__ __forceinline__ void merge_epilogue(const FwdParams& p, const Tile& T, int q, int sub,
-                                               int lane, const RowInfo& ri, uint32_t ocol,
-                                               float m, float l, float l_r) {
+__device__ __forceinline__ void merge_epilogue_rows(const FwdParams& p, const Tile& T, int q, int sub,
+                                                    int lane, const RowInfo& ri, uint32_t ocol,
+                                                    float m, float l, float l_r) {
   const int g0 = q * kBM + sub * 32;  // first row of this warp in the work tile
   const int rr = g0 + lane;
   // warp-uniform: the warp's rows lie within the stored (padded) rows of the unit
@@ -850,7 +972,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
   const float c = p.c;
   constexpr bool kWin = NQ == 1 || WIN;  // kernels that take key windows
-  uint32_t s_phase[2] = {0u, 0u}, of_phase = 0u, pv_seen = 0u;
+  uint32_t s_phase[2] = {0u, 0u}, of_phase = 0u, pv_seen = 0u, m_phase = 0u;
   uint32_t b_cnt = 0, b_phase = 0u;  // bias tiles consumed; parity bit per stage
   const int q = (NQ == 2) ? wg : 0;
 
@@ -1018,7 +1140,12 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     const bool live = ri.live;
     const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
     if (T.slot >= 0) {
-      merge_epilogue<D, NQ, BF16>(p, T, q, sub, lane, ri, tm + 256 + q * D, m_sub, l, l_r);
+      if constexpr (NQ == 2) {
+        merge_epilogue_rows<D, NQ, BF16>(p, T, q, sub, lane, ri, tm + 256 + q * D, m_sub, l, l_r);
+      } else if (!merge_epilogue<D, NQ, BF16, G>(cx, m_phase, p, T, q, sub, lane, tm + 256 + q * D,
+                                                 m_sub, l, l_r)) {
+        return;
+      }
     } else {
       // a row that saw no key (key windows only) has no softmax: O = 0, LSE = -inf
       const bool empty = kWin && m_used == -INFINITY;
@@ -1083,6 +1210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(B(G::B_OEMPTY + q), 4);
     }
     mbar_init(B(G::B_PVDONE), 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(B(G::B_MSTORED + q), 4);  // the four warps of query tile q's warpgroup
+      mbar_init(B(G::B_MLAST + q), 1);
+    }
     for (int k = 0; k < kTileRing; ++k) {
       mbar_init(B(G::B_TFULL + k), 1);
       mbar_init(B(G::B_TEMPTY + k), 1 + 4 * NQ);  // the MMA thread and the softmax warps
