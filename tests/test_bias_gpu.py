@@ -105,3 +105,18 @@ def test_unaligned_key_count_is_padded(cuda_dev):
     # Nk = 77: the binding copies the bias into rows padded to 80 keys
     w = Workload("Nk 77 D64 fp16", 1, 2, 2, 90, 77, 64, "fp16", False, seed=118)
     _check(w, _bias(w, (1, 2, 90, 77), 6), cuda_dev)
+
+
+def test_bias_many_tiles_per_cta(cuda_dev):
+    # two-query-tile bias kernel over several work tiles per CTA (CTA cap 8):
+    # the bias producer and the softmax warps stay in step across units
+    w = Workload("shared [N,N] D128 fp16 many tiles", 2, 8, 8, 1024, 1024, 128, "fp16", False,
+                 seed=119)
+    prev = fa.set_max_ctas(8)
+    try:
+        _check(w, _bias(w, (1, 1, 1024, 1024), 7), cuda_dev)
+        wc = w.with_(name="per head [1,H,N,N] D64 bf16 causal many tiles", D=64, dtype="bf16",
+                     causal=True, seed=120)
+        _check(wc, _bias(wc, (1, 8, 1024, 1024), 8), cuda_dev)
+    finally:
+        fa.set_max_ctas(prev)

@@ -72,9 +72,11 @@ struct Geometry {
   static constexpr int CHUNK_KV = kBN * 128;  // one 64-column chunk of a K/V block
   // K/V stages: what the shared memory left by the Q tiles holds (one query
   // tile leaves room for deeper staging, which decode-like launches need)
-  static constexpr int NST = BIAS ? (D == 64 ? 8 : (D == 128 ? 4 : 2))
+  // (score bias with two query tiles: one bias tile per query tile, 3 K/V stages at D = 128)
+  static constexpr int NST = BIAS ? (NQ == 2 ? (D == 64 ? 8 : 3) : (D == 64 ? 8 : (D == 128 ? 4 : 2)))
                                   : NQ == 2 ? (D == 64 ? 8 : 4) : (D == 64 ? 12 : (D == 128 ? 6 : 2));
-  // score-bias tiles (bias launches: one query tile): [2 boxes][128 rows][64 keys], 16-bit
+  // score-bias tiles: [2 boxes][128 rows][64 keys], 16-bit; one query tile: a
+  // ring of NBS, two query tiles: one per query tile
   static constexpr int NBS = BIAS ? (D == 256 ? 1 : 2) : 0;
   static constexpr int BIAS_BYTES = 128 * 128 * 2;
   static constexpr int OFF_Q = 0;
@@ -484,7 +486,7 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
     //   NQ = 2: K0, V0, K1, V1, ...      NQ = 1: K0, K1, V0, K2, V1, ...
     if (T.nblk[0] > 0 && !load_q(T, 0)) { ok = false; break; }
     if (!load_kv(T, tk, 0)) { ok = false; break; }
-    if (BIAS && !load_bias(T, 0)) { ok = false; break; }
+    if (BIAS && NQ == 1 && !load_bias(T, 0)) { ok = false; break; }
     if (NQ == 2 && T.nblk[1] > 0 && !load_q(T, 1)) { ok = false; break; }
     for (int s = 1; s < 2 * T.nb && ok; ++s) {
       int j;
@@ -495,7 +497,7 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
         else { is_k = (s & 1) == 1; j = is_k ? (s + 1) / 2 : s / 2 - 1; }
       }
       if (!load_kv(T, is_k ? tk : tv, j)) ok = false;
-      if (BIAS && ok && is_k && !load_bias(T, j)) ok = false;
+      if (BIAS && NQ == 1 && ok && is_k && !load_bias(T, j)) ok = false;
     }
   }
   if (!ok) {  // abort: let this CTA's own loads land before the CTA exits
@@ -507,6 +509,52 @@ __device__ __forceinline__ void role_load(const Ctx& cx, const FwdParams& p, con
       for (uint32_t n = (b_it > (uint32_t)G::NBS ? b_it - G::NBS : 0); n < b_it; ++n)
         drain_bar(cx.bar(G::B_BFULL + n % G::NBS, G::OFF_BAR), (n / G::NBS) & 1u);
   }
+}
+
+// ---------------------------------------------------------------- score-bias producer
+// Two query tiles with a score bias: one thread of warp 10 streams, per key
+// block, each query tile's [128 x 128] bias tile into that query tile's own
+// buffer (two 64-key boxes, 128-byte swizzle; one row when the bias is
+// broadcast over queries), as soon as the tile's softmax warps have read the
+// previous block's.  It takes the units from the same schedule as the others.
+template <int D, int NQ, bool BIAS, bool WIN>
+__device__ __forceinline__ void role_bias_load(const Ctx& cx, const FwdParams& p, const CUtensorMap* tb,
+                                               int bias_mode) {
+  using G = Geometry<D, NQ, BIAS>;
+  prefetch_tmap(tb);
+  const uint64_t pol = policy_evict_last();
+  uint32_t issued[2] = {0u, 0u};
+  bool ok = true;
+  TileIter it(p.n_units);
+  uint32_t n_units_seen = 0;
+  int t;
+  while (ok && consume_unit<D, NQ, BIAS>(cx, p, it, n_units_seen, t, -1)) {
+    const Tile T = get_tile<NQ, WIN>(p, t);
+    const int hq = T.bh % p.Hq, b = T.bh / p.Hq;
+    const int rows = (bias_mode & kBiasRowBcast) ? 1 : kBM;
+    for (int j = 0; j < T.nb && ok; ++j) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (j >= T.nblk[q]) continue;
+        if (issued[q] > 0 &&
+            !wait_bar(cx.bar(G::B_BEMPTY + q, G::OFF_BAR), (issued[q] - 1) & 1u, cx.abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(cx.bar(G::B_BFULL + q, G::OFF_BAR), 2 * rows * 128);
+#pragma unroll
+        for (int box = 0; box < 2; ++box)
+          tma_load_4d(cx.sbase + G::OFF_BIAS + q * G::BIAS_BYTES + box * (G::BIAS_BYTES / 2), tb,
+                      cx.bar(G::B_BFULL + q, G::OFF_BAR), (T.jb + j) * kBN + box * 64,
+                      (bias_mode & kBiasRowBcast) ? 0 : T.row0 + q * kBM,
+                      (bias_mode & kBiasPerHead) ? hq : 0, (bias_mode & kBiasPerBatch) ? b : 0, pol);
+        ++issued[q];
+      }
+    }
+  }
+  if (!ok)  // abort: let this thread's own loads land before the CTA exits
+    for (int q = 0; q < 2; ++q)
+      if (issued[q] > 0) drain_bar(cx.bar(G::B_BFULL + q, G::OFF_BAR), (issued[q] - 1) & 1u);
 }
 
 // ---------------------------------------------------------------- MMA issuer
@@ -828,14 +876,29 @@ __device__ __forceinline__ bool merge_epilogue(const Ctx& cx, uint32_t& m_phase,
   const int c4a = slice * (D / 4) / per, c4b = (slice + 1) * (D / 4) / per;
   const int gr = q * kBM + gsel * 32;
   const RowInfo ri = row_info(p, T, q, gsel * 32 + lane);
+  // Parts are read four at a time with all their loads issued before use, so
+  // a tile merged from many parts (stream-K) pays one memory latency per four.
+  const int np = T.nparts;
   float M = -INFINITY;
-  for (int s = 0; s < T.nparts; ++s) M = fmaxf(M, __ldcg(p.ws_ml + mlx(s, gr + lane)).x);
+  for (int s0 = 0; s0 < np; s0 += 4) {
+    float mk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mk[k] = s0 + k < np ? __ldcg(p.ws_ml + mlx(s0 + k, gr + lane)).x : -INFINITY;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) M = fmaxf(M, mk[k]);
+  }
   float L = 0.f, Lr = 0.f;
-  for (int s = 0; s < T.nparts; ++s) {
-    const float4 ml = __ldcg(p.ws_ml + mlx(s, gr + lane));
-    const float a = ex2(ml.x - M);
-    L = fmaf(a, ml.y, L);
-    Lr = fmaf(a, ml.z, Lr);
+  for (int s0 = 0; s0 < np; s0 += 4) {
+    float4 mk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      mk[k] = s0 + k < np ? __ldcg(p.ws_ml + mlx(s0 + k, gr + lane)) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = ex2(mk[k].x - M);
+      L = fmaf(a, mk[k].y, L);
+      Lr = fmaf(a, mk[k].z, Lr);
+    }
   }
   const float inv = 1.f / (BF16 ? Lr : L);
   uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
@@ -844,18 +907,26 @@ __device__ __forceinline__ bool merge_epilogue(const Ctx& cx, uint32_t& m_phase,
     float z[16];
 #pragma unroll
     for (int x = 0; x < 16; ++x) z[x] = 0.f;
-    for (int s = 0; s < T.nparts; ++s) {
-      const float sc = ex2(__ldcg(p.ws_ml + mlx(s, gr + lane)).x - M) * inv;
-      float4 u[4];
+    for (int s0 = 0; s0 < np; s0 += 4) {
+      float sc[4];
+      float4 u[4][4];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) u[x] = __ldcg(p.ws_o + ox(s, gr, c4 + x));
+      for (int k = 0; k < 4; ++k) {
+        const bool in = s0 + k < np;
+        const int sk = in ? s0 + k : s0;  // (a valid address; its weight is 0)
+        sc[k] = in ? ex2(__ldcg(p.ws_ml + mlx(sk, gr + lane)).x - M) * inv : 0.f;
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        z[4 * x] = fmaf(u[x].x, sc, z[4 * x]);
-        z[4 * x + 1] = fmaf(u[x].y, sc, z[4 * x + 1]);
-        z[4 * x + 2] = fmaf(u[x].z, sc, z[4 * x + 2]);
-        z[4 * x + 3] = fmaf(u[x].w, sc, z[4 * x + 3]);
+        for (int x = 0; x < 4; ++x) u[k][x] = __ldcg(p.ws_o + ox(sk, gr, c4 + x));
       }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          z[4 * x] = fmaf(u[k][x].x, sc[k], z[4 * x]);
+          z[4 * x + 1] = fmaf(u[k][x].y, sc[k], z[4 * x + 1]);
+          z[4 * x + 2] = fmaf(u[k][x].z, sc[k], z[4 * x + 2]);
+          z[4 * x + 3] = fmaf(u[k][x].w, sc[k], z[4 * x + 3]);
+        }
     }
     if (ri.live) {
       uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 4);
@@ -1017,7 +1088,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
           // values as 16 swizzled 16-byte units (one row for every query when
           // broadcast over queries)
           if (p.causal) lim = min(lim, row - kbase + 1);
-          const int bs = b_cnt % G::NBS;
+          const int bs = NQ == 2 ? q : static_cast<int>(b_cnt % G::NBS);
           ok = wait_bar(B(G::B_BFULL + bs), (b_phase >> bs) & 1u, cx.abort_flag);
           if (!__all_sync(0xffffffffu, ok)) return;
           b_phase ^= 1u << bs;
@@ -1147,8 +1218,9 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
         return;
       }
     } else {
-      // a row that saw no key (key windows only) has no softmax: O = 0, LSE = -inf
-      const bool empty = kWin && m_used == -INFINITY;
+      // a row that saw no key (key windows, or a bias of -inf on every key) has no
+      // softmax: O = 0, LSE = -inf
+      const bool empty = (kWin || BIAS) && m_used == -INFINITY;
       const float inv_l = empty ? 0.f : 1.f / (BF16 ? l_r : l);
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
 #pragma unroll 1
@@ -1216,7 +1288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int k = 0; k < kTileRing; ++k) {
       mbar_init(B(G::B_TFULL + k), 1);
-      mbar_init(B(G::B_TEMPTY + k), 1 + 4 * NQ);  // the MMA thread and the softmax warps
+      // the MMA thread, the softmax warps (and the bias producer)
+      mbar_init(B(G::B_TEMPTY + k), 1 + 4 * NQ + ((BIAS && NQ == 2) ? 1 : 0));
     }
     for (int k = 0; k < G::NBS; ++k) {
       mbar_init(B(G::B_BFULL + k), 1);
@@ -1257,6 +1330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) role_mma<D, NQ, BF16, BIAS, WIN>(cx, p);
   } else if (warp == 9) {
     if (lane == 0) role_load<D, NQ, BIAS, WIN>(cx, p, &tm_q, &tm_q4, &tm_k, &tm_v, &tm_b, bias_mode);
+  } else if (warp == 10) {
+    if (BIAS && NQ == 2 && lane == 0) role_bias_load<D, NQ, BIAS, WIN>(cx, p, &tm_b, bias_mode);
   }
   __syncwarp();
   tc_fence_before();
@@ -1657,6 +1732,11 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   if (bias != nullptr) {  // score bias: the one-query-tile kernels with bias staging
 #define FA_BARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, -1, -1, st, dev, nullptr, 0, \
                  Scratch::kCaller, bias
+    // more than 128 query rows (D <= 128): the two-query-tile kernel
+    if (D == 64 && Nq > fa::kBM)
+      return bf ? launch<64, 2, true, true>(FA_BARGS) : launch<64, 2, false, true>(FA_BARGS);
+    if (D == 128 && Nq > fa::kBM)
+      return bf ? launch<128, 2, true, true>(FA_BARGS) : launch<128, 2, false, true>(FA_BARGS);
     switch (D) {
       case 64: return bf ? launch<64, 1, true, true>(FA_BARGS) : launch<64, 1, false, true>(FA_BARGS);
       case 128: return bf ? launch<128, 1, true, true>(FA_BARGS) : launch<128, 1, false, true>(FA_BARGS);

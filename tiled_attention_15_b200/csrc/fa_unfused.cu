@@ -55,8 +55,9 @@ __device__ __forceinline__ float block_reduce_sum(float x, float* red) {
 
 // One CTA per score row (b, h, i): m = max over the visible keys of scale * s_j,
 // Z = sum exp(scale * s_j - m), P_j = exp(scale * s_j - m) / Z rounded to the
-// input dtype (0 for keys the causal mask removes), LSE = m + ln Z.  The row is
-// read three times; the second and third reads hit the cache.
+// input dtype (0 for keys the causal mask removes), LSE = m + ln Z.  For rows
+// longer than the register-resident kernel below takes, the row is read three
+// times; the second and third reads hit the cache.
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads) softmax_rows_kernel(const float* __restrict__ S,
                                                                  uint16_t* __restrict__ P,
@@ -86,6 +87,68 @@ __global__ void __launch_bounds__(kThreads) softmax_rows_kernel(const float* __r
     }
   }
   if (lse != nullptr && threadIdx.x == 0) lse[row] = m + logf(z);
+}
+
+// The same for rows of at most kThreads * VPT keys, with the row held in
+// registers: S is read once and P written once.
+template <bool BF16, int VPT>
+__global__ void __launch_bounds__(kThreads) softmax_rows_reg_kernel(const float* __restrict__ S,
+                                                                     uint16_t* __restrict__ P,
+                                                                     float* __restrict__ lse, int Nq,
+                                                                     int Nk, float scale, int causal) {
+  __shared__ float red[kThreads / 32];
+  const long long row = blockIdx.x;
+  const int i = static_cast<int>(row % Nq);
+  const int nvis = causal ? min(Nk, i + 1) : Nk;
+  const float* s = S + row * Nk;
+  uint16_t* p = P + row * Nk;
+  float x[VPT];
+  float m = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int j = threadIdx.x + k * kThreads;
+    x[k] = j < nvis ? scale * s[j] : -INFINITY;
+    m = fmaxf(m, x[k]);
+  }
+  m = block_reduce_max(m, red);
+  float z = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    x[k] = expf(x[k] - m);  // 0 for the keys the mask removes
+    z += x[k];
+  }
+  z = block_reduce_sum(z, red);
+  const float inv = 1.f / z;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int j = threadIdx.x + k * kThreads;
+    if (j < Nk) {
+      const float pj = x[k] * inv;
+      if (BF16) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(pj);
+        p[j] = *reinterpret_cast<const uint16_t*>(&h);
+      } else {
+        const __half h = __float2half_rn(pj);
+        p[j] = *reinterpret_cast<const uint16_t*>(&h);
+      }
+    }
+  }
+  if (lse != nullptr && threadIdx.x == 0) lse[row] = m + logf(z);
+}
+
+template <bool BF16>
+void launch_softmax(const float* S, uint16_t* P, float* lse, int Nq, int Nk, float scale, int causal,
+                    unsigned rows, cudaStream_t st) {
+  if (Nk <= kThreads * 4)
+    softmax_rows_reg_kernel<BF16, 4><<<rows, kThreads, 0, st>>>(S, P, lse, Nq, Nk, scale, causal);
+  else if (Nk <= kThreads * 8)
+    softmax_rows_reg_kernel<BF16, 8><<<rows, kThreads, 0, st>>>(S, P, lse, Nq, Nk, scale, causal);
+  else if (Nk <= kThreads * 16)
+    softmax_rows_reg_kernel<BF16, 16><<<rows, kThreads, 0, st>>>(S, P, lse, Nq, Nk, scale, causal);
+  else if (Nk <= kThreads * 32)
+    softmax_rows_reg_kernel<BF16, 32><<<rows, kThreads, 0, st>>>(S, P, lse, Nq, Nk, scale, causal);
+  else
+    softmax_rows_kernel<BF16><<<rows, kThreads, 0, st>>>(S, P, lse, Nq, Nk, scale, causal);
 }
 
 }  // namespace fau
@@ -174,9 +237,9 @@ int fa_fwd_unfused(const void* q, const void* k, const void* v, void* o, float* 
   }
   const unsigned rows = static_cast<unsigned>(static_cast<long long>(B) * Hq * Nq);
   if (dtype == FA_BF16)
-    fau::softmax_rows_kernel<true><<<rows, fau::kThreads, 0, st>>>(S, P, lse, Nq, Nk, scale, causal);
+    fau::launch_softmax<true>(S, P, lse, Nq, Nk, scale, causal, rows, st);
   else
-    fau::softmax_rows_kernel<false><<<rows, fau::kThreads, 0, st>>>(S, P, lse, Nq, Nk, scale, causal);
+    fau::launch_softmax<false>(S, P, lse, Nq, Nk, scale, causal, rows, st);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   for (int r = 0; r < g; ++r) {
     if (cublasGemmStridedBatchedEx(h, CUBLAS_OP_N, CUBLAS_OP_N, D, Nq, Nk, &one, v, t16, D, nkd,
