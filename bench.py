@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward-pass measurement")
     ap.add_argument("--no-bias", action="store_true", help="skip the score-bias measurement")
+    ap.add_argument("--no-unfused", action="store_true",
+                    help="skip the unfused (standard attention) comparison")
     return ap.parse_args()
 
 
@@ -149,6 +151,7 @@ class ClockSampler:
         self.ok = False
         self.samples = []  # (time, mhz, reason bits)
         self.window = [None, None]
+        self.sections = []
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -175,6 +178,10 @@ class ClockSampler:
         """Mark the start (0) or end (1) of the timed region."""
         self.window[i] = time.perf_counter()
 
+    def section(self, name: str):
+        """Start a named section (it ends where the next one starts)."""
+        self.sections.append((name, time.perf_counter()))
+
     def __enter__(self):
         if self.ok:
             self.t = threading.Thread(target=self._run, daemon=True)
@@ -195,10 +202,17 @@ class ClockSampler:
             reasons |= {n for b, n in self.REASONS.items() if r & b}
         t0, t1 = self.window
         timed = [m for t, m, _ in busy if t0 is not None and t1 is not None and t0 <= t <= t1]
+        per_section = {}
+        bounds = self.sections + [("", float("inf"))]
+        for (name, a), (_, b) in zip(bounds[:-1], bounds[1:]):
+            xs = [m for t, m, _ in busy if a <= t < b]
+            if xs:
+                per_section[name] = statistics.median(xs)
         return {"sm_mhz": statistics.median(m for _, m, _ in busy), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(reasons), "samples": len(busy),
                 "timed_region_samples": len(timed),
                 "timed_region_sm_mhz": statistics.median(timed) if timed else None,
+                "sm_mhz_by_section": per_section,
                 "window": "warm-up through the per-workload lines (GPU busy)"}
 
 
@@ -361,6 +375,7 @@ def main():
            for _ in ws] for _ in range(K)]
     barrier()
     torch.cuda.synchronize()
+    clk.section("step")
     clk.mark(0)
     for i in range(K):
         for j in range(len(ws)):
@@ -382,6 +397,7 @@ def main():
                    "l2": "flushed before the pass"}
                   for j, w in enumerate(ws)}
 
+    clk.section("e2e")
     # ---- end to end through the public API: pinned host inputs -> device -> both
     # passes -> O and LSE back to pinned host memory, every step.  Copies in and
     # out run on their own streams with two device buffer sets, so the upload of
@@ -445,45 +461,7 @@ def main():
     assert fa.device_status(reset=True) == 0
     del dbuf, dout
 
-    # ---- every other workload the pages measure on, one line each (10 launches,
-    # L2 flushed before each; the median)
-    from fa_inputs import TINY, LONG, gqa, seq_sweep
-    configs = {}
-    if not args.no_configs:
-        cases = [("tiny B1 H1 N256 D64 fp16", TINY, None)]
-        for n in (512, 2048, 4096, 8192):
-            for causal in (False, True):
-                cases.append((f"sweep B1 H32 N{n} D128 fp16 {'causal' if causal else 'non-causal'}",
-                              seq_sweep(n, causal), None))
-        for hkv, d in ((8, 128), (1, 128), (8, 64), (8, 256)):
-            cases.append((f"gqa B4 Hq32 Hkv{hkv} N8192 D{d} bf16 causal", gqa(hkv, d), 11))
-        cases.append(("long B1 Hq32 Hkv8 N131072 D128 bf16 causal, 1% outlier keys", LONG, 12))
-        for name, w, dseed in cases:
-            if dseed is None:
-                cq, ck, cv = (x.to(dev) for x in make_qkv(w))
-            else:
-                cq, ck, cv = device_qkv(w, dev, dseed)
-            co = torch.empty_like(cq)
-            cl = torch.empty(cq.shape[:3], dtype=torch.float32, device=dev)
-            n_launch = 3 if w.Nq > 65536 else 10
-            ms = time_launches(lambda: fa.fa_fwd(cq, ck, cv, o=co, lse=cl, scale=w.softmax_scale,
-                                                 causal=w.causal, stream=sptr),
-                               flush, stream, n=n_launch, warm=2)
-            configs[name] = workload_line(w, ms, peak, hbm)
-            del cq, ck, cv, co, cl
-        configs["note"] = ("ms: median CUDA-event time of one launch, L2 flushed before each; "
-                           "alg_gbs: algorithmic bytes (read Q, K, V once, write O and LSE once) "
-                           "per second, frac_of_hbm against the measured copy bandwidth")
-        assert fa.device_status(reset=True) == 0
-    clk.__exit__(None, None, None)
-    gate = {}
-    for n in (4096, 8192):
-        for cz in ("non-causal", "causal"):
-            c = configs.get(f"sweep B1 H32 N{n} D128 fp16 {cz}")
-            if c:
-                gate[f"N{n}_{cz.replace('-', '')}"] = {"ms": c["ms"], "tflops": c["tflops"],
-                                                       "frac_of_peak": c["frac_of_peak"]}
-
+    clk.section("backward")
     # ---- backward pass on the bench workload (LLaMA-7B layer), both passes
     backward = {}
     if not args.no_backward:
@@ -505,6 +483,7 @@ def main():
         del bdo, bws, bdq, bdk, bdv
         assert fa.device_status(reset=True) == 0
 
+    clk.section("bias")
     # ---- additive score bias on the bench workload: one [N, N] bias shared by all heads
     bias_line = {}
     if not args.no_bias:
@@ -519,6 +498,7 @@ def main():
         del bb, bo, bl
         assert fa.device_status(reset=True) == 0
 
+    clk.section("window")
     # ---- sliding-window attention (causal, 1024-key window, 8192 positions, GQA 4)
     window = {}
     if not args.no_window:
@@ -539,6 +519,7 @@ def main():
         del wq, wk, wv, wo, wl_
         assert fa.device_status(reset=True) == 0
 
+    clk.section("decode")
     # ---- KV-cache decode (one query row per head, long cache, GQA 4): HBM-bound
     decode = {}
     if not args.no_decode:
@@ -574,6 +555,71 @@ def main():
             del dq, dk, dv, do_, dl_
         assert fa.device_status(reset=True) == 0
 
+    clk.section("unfused")
+    # ---- standard attention (the pages' comparison): S and P through device memory
+    unfused = {}
+    if not args.no_unfused:
+        uws = torch.empty(int(fa.load_library().fa_fwd_unfused_workspace_size(*q.shape[:3], k.shape[2])),
+                          dtype=torch.uint8, device=dev)
+        uo, ul = torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        for w in ws:
+            ms = time_launches(lambda: fa.fa_fwd_unfused(q, k, v, o=uo, lse=ul, scale=w.softmax_scale,
+                                                         causal=w.causal, stream=sptr,
+                                                         workspace=uws), flush, stream)
+            fused_ms = statistics.median(per_pass[ws.index(w)])
+            n_scores = w.B * w.Hq * w.Nq * w.Nk
+            unfused["causal" if w.causal else "non-causal"] = {
+                "ms": round(ms, 4), "tflops": round(w.flops() / (ms * 1e-3) / 1e12, 1),
+                "fused_ms": round(fused_ms, 4), "speedup_of_fused": round(ms / fused_ms, 2),
+                "alg_bytes": w.io_bytes() + 12 * n_scores,
+                "fused_alg_bytes": w.io_bytes()}
+        unfused["alg_bytes_note"] = ("unfused: Q, K, V, O, LSE once plus S written and read (fp32) and "
+                                     "P written and read (16-bit): 12 bytes per score; fused: none")
+        unfused["workspace_bytes"] = uws.numel()
+        del uws, uo, ul
+        assert fa.device_status(reset=True) == 0
+
+    clk.section("configs")
+    # ---- every other workload the pages measure on, one line each (10 launches,
+    # L2 flushed before each; the median).  Last: the long ones heat the GPU
+    # into its power cap, which would slow the lines measured after them.
+    from fa_inputs import TINY, LONG, gqa, seq_sweep
+    configs = {}
+    if not args.no_configs:
+        cases = [("tiny B1 H1 N256 D64 fp16", TINY, None)]
+        for n in (512, 2048, 4096, 8192):
+            for causal in (False, True):
+                cases.append((f"sweep B1 H32 N{n} D128 fp16 {'causal' if causal else 'non-causal'}",
+                              seq_sweep(n, causal), None))
+        for hkv, d in ((8, 128), (1, 128), (8, 64), (8, 256)):
+            cases.append((f"gqa B4 Hq32 Hkv{hkv} N8192 D{d} bf16 causal", gqa(hkv, d), 11))
+        cases.append(("long B1 Hq32 Hkv8 N131072 D128 bf16 causal, 1% outlier keys", LONG, 12))
+        for name, w, dseed in cases:
+            if dseed is None:
+                cq, ck, cv = (x.to(dev) for x in make_qkv(w))
+            else:
+                cq, ck, cv = device_qkv(w, dev, dseed)
+            co = torch.empty_like(cq)
+            cl = torch.empty(cq.shape[:3], dtype=torch.float32, device=dev)
+            n_launch = 3 if w.Nq > 65536 else 10
+            ms = time_launches(lambda: fa.fa_fwd(cq, ck, cv, o=co, lse=cl, scale=w.softmax_scale,
+                                                 causal=w.causal, stream=sptr),
+                               flush, stream, n=n_launch, warm=2)
+            configs[name] = workload_line(w, ms, peak, hbm)
+            del cq, ck, cv, co, cl
+        configs["note"] = ("ms: median CUDA-event time of one launch, L2 flushed before each; "
+                           "alg_gbs: algorithmic bytes (read Q, K, V once, write O and LSE once) "
+                           "per second, frac_of_hbm against the measured copy bandwidth")
+        assert fa.device_status(reset=True) == 0
+    gate = {}
+    for n in (4096, 8192):
+        for cz in ("non-causal", "causal"):
+            c = configs.get(f"sweep B1 H32 N{n} D128 fp16 {cz}")
+            if c:
+                gate[f"N{n}_{cz.replace('-', '')}"] = {"ms": c["ms"], "tflops": c["tflops"],
+                                                       "frac_of_peak": c["frac_of_peak"]}
+
+    clk.__exit__(None, None, None)
     launch_ms = total_ms / world / (K * len(ws)) if world > 1 else total_ms / (K * len(ws))
     achieved = (flops_step / len(ws)) / (launch_ms * 1e-3) / 1e12
     traffic = recorded_traffic()
@@ -603,6 +649,7 @@ def main():
         "gpu_launches": K * len(ws),
         "clocks": clk.summary(),
         "configs": configs,
+        "unfused": unfused,
         "gate_d128": gate,
         "decode": decode,
         "window": window,
