@@ -320,8 +320,10 @@ int fa_debug_exp2_fma(const float *x, float *y, int n, void *stream);
  */
 int fa_debug_wait_timeout(void *stream);
 
-/* Number of work tiles (CTAs' units of work) one fa_fwd call would schedule;
- * 0 for invalid arguments.  Host only; used to count launches and to size tests. */
+/* Number of 256-row work tiles (128-row at D = 256) of the two-query-tile
+ * kernel for these sizes; 0 for invalid arguments.  Host only; used to size
+ * tests.  (Launches with at most 128 query rows, key windows, or fewer of these
+ * tiles than half the CTAs run 128-row tiles instead.) */
 long long fa_fwd_num_tiles(int B, int Hq, int Nq, int D);
 
 #ifdef __cplusplus

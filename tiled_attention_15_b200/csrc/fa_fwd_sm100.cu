@@ -1095,6 +1095,9 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
           ++b_cnt;
           const uint32_t brow = (bias_mode & kBiasRowBcast) ? 0u : static_cast<uint32_t>(sub * 32 + lane);
           const uint32_t bbase = cx.sbase + G::OFF_BIAS + bs * G::BIAS_BYTES + brow * 128u;
+          // (pairs: one packed multiply-add per two keys; the key-range test only
+          // where some lane's row ends inside the block)
+          const bool all_visible = __all_sync(0xffffffffu, lim >= kBN);
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             uint32_t w[4];
@@ -1103,13 +1106,24 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
                          : "r"(bbase + (u >> 3) * (G::BIAS_BYTES / 2) +
                                ((static_cast<uint32_t>(u & 7) ^ (brow & 7u)) << 4)));
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int i = u * 8 + e;
-              const uint32_t h16 = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xffffu);
-              const float bv = BF16 ? __uint_as_float(h16 << 16)
-                                    : __half2float(__ushort_as_half(static_cast<unsigned short>(h16)));
-              sr[i] = __float_as_uint(i < lim ? fmaf(__uint_as_float(sr[i]), c, bv * kLog2e)
-                                              : -INFINITY);
+            for (int e = 0; e < 4; ++e) {
+              const int i = u * 8 + 2 * e;
+              F2 bv;
+              if (BF16) {
+                bv = unpack_bf16x2(w[e]);
+              } else {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+                bv = f2(f.x, f.y);
+              }
+              const F2 x = ffma2(f2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), f2(c, c),
+                                 fmul2(bv, f2(kLog2e, kLog2e)));
+              if (all_visible) {
+                sr[i] = __float_as_uint(x.x);
+                sr[i + 1] = __float_as_uint(x.y);
+              } else {
+                sr[i] = __float_as_uint(i < lim ? x.x : -INFINITY);
+                sr[i + 1] = __float_as_uint(i + 1 < lim ? x.y : -INFINITY);
+              }
             }
           }
           __syncwarp();
@@ -1316,10 +1330,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Registers: 168 per thread at launch (384 threads, one CTA per SM); the two
   // softmax warpgroups take kSoftmaxRegs, the MMA / TMA / idle warpgroup keeps
   // the rest (2 x 128 x 208 + 128 x 88 = 2 x 128 x 200 + 128 x 104 = 64512 =
-  // 384 x 168); bf16 needs the larger softmax share (it also sums rounded P).
+  // 384 x 168). The two-query-tile kernel's MMA, TMA and bias-producer code
+  // needs the 104 of the second split (with 88 it spills in its loops); bf16
+  // with one query tile or a key window takes the first split, whose softmax
+  // sums rounded P in registers that 200 do not hold without spilling.
   // The wait helpers are inlined: ptxas cannot allocate a call inside a region
   // resized this way.
-  constexpr int kSoftmaxRegs = BF16 ? 208 : 200;
+  constexpr int kSoftmaxRegs = (BF16 && (NQ == 1 || WIN)) ? 208 : 200;
   constexpr int kOtherRegs = (384 * 168 - 256 * kSoftmaxRegs) / 128;
   if (warp < 8) setmaxnreg_inc<kSoftmaxRegs>();
   else setmaxnreg_dec<kOtherRegs>();
@@ -1754,8 +1771,14 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
     return bf ? launch<128, 2, true, false, true>(FA_WARGS) : launch<128, 2, false, false, true>(FA_WARGS);
 #undef FA_WARGS
   }
-  const bool one_tile =
-      windowed || (pack_heads(Hq, Hkv, Nq, causal) ? (Hq / Hkv) * Nq : Nq) <= fa::kBM;
+  // ... and so does a problem too small to give half of the CTAs a 256-row
+  // tile: 128-row tiles double the CTAs that take part (short sequences).
+  const long long tiles2 = (long long)B * Hq * ((Nq + 2 * fa::kBM - 1) / (2 * fa::kBM));
+  const int cap = g_max_ctas.load();
+  const int ctas = (cap > 0 && cap < ds.sms) ? cap : ds.sms;
+  const bool one_tile = windowed ||
+                        (pack_heads(Hq, Hkv, Nq, causal) ? (Hq / Hkv) * Nq : Nq) <= fa::kBM ||
+                        2 * tiles2 < ctas;
 #define FA_ARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, wl, wr, st, dev, ws, ws_bytes, mode
   switch (D) {
     case 64:
