@@ -171,6 +171,23 @@ int fa_fwd_bias(const void *q, const void *k, const void *v, void *o, float *lse
                 void *stream, int dtype);
 
 /*
+ * fa_fwd_bias with a key window as well (both masks of the mask step at once):
+ * key j is visible to query i iff i - window_left <= j <= i + window_right
+ * (-1: no bound; causal = 1 adds j <= i) and its bias is not -inf; the visible
+ * scores get the bias added as in fa_fwd_bias.  A row with no visible key gets
+ * O = 0 and LSE = -inf.  Windowed calls run the 128-row-tile kernel, which
+ * takes each tile's own key-block range.  Arguments, layout and errors as
+ * fa_fwd_bias and fa_fwd_window (FA_ERR_BAD_WINDOW for a bound < -1, or
+ * window_right > 0 with causal = 1); window_left = window_right = -1 is
+ * fa_fwd_bias.
+ */
+int fa_fwd_bias_window(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                       int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
+                       const void *bias, long long bias_stride_b, long long bias_stride_h,
+                       long long bias_stride_q, int window_left, int window_right, void *stream,
+                       int dtype);
+
+/*
  * Backward pass: the gradients of the attention above for an upstream gradient
  * dout (the pages mention only that training keeps gradients -- hwcomputing.
  * csdn.net page, section on standard attention; the operation is taken as the
@@ -188,10 +205,13 @@ int fa_fwd_bias(const void *q, const void *k, const void *v, void *o, float *lse
  *               bytes, 256-byte aligned, caller-owned (Delta and lse * log2 e,
  *               padded to 128-row blocks; no zero-fill needed); else
  *               FA_ERR_BAD_WORKSPACE / FA_ERR_MISALIGNED.
- * D must be 64 or 128 (else FA_ERR_UNSUPPORTED_HEAD_DIM).  Outputs and the
- * workspace may not overlap any input or each other (FA_ERR_OVERLAP).  Three
- * kernels on `stream` (Delta, dK and dV, dQ); asynchronous; deterministic (no
- * atomics).  Other errors as fa_fwd.
+ * D must be 64, 128 or 256 (else FA_ERR_UNSUPPORTED_HEAD_DIM).  Outputs and
+ * the workspace may not overlap any input or each other (FA_ERR_OVERLAP).
+ * Kernels on `stream`: Delta, then dK and dV, then dQ (at D = 256 dV and dK
+ * are two launches over 64-row query blocks, and dQ runs over 64-key blocks:
+ * one CTA's tensor memory holds only one 256-column accumulator next to the
+ * score blocks); asynchronous; deterministic (no atomics).  Other errors as
+ * fa_fwd.
  */
 int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
            const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk,

@@ -171,6 +171,21 @@ def test_bias_entry_point_host_checks(lib):
 
 
 
+def test_bias_window_entry_point_host_checks(lib):
+    import torch
+    a = dict(GOOD)
+
+    def call(wl=-1, wr=-1, causal=0, bias=9 * A):
+        return lib.fa_fwd_bias_window(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"],
+                                      a["Hkv"], a["Nq"], a["Nk"], a["D"], ctypes.c_float(a["scale"]),
+                                      causal, bias, 0, 0, 64, wl, wr, None, a["dtype"])
+    assert call(bias=None) == 1
+    assert call(wl=-2) == 14 and call(wr=-3) == 14 and call(wl=4, wr=2, causal=1) == 14
+    if not torch.cuda.is_available():
+        for wl, wr, causal in ((-1, -1, 0), (16, -1, 1), (3, 7, 0), (0, 0, 0)):
+            assert call(wl, wr, causal) == 8  # valid: reaches the device check
+
+
 def test_bwd_window_host_checks(lib):
     a = dict(GOOD)
 
@@ -220,7 +235,7 @@ def test_bwd_host_checks(lib):
         return lib.fa_bwd(a["q"], a["k"], a["v"], 6 * A, 7 * A, lse, dq, 10 * A, 11 * A, a["B"],
                           a["Hq"], a["Hkv"], a["Nq"], a["Nk"], D, ctypes.c_float(a["scale"]), 0,
                           None, dtype, ws, ws_bytes)
-    assert call(D=256) == 5              # backward: head_dim 64 or 128
+    assert call(D=96) == 5               # backward: head_dim 64, 128 or 256
     assert call(dtype=3) == 7
     assert call(ws=None) == fa.FA_ERR_BAD_WORKSPACE
     assert call(ws_bytes=16) == fa.FA_ERR_BAD_WORKSPACE

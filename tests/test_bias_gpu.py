@@ -29,13 +29,14 @@ def _bias(w, shape, seed, scale=2.0, neg_inf_frac=0.0):
     return torch.from_numpy(b).to(TD[w.dtype])
 
 
-def _check(w, bias, dev, tag=""):
+def _check(w, bias, dev, tag="", window=(-1, -1)):
     q, k, v = make_qkv(w)
     o, lse = fa.fa_fwd(q.to(dev), k.to(dev), v.to(dev), scale=w.softmax_scale, causal=w.causal,
-                       bias=bias.to(dev))
+                       bias=bias.to(dev), window=window)
     torch.cuda.synchronize()
     assert fa.device_status(reset=True) == 0
-    ref_o, ref_l = oracle.attention(q, k, v, w.softmax_scale, w.causal, bias=bias.float())
+    ref_o, ref_l = oracle.attention(q, k, v, w.softmax_scale, w.causal, bias=bias.float(),
+                                    window=window)
     got_o, got_l = o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy()
     empty = np.isneginf(ref_l)
     np.testing.assert_array_equal(np.isneginf(got_l), empty)
@@ -120,3 +121,38 @@ def test_bias_many_tiles_per_cta(cuda_dev):
         _check(wc, _bias(wc, (1, 8, 1024, 1024), 8), cuda_dev)
     finally:
         fa.set_max_ctas(prev)
+
+
+# ---- key window and score bias in one call (fa_fwd_bias_window)
+
+def test_window_and_bias_causal_sliding(cuda_dev):
+    # causal sliding window of 200 keys over three 128-row tiles and a ragged tail,
+    # with a full [B, H, Nq, Nk] bias
+    w = Workload("window 200 causal + full bias D128 fp16", 1, 4, 2, 600, 600, 128, "fp16", True,
+                 seed=121)
+    _check(w, _bias(w, (1, 4, 600, 600), 9), cuda_dev, " window", window=(200, -1))
+
+
+def test_window_and_bias_two_sided_padding_mask(cuda_dev):
+    # two-sided window (37 left, 19 right) with a key-padding mask of -inf and
+    # per-key values, broadcast over heads and queries
+    w = Workload("window 37/19 + padding mask D64 bf16", 2, 4, 4, 300, 320, 64, "bf16", False,
+                 seed=122)
+    b = _bias(w, (2, 1, 1, 320), 10, neg_inf_frac=0.2)
+    _check(w, b, cuda_dev, " window", window=(37, 19))
+
+
+def test_window_and_bias_rows_without_keys(cuda_dev):
+    # window (0, 0): query i sees key i only; rows i >= Nk see nothing, and a
+    # bias of -inf on some keys empties their rows too: O = 0, LSE = -inf there
+    w = Workload("window 0/0 + -inf bias D128 fp16", 1, 2, 2, 260, 200, 128, "fp16", False,
+                 seed=123)
+    b = _bias(w, (1, 2, 260, 200), 11, neg_inf_frac=0.3)
+    o, lse = _check(w, b, cuda_dev, " window", window=(0, 0))
+    assert torch.isneginf(lse[:, :, 200:]).all()
+
+
+def test_window_and_bias_d256_per_head(cuda_dev):
+    w = Workload("window 96 causal + per-head bias D256 bf16", 1, 4, 1, 400, 400, 256, "bf16",
+                 True, seed=124)
+    _check(w, _bias(w, (1, 4, 400, 400), 12), cuda_dev, " window", window=(96, -1))

@@ -84,6 +84,11 @@ CASES = [
     Workload("bwd D64 fp16 odd sizes", 2, 3, 3, 129, 255, 64, "fp16", False, seed=97),
     Workload("bwd D128 fp16 N2048 causal", 1, 4, 4, 2048, 2048, 128, "fp16", True, seed=98),
     Workload("bwd D128 bf16 N2048", 1, 4, 4, 2048, 2048, 128, "bf16", False, seed=99),
+    # head_dim 256: 64-row streamed blocks, dV and dK from separate launches
+    Workload("bwd D256 fp16 ragged", 1, 2, 2, 300, 333, 256, "fp16", False, seed=141),
+    Workload("bwd D256 bf16 causal GQA 4", 1, 8, 2, 520, 520, 256, "bf16", True, seed=142),
+    Workload("bwd D256 fp16 causal Nk>Nq", 2, 2, 1, 200, 700, 256, "fp16", True, seed=143),
+    Workload("bwd D256 bf16 N1024", 1, 4, 4, 1024, 1024, 256, "bf16", False, seed=144),
 ]
 
 
@@ -121,6 +126,8 @@ WINDOW_CASES = [
     (Workload("bwd empty rows D64 fp16", 1, 2, 2, 700, 300, 64, "fp16", False, seed=134), (110, 10)),
     (Workload("bwd right only 64 D128 bf16 GQA", 1, 4, 2, 500, 600, 128, "bf16", False, seed=135), (-1, 64)),
     (Workload("bwd causal window 128 D128 fp16 Nk>Nq", 1, 2, 2, 300, 900, 128, "fp16", True, seed=136), (128, 0)),
+    (Workload("bwd local 70/30 D256 bf16", 1, 2, 2, 400, 400, 256, "bf16", False, seed=137), (70, 30)),
+    (Workload("bwd empty rows D256 fp16", 1, 2, 1, 500, 200, 256, "fp16", False, seed=138), (40, 5)),
 ]
 
 

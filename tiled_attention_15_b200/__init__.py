@@ -26,7 +26,7 @@ FA_ERR_BAD_WORKSPACE = 15
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
-            "fa_fwd_window", "fa_fwd_bias", "fa_bwd", "fa_bwd_window",
+            "fa_fwd_window", "fa_fwd_bias", "fa_fwd_bias_window", "fa_bwd", "fa_bwd_window",
             "fa_bwd_workspace_size",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
             "fa_fwd_unfused", "fa_fwd_unfused_workspace_size",
@@ -66,6 +66,8 @@ def load_library() -> ctypes.CDLL:
     ll = ctypes.c_longlong
     lib.fa_fwd_bias.argtypes = fwd_args[:13] + [vp, ll, ll, ll, vp, i]
     lib.fa_fwd_bias.restype = i
+    lib.fa_fwd_bias_window.argtypes = fwd_args[:13] + [vp, ll, ll, ll, i, i, vp, i]
+    lib.fa_fwd_bias_window.restype = i
     lib.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, vp, i, vp, ctypes.c_size_t]
     lib.fa_bwd.restype = i
     lib.fa_bwd_window.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, i, i, vp, i, vp, ctypes.c_size_t]
@@ -181,7 +183,8 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
     per-(device, stream) workspace (load balance), else fa_fwd.  window:
     (left, right) key window, -1 = unbounded (fa_fwd_window when either is set).
     bias: additive score bias (fa_fwd_bias), a CUDA tensor of q's dtype that
-    broadcasts to [B, Hq, Nq, Nk] (size-1 dims broadcast).
+    broadcasts to [B, Hq, Nq, Nk] (size-1 dims broadcast); with a window as
+    well, fa_fwd_bias_window.
     Returns (o, lse or None).
     """
     import torch
@@ -216,9 +219,13 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
             ctypes.c_float(scale), 1 if causal else 0, stream or None, dtype)
     wl, wr = (int(x) for x in window)
     if bias is not None:
-        if (wl, wr) != (-1, -1):
-            raise ValueError("a bias and a key window cannot be combined")
         bt, sb, sh, sq = _bias_view(bias, q.dtype, B, Hq, Nq, Nk)
+        if (wl, wr) != (-1, -1):
+            rc = lib.fa_fwd_bias_window(*args[:13], bt.data_ptr(), sb, sh, sq, wl, wr, args[13],
+                                        dtype)
+            if rc != FA_OK:
+                raise FaError(rc, "fa_fwd_bias_window")
+            return o, lse
         rc = lib.fa_fwd_bias(*args[:13], bt.data_ptr(), sb, sh, sq, args[13], dtype)
         if rc != FA_OK:
             raise FaError(rc, "fa_fwd_bias")
@@ -282,7 +289,7 @@ def fa_bwd(q, k, v, o, lse, dout, scale: Optional[float] = None, causal: bool = 
 
     q, o, dout: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] contiguous CUDA tensors of
     one dtype (fp16 or bf16); lse: float32 [B, Hq, Nq] from fa_fwd.  D must be
-    64 or 128.  Optional outputs dq (like q), dk, dv (like k); optional
+    64, 128 or 256.  Optional outputs dq (like q), dk, dv (like k); optional
     workspace: a uint8 CUDA tensor of at least fa_bwd_workspace_size bytes
     (allocated here when None).  window: (left, right) key window of the
     forward pass (fa_bwd_window), -1 = unbounded.  Returns (dq, dk, dv).

@@ -25,6 +25,8 @@
 // dQ is computed in its own pass (S and dP recomputed: two extra MMAs per block
 // pair) instead of being accumulated across key tiles with atomics: no atomic
 // traffic, and the result does not depend on the order CTAs finish in.
+// Head dimension 256 has its own three kernels (end of the device code): the
+// streamed operand in 64-row blocks, and dV and dK from separate launches.
 //
 // Warp roles (384 threads, one CTA per SM): warps 0-7 two compute warpgroups
 // that split each block's 128 columns into halves (warp w reads TMEM lanes
@@ -229,7 +231,8 @@ struct KVTile {
   int nb;   // blocks: group heads x query blocks
 };
 
-__device__ __forceinline__ KVTile kv_tile(const BwdParams& p) {
+// bq: rows of a query block (128, or 64 at head_dim 256)
+__device__ __forceinline__ KVTile kv_tile(const BwdParams& p, int bq = kBM) {
   KVTile T;
   const int BK = p.B * p.Hkv;
   const int t = blockIdx.x;
@@ -242,9 +245,9 @@ __device__ __forceinline__ KVTile kv_tile(const BwdParams& p) {
   }
   // query blocks that see a key of this tile: q >= k0 - wr and q <= k0 + 127 + wl
   // (causal: wr = 0, so from the diagonal block on; top-left aligned)
-  const int k0 = T.kt * kBN;
-  T.i0 = p.wr >= 0 ? max(0, k0 - p.wr) / kBM : 0;
-  const int i1 = p.wl >= 0 ? min(p.nqt - 1, (k0 + kBN - 1 + p.wl) / kBM) : p.nqt - 1;
+  const int k0 = T.kt * kBN, nqblk = p.Nq_pad / bq;
+  T.i0 = p.wr >= 0 ? max(0, k0 - p.wr) / bq : 0;
+  const int i1 = p.wl >= 0 ? min(nqblk - 1, (k0 + kBN - 1 + p.wl) / bq) : nqblk - 1;
   T.nqb = i1 >= T.i0 ? i1 - T.i0 + 1 : 0;
   T.nb = p.group * T.nqb;
   return T;
@@ -733,6 +736,536 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+
+// ================================================================== head_dim 256
+// At D = 256 one CTA cannot keep what the kernels above keep on chip: dK and
+// dV alone fill the 512 tensor-memory columns, and 128-row K, V, Q and dO
+// tiles are 64 KB each.  So here
+//   * the streamed operand comes in blocks of 64 rows (query blocks in the
+//     key-tile kernels, key blocks in the dQ kernel), 32 KB each;
+//   * dV and dK come from two launches of one key-tile kernel, each with a
+//     single 256-column accumulator:
+//       DK = false:  S^T = K Q^T, P^T, dV += P^T dO
+//       DK = true:   S^T = K Q^T, dP^T = V dO^T, dS^T, dK += dS^T Q
+//     (S^T is formed in both: one extra MMA group per block pair);
+//   * bwd_dq256_kernel: S = Q K^T, dP = dO V^T, dS, dQ += dS K.
+// The blocks stream through two sets of slots: one for the operand held until
+// the block's last MMA (Q in the key-tile kernels, K in dQ), one for the
+// operand released early (dO after dP^T or dV; V after dP).
+constexpr int kBS = 64;  // rows of a streamed block at head_dim 256
+
+// Accumulating MMA over KSTEPS steps of 16 along K, A (16-bit) in tensor
+// memory at column acol(kk), B an MN-major SW128 block (16 rows of K per step).
+template <int KSTEPS, typename ACol>
+__device__ __forceinline__ void mma_tn_steps(uint32_t d, uint32_t a, uint64_t b0, uint32_t idesc,
+                                             bool acc, ACol acol) {
+#pragma unroll
+  for (int kk = 0; kk < KSTEPS; ++kk)
+    mma_ts(d, a + acol(kk), b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+           (acc || kk > 0) ? 1u : 0u);
+}
+
+struct Geo256 {
+  static constexpr int CH_R = 128 * 128;   // one 64-column chunk of a 128-row tile
+  static constexpr int CH_S = kBS * 128;   // one 64-column chunk of a 64-row block
+  static constexpr int TILE_R = 4 * CH_R;  // 64 KB
+  static constexpr int TILE_S = 4 * CH_S;  // 32 KB
+};
+
+template <bool DK>
+struct Geo256KV : Geo256 {
+  // slot sets: NA for Q blocks (with their lse2 and delta), NB for dO blocks;
+  // item m is Q_{m/2} (even) or dO_{m/2} (odd)
+  static constexpr int NA = DK ? 2 : 3, NB = DK ? 1 : 2, NSLOT = NA + NB;
+  __device__ static int slot(int m) { return (m & 1) ? NA + (m >> 1) % NB : (m >> 1) % NA; }
+  __device__ static int use(int m) { return (m & 1) ? (m >> 1) / NB : (m >> 1) / NA; }
+  static constexpr int OFF_K = 0, OFF_V = TILE_R, OFF_SL = DK ? 2 * TILE_R : TILE_R;
+  static constexpr int OFF_SIDE = OFF_SL + NSLOT * TILE_S;  // per Q slot: lse2[64], delta[64]
+  static constexpr int OFF_BAR = OFF_SIDE + NA * 512;
+  static constexpr int B_KV = 0, B_SLF = 1, B_SLE = 1 + NSLOT, B_SF = 1 + 2 * NSLOT,
+                       B_DPF = B_SF + 1, B_PF = B_SF + 2, B_ACC = B_SF + 3, NBAR = B_SF + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // TMEM columns: S^T 0..63 (P^T packed over it), dP^T 64..127 (dS^T packed
+  // over it), the accumulator (dV or dK) 256..511
+  static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_ACC = 256;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <bool BF16, bool DK>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kv256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const BwdParams p) {
+  using G = Geo256KV<DK>;
+  constexpr int D = 256;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(gbase + G::OFF_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Ctx cx;
+  cx.sbase = sbase;
+  cx.abort_flag = misc + 1;
+  auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
+  const KVTile T = kv_tile(p, kBS);
+
+  if (threadIdx.x == 0) {
+    mbar_init(B(G::B_KV), 1);
+    for (int s = 0; s < G::NSLOT; ++s) {
+      mbar_init(B(G::B_SLF + s), 1);
+      mbar_init(B(G::B_SLE + s), 1);
+    }
+    mbar_init(B(G::B_SF), 1);
+    mbar_init(B(G::B_DPF), 1);
+    mbar_init(B(G::B_PF), 8);
+    mbar_init(B(G::B_ACC), 1);
+    misc[1] = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(misc), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cx.tmem = misc[0];
+
+  // Registers: 176 for the compute warpgroups (32 scores a thread per block),
+  // 152 for the rest, whose MMA groups run 16 steps of K (2 x 128 x 176 +
+  // 128 x 152 = 384 x 168).
+  const int kv_row0 = T.kt * kBN;
+  const int nqb = T.nqb;
+  if (warp >= 8) setmaxnreg_dec<152>();
+  if (warp == 9 && lane == 0 && T.nb > 0) {
+    // ---- TMA: K (and V) once, then (Q + lse2 [+ delta], dO) per 64-row query block
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_do);
+    const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
+    mbar_arrive_expect_tx(B(G::B_KV), (DK ? 2 : 1) * G::TILE_R);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      tma_load_3d(sbase + G::OFF_K + c * G::CH_R, &tm_k, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
+      if (DK)
+        tma_load_3d(sbase + G::OFF_V + c * G::CH_R, &tm_v, B(G::B_KV), c * 64, kv_row0, T.bkv,
+                    pol_first);
+    }
+    for (int m = 0; m < 2 * T.nb; ++m) {
+      const int sl = G::slot(m), u = G::use(m), n = m >> 1;
+      if (u > 0 && !wait_bar(B(G::B_SLE + sl), (u - 1) & 1u, cx.abort_flag)) break;
+      const int h = n / nqb, i = T.i0 + n % nqb;
+      const int bh = (T.bkv / p.Hkv) * p.Hq + (T.bkv % p.Hkv) * p.group + h;
+      const bool is_q = (m & 1) == 0;
+      mbar_arrive_expect_tx(B(G::B_SLF + sl), G::TILE_S + (is_q ? (DK ? 512 : 256) : 0));
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tma_load_3d(sbase + G::OFF_SL + sl * G::TILE_S + c * G::CH_S, is_q ? &tm_q : &tm_do,
+                    B(G::B_SLF + sl), c * 64, i * kBS, bh, pol_last);
+      if (is_q) {
+        const size_t row = static_cast<size_t>(bh) * p.Nq_pad + static_cast<size_t>(i) * kBS;
+        const uint32_t side = sbase + G::OFF_SIDE + sl * 512;
+        bulk_load(side, p.lse2 + row, 256, B(G::B_SLF + sl));
+        if (DK) bulk_load(side + 256, p.delta + row, 256, B(G::B_SLF + sl));
+      }
+    }
+  } else if (warp == 8 && lane == 0 && T.nb > 0) {
+    // ---- MMA.  dV: S^T(0) | dV(n) S^T(n+1) | ...;  dK: S^T(0) dP^T(0) | dK(n) S^T(n+1) dP^T(n+1) | ...
+    constexpr uint32_t kIdNT = idesc_f16(128, kBS, BF16, false);
+    constexpr uint32_t kIdTN = idesc_f16(128, D, BF16, true);
+    const uint32_t tm = cx.tmem;
+    const uint64_t dk0 = sdesc_sw128(sbase + G::OFF_K, 16, 1024);
+    const uint64_t dv0 = sdesc_sw128(sbase + G::OFF_V, 16, 1024);
+    auto st_desc = [&](int m, bool mn) {
+      const uint32_t a = sbase + G::OFF_SL + G::slot(m) * G::TILE_S;
+      return mn ? sdesc_sw128(a, G::CH_S, 1024) : sdesc_sw128(a, 16, 1024);
+    };
+    auto wait_item = [&](int m) {
+      return wait_bar(B(G::B_SLF + G::slot(m)), G::use(m) & 1u, cx.abort_flag);
+    };
+    // P^T / dS^T of query column x: warpgroup x / 32 packed its 32 columns into
+    // its own first 16 -> K step kk (16 queries) at (kk / 2) * 32 + (kk % 2) * 8
+    auto acol = [](int kk) { return static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8); };
+    auto issue_s = [&](int n) {  // S^T(n), and dP^T(n) for dK (dO_n's slot is then free)
+      mma_nt<D>(tm + G::TM_S, dk0, st_desc(2 * n, false), kIdNT, G::CH_R, G::CH_S);
+      mma_commit(B(G::B_SF));
+      if (DK) {
+        mma_nt<D>(tm + G::TM_DP, dv0, st_desc(2 * n + 1, false), kIdNT, G::CH_R, G::CH_S);
+        mma_commit(B(G::B_DPF));
+        mma_commit(B(G::B_SLE + G::slot(2 * n + 1)));
+      }
+    };
+    bool ok = wait_bar(B(G::B_KV), 0u, cx.abort_flag) && wait_item(0) && (!DK || wait_item(1));
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+    }
+    for (int n = 0; ok && n < T.nb; ++n) {
+      if (!wait_bar(B(G::B_PF), n & 1u, cx.abort_flag)) break;
+      if (!DK && !wait_item(2 * n + 1)) break;
+      tc_fence_after();
+      if (DK) {  // dK += dS^T Q_n
+        mma_tn_steps<kBS / 16>(tm + G::TM_ACC, tm + G::TM_DP, st_desc(2 * n, true), kIdTN, n > 0, acol);
+      } else {  // dV += P^T dO_n
+        mma_tn_steps<kBS / 16>(tm + G::TM_ACC, tm + G::TM_S, st_desc(2 * n + 1, true), kIdTN, n > 0, acol);
+        mma_commit(B(G::B_SLE + G::slot(2 * n + 1)));
+      }
+      mma_commit(B(G::B_SLE + G::slot(2 * n)));  // Q_n's slot (and its lse2, delta)
+      if (n + 1 < T.nb) {
+        if (!wait_item(2 * n + 2) || (DK && !wait_item(2 * n + 3))) break;
+        tc_fence_after();
+        issue_s(n + 1);
+      } else {
+        mma_commit(B(G::B_ACC));
+      }
+    }
+  } else if (warp < 8) {
+    // ---- compute: thread = key row r of the tile, warpgroup h = query columns h*32 .. +31
+    setmaxnreg_inc<176>();
+    const int h = warp >> 2, r = (warp & 3) * 32 + lane;
+    const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const float c = p.c;
+    bool ok = true;
+    for (int n = 0; ok && n < T.nb; ++n) {
+      const int sl = G::slot(2 * n);  // the slot of Q_n, with lse2 and delta
+      const int i = T.i0 + n % nqb;
+      // lse2 / delta of this block were written by the TMA unit: observe its barrier
+      ok = wait_bar(B(G::B_SLF + sl), G::use(2 * n) & 1u, cx.abort_flag) &&
+           wait_bar(B(G::B_SF), n & 1u, cx.abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const float* l2 = reinterpret_cast<const float*>(gbase + G::OFF_SIDE + sl * 512) + h * 32;
+      const float* dl = l2 + 64;
+      uint32_t sr[32];
+      tmem_ld_x32(tm + G::TM_S + h * 32, sr);
+      // visible query columns of this key row: [lo_c, lo_c + span) -- key k0 + r
+      // is seen by query q0 + col iff k0 + r <= q0 + col + wr and k0 + r >= q0 + col - wl
+      const int q0 = i * kBS;
+      const int dqk = kv_row0 + r - q0;
+      const bool msk = (p.wr >= 0 && kv_row0 + kBN - 1 - p.wr > q0) ||
+                       (p.wl >= 0 && kv_row0 + p.wl < q0 + kBS - 1);
+      const int lo_c = p.wr >= 0 ? dqk - p.wr : -kBN;
+      const int hi_c = p.wl >= 0 ? dqk + p.wl : kBN + kBS;
+      const uint32_t span = static_cast<uint32_t>(max(hi_c - lo_c + 1, 0));
+      float pv[32];
+#pragma unroll
+      for (int x = 0; x < 32; x += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(l2 + x);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float e2 = ex2(fmaf(__uint_as_float(sr[x + e]), c, -lv[e]));
+          pv[x + e] = (msk && static_cast<uint32_t>(h * 32 + x + e - lo_c) >= span) ? 0.f : e2;
+        }
+      }
+      uint32_t pk[16];
+      if (DK) {  // dS^T = P^T (dP^T - Delta), over dP^T
+        ok = wait_bar(B(G::B_DPF), n & 1u, cx.abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+        uint32_t dr[32];
+        tmem_ld_x32(tm + G::TM_DP + h * 32, dr);
+#pragma unroll
+        for (int x = 0; x < 32; x += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(dl + x);
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pv[x + e] *= __uint_as_float(dr[x + e]) - dv4[e];
+        }
+#pragma unroll
+        for (int x = 0; x < 16; ++x) pk[x] = pack2(pv[2 * x], pv[2 * x + 1], BF16);
+        tmem_st_x16(tm + G::TM_DP + h * 32, pk);
+      } else {  // P^T, over S^T
+#pragma unroll
+        for (int x = 0; x < 16; ++x) pk[x] = pack2(pv[2 * x], pv[2 * x + 1], BF16);
+        tmem_st_x16(tm + G::TM_S + h * 32, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_PF));
+    }
+    // ---- epilogue: warpgroup h writes columns h*128 .. +127 of dV, or of dK (times scale)
+    const int key = kv_row0 + r;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(DK ? p.dk : p.dv) +
+                    (static_cast<size_t>(T.bkv) * p.Nk + (key < p.Nk ? key : 0)) * D;
+    const float mul = DK ? p.scale : 1.f;
+    if (T.nb == 0) {  // no query sees these keys: zero gradients
+      if (key < p.Nk)
+        for (int c0 = h * 128; c0 < (h + 1) * 128; c0 += 8)
+          *reinterpret_cast<uint4*>(dst + c0) = make_uint4(0, 0, 0, 0);
+    } else if (ok) {
+      ok = wait_bar(B(G::B_ACC), 0u, cx.abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = h * 128; c0 < (h + 1) * 128; c0 += 32) {
+          uint32_t a[32];
+          tmem_ld_x32(tm + G::TM_ACC + c0, a);
+          uint32_t w[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            w[x] = pack2(__uint_as_float(a[2 * x]) * mul, __uint_as_float(a[2 * x + 1]) * mul, BF16);
+          if (key < p.Nk) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*cx.abort_flag) {  // let issued copies and MMAs land before tensor memory is freed
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) {
+    }
+  }
+  if (threadIdx.x == 0) publish_abort(*cx.abort_flag);
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(cx.tmem, 512);
+  }
+}
+
+struct Geo256Q : Geo256 {
+  // slot sets: NA for K blocks (held until dQ), NB for V blocks (free after dP);
+  // item m is K_{m/2} (even) or V_{m/2} (odd)
+  static constexpr int NA = 2, NB = 1, NSLOT = NA + NB;
+  __device__ static int slot(int m) { return (m & 1) ? NA + (m >> 1) % NB : (m >> 1) % NA; }
+  __device__ static int use(int m) { return (m & 1) ? (m >> 1) / NB : (m >> 1) / NA; }
+  static constexpr int OFF_Q = 0, OFF_DO = TILE_R, OFF_SL = 2 * TILE_R;
+  static constexpr int OFF_BAR = OFF_SL + NSLOT * TILE_S;
+  static constexpr int B_QF = 0, B_SLF = 1, B_SLE = 1 + NSLOT, B_SDP = 1 + 2 * NSLOT,
+                       B_SFREE = B_SDP + 1, B_DSF = B_SDP + 2, B_DSE = B_SDP + 3, B_DQF = B_SDP + 4,
+                       NBAR = B_SDP + 5;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // TMEM columns: S 0..63, dP 64..127, dS (packed) 128..159, dQ 256..511
+  static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_DS = 128, TM_DQ = 256;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const BwdParams p) {
+  using G = Geo256Q;
+  constexpr int D = 256;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(gbase + G::OFF_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Ctx cx;
+  cx.sbase = sbase;
+  cx.abort_flag = misc + 1;
+  auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
+
+  // tile: (b, hq, 128-row query block); causal: the last query blocks (most keys) first
+  const int BH = p.B * p.Hq, t = blockIdx.x;
+  int bh, qt;
+  if (p.causal) {
+    qt = p.nqt - 1 - t / BH;
+    bh = t % BH;
+  } else {
+    bh = t / p.nqt;
+    qt = t % p.nqt;
+  }
+  const int q0 = qt * kBM;
+  const int kvz = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
+  const int nkb = (p.Nk + kBS - 1) / kBS;
+  // 64-key blocks this tile's rows see: keys q - wl .. q + wr (causal: wr = 0)
+  const int qlast = min(q0 + kBM, p.Nq) - 1;
+  const int jb0 = p.wl >= 0 ? min(max(0, q0 - p.wl) / kBS, nkb) : 0;
+  const int jb1 = p.wr >= 0 ? min(nkb - 1, (qlast + p.wr) / kBS) : nkb - 1;
+  const int nb = jb1 >= jb0 ? jb1 - jb0 + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(B(G::B_QF), 1);
+    for (int s = 0; s < G::NSLOT; ++s) {
+      mbar_init(B(G::B_SLF + s), 1);
+      mbar_init(B(G::B_SLE + s), 1);
+    }
+    mbar_init(B(G::B_SDP), 1);
+    mbar_init(B(G::B_SFREE), 8);
+    mbar_init(B(G::B_DSF), 8);
+    mbar_init(B(G::B_DSE), 1);
+    mbar_init(B(G::B_DQF), 1);
+    misc[1] = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(misc), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cx.tmem = misc[0];
+
+  // Registers: as in bwd_kv256_kernel (176 / 152).
+  if (warp >= 8) setmaxnreg_dec<152>();
+  if (warp == 9 && lane == 0 && nb > 0) {
+    // ---- TMA: Q and dO once, then (K_j, V_j) per 64-key block
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
+    mbar_arrive_expect_tx(B(G::B_QF), 2 * G::TILE_R);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      tma_load_3d(sbase + G::OFF_Q + c * G::CH_R, &tm_q, B(G::B_QF), c * 64, q0, bh, pol_first);
+      tma_load_3d(sbase + G::OFF_DO + c * G::CH_R, &tm_do, B(G::B_QF), c * 64, q0, bh, pol_first);
+    }
+    for (int m = 0; m < 2 * nb; ++m) {
+      const int sl = G::slot(m), u = G::use(m);
+      if (u > 0 && !wait_bar(B(G::B_SLE + sl), (u - 1) & 1u, cx.abort_flag)) break;
+      mbar_arrive_expect_tx(B(G::B_SLF + sl), G::TILE_S);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tma_load_3d(sbase + G::OFF_SL + sl * G::TILE_S + c * G::CH_S, (m & 1) ? &tm_v : &tm_k,
+                    B(G::B_SLF + sl), c * 64, (jb0 + (m >> 1)) * kBS, kvz, pol_last);
+    }
+  } else if (warp == 8 && lane == 0 && nb > 0) {
+    // ---- MMA: S(0) dP(0) | S(j+1) dP(j+1) dQ(j) | ...
+    constexpr uint32_t kIdNT = idesc_f16(128, kBS, BF16, false);
+    constexpr uint32_t kIdTN = idesc_f16(128, D, BF16, true);
+    const uint32_t tm = cx.tmem;
+    const uint64_t dq0 = sdesc_sw128(sbase + G::OFF_Q, 16, 1024);
+    const uint64_t ddo0 = sdesc_sw128(sbase + G::OFF_DO, 16, 1024);
+    auto kv_desc = [&](int m, bool mn) {
+      const uint32_t a = sbase + G::OFF_SL + G::slot(m) * G::TILE_S;
+      return mn ? sdesc_sw128(a, G::CH_S, 1024) : sdesc_sw128(a, 16, 1024);
+    };
+    auto wait_item = [&](int m) {
+      return wait_bar(B(G::B_SLF + G::slot(m)), G::use(m) & 1u, cx.abort_flag);
+    };
+    auto issue_sdp = [&](int j) {  // S(j), dP(j); V_j's slot is free once dP(j) completes
+      mma_nt<D>(tm + G::TM_S, dq0, kv_desc(2 * j, false), kIdNT, G::CH_R, G::CH_S);
+      mma_nt<D>(tm + G::TM_DP, ddo0, kv_desc(2 * j + 1, false), kIdNT, G::CH_R, G::CH_S);
+      mma_commit(B(G::B_SDP));
+      mma_commit(B(G::B_SLE + G::slot(2 * j + 1)));
+    };
+    // dS of key column x: warpgroup x / 32 packed its 32 columns at 16 * (x / 32) ..
+    auto acol = [](int kk) { return static_cast<uint32_t>(kk * 8); };
+    bool ok = wait_bar(B(G::B_QF), 0u, cx.abort_flag) && wait_item(0) && wait_item(1);
+    if (ok) {
+      tc_fence_after();
+      issue_sdp(0);
+    }
+    for (int j = 0; ok && j < nb; ++j) {
+      if (j + 1 < nb) {  // next S and dP once the compute warps have read this block's
+        if (!wait_bar(B(G::B_SFREE), j & 1u, cx.abort_flag)) break;
+        if (!wait_item(2 * j + 2) || !wait_item(2 * j + 3)) break;
+        tc_fence_after();
+        issue_sdp(j + 1);
+      }
+      if (!wait_bar(B(G::B_DSF), j & 1u, cx.abort_flag)) break;
+      tc_fence_after();
+      mma_tn_steps<kBS / 16>(tm + G::TM_DQ, tm + G::TM_DS, kv_desc(2 * j, true), kIdTN, j > 0, acol);
+      mma_commit(B(G::B_DSE));
+      mma_commit(B(G::B_SLE + G::slot(2 * j)));  // K_j's slot
+      if (j + 1 == nb) mma_commit(B(G::B_DQF));
+    }
+  } else if (warp < 8) {
+    // ---- compute: thread = query row r, warpgroup h = key columns h*32 .. +31
+    setmaxnreg_inc<176>();
+    const int h = warp >> 2, r = (warp & 3) * 32 + lane;
+    const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const float c = p.c;
+    const size_t srow = static_cast<size_t>(bh) * p.Nq_pad + q0 + r;
+    const float lse2 = p.lse2[srow], dlt = p.delta[srow];
+    const int qpos = q0 + r;
+    bool ok = true;
+    for (int j = 0; ok && j < nb; ++j) {
+      ok = wait_bar(B(G::B_SDP), j & 1u, cx.abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t sr[32], dr[32];
+      tmem_ld_x32(tm + G::TM_S + h * 32, sr);
+      tmem_ld_x32(tm + G::TM_DP + h * 32, dr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_SFREE));
+      // visible keys of this row in the block half: [lo, lim)
+      const int kbase = (jb0 + j) * kBS + h * 32;
+      int lim = p.Nk - kbase;
+      if (p.wr >= 0) lim = min(lim, qpos + p.wr - kbase + 1);
+      const int lo = p.wl >= 0 ? qpos - p.wl - kbase : 0;
+      const uint32_t span = static_cast<uint32_t>(max(lim - lo, 0));
+      uint32_t pk[16];
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        float v2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 2 * x + e;
+          const float pe = ex2(fmaf(__uint_as_float(sr[i]), c, -lse2));
+          v2[e] = static_cast<uint32_t>(i - lo) < span ? pe * (__uint_as_float(dr[i]) - dlt) : 0.f;
+        }
+        pk[x] = pack2(v2[0], v2[1], BF16);
+      }
+      if (j > 0) {  // dQ(j-1) has read the previous dS
+        ok = wait_bar(B(G::B_DSE), (j - 1) & 1u, cx.abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+      }
+      tmem_st_x16(tm + G::TM_DS + h * 16, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_DSF));
+    }
+    // ---- epilogue: dQ = scale * acc, warpgroup h writes columns h*128 .. +127
+    if (nb == 0 && qpos < p.Nq) {  // no key seen by this tile's rows (key windows): dQ = 0
+      uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) + (static_cast<size_t>(bh) * p.Nq + qpos) * D;
+      for (int c0 = h * 128; c0 < (h + 1) * 128; c0 += 8)
+        *reinterpret_cast<uint4*>(dst + c0) = make_uint4(0, 0, 0, 0);
+    }
+    if (ok && nb > 0) {
+      ok = wait_bar(B(G::B_DQF), 0u, cx.abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) +
+                        (static_cast<size_t>(bh) * p.Nq + (qpos < p.Nq ? qpos : 0)) * D;
+#pragma unroll 1
+        for (int c0 = h * 128; c0 < (h + 1) * 128; c0 += 32) {
+          uint32_t a[32];
+          tmem_ld_x32(tm + G::TM_DQ + c0, a);
+          uint32_t w[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            w[x] = pack2(__uint_as_float(a[2 * x]) * p.scale, __uint_as_float(a[2 * x + 1]) * p.scale,
+                         BF16);
+          if (qpos < p.Nq) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*cx.abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) {
+    }
+  }
+  if (threadIdx.x == 0) publish_abort(*cx.abort_flag);
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(cx.tmem, 512);
+  }
+}
+
 }  // namespace fab
 
 // ============================================================================ host side
@@ -757,13 +1290,14 @@ EncodeTiledFnB encode_fn_b() {
   return fn;
 }
 
-// [Z][rows][D] 16-bit tensor, 64 x 128 boxes, 128-byte swizzle, zero fill out of range.
-bool map_rows(CUtensorMap* m, const void* ptr, int D, long long rows, long long Z, bool bf16) {
+// [Z][rows][D] 16-bit tensor, 64 x box_rows boxes, 128-byte swizzle, zero fill out of range.
+bool map_rows(CUtensorMap* m, const void* ptr, int D, long long rows, long long Z, bool bf16,
+              int box_rows = 128) {
   EncodeTiledFnB enc = encode_fn_b();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)Z};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-  const cuuint32_t box[3] = {64u, 128u, 1u};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t es[3] = {1u, 1u, 1u};
   return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
              const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -777,6 +1311,92 @@ bool overlaps_b(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 int nq_pad(int Nq) { return (Nq + 127) / 128 * 128; }
+
+// Parameters shared by the kernels, and the Delta / LSE * log2(e) pass.
+template <int D, bool BF16>
+int setup_bwd(fab::BwdParams& p, const void* o, const void* dout, const float* lse, void* dq,
+              void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
+              int wl, int wr, cudaStream_t st, void* ws, int sms) {
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.Nq_pad = nq_pad(Nq);
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.wl = wl;
+  p.wr = causal ? 0 : wr;
+  p.scale = scale;
+  p.c = scale * fab::kLog2e;
+  p.nqt = p.Nq_pad / 128;
+  p.nkt = (Nk + 127) / 128;
+  float* lse2 = static_cast<float*>(ws);
+  float* delta = lse2 + (size_t)B * Hq * p.Nq_pad;
+  p.lse2 = lse2;
+  p.delta = delta;
+  const long long rows = (long long)B * Hq * p.Nq_pad;
+  const long long warps_needed = (rows * (D / 8) + 31) / 32;
+  long long blocks = (warps_needed + 7) / 8;
+  if (blocks > 16LL * sms) blocks = 16LL * sms;
+  fab::bwd_prep_kernel<D, BF16><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, lse2, delta,
+      B * Hq, Nq, p.Nq_pad);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+// head_dim 256: dV and dK from two launches of the key-tile kernel (64-row
+// query blocks), dQ over 64-key blocks
+template <bool BF16>
+int launch_bwd256(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                  int Nk, float scale, int causal, int wl, int wr, cudaStream_t st, void* ws,
+                  int sms) {
+  using GV = fab::Geo256KV<false>;
+  using GK = fab::Geo256KV<true>;
+  using GQ = fab::Geo256Q;
+  static std::once_flag once;
+  static bool attr_ok = false;
+  std::call_once(once, [] {
+    attr_ok = cudaFuncSetAttribute(fab::bwd_kv256_kernel<BF16, false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   GV::SMEM_BYTES) == cudaSuccess &&
+              cudaFuncSetAttribute(fab::bwd_kv256_kernel<BF16, true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   GK::SMEM_BYTES) == cudaSuccess &&
+              cudaFuncSetAttribute(fab::bwd_dq256_kernel<BF16>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   GQ::SMEM_BYTES) == cudaSuccess;
+  });
+  if (!attr_ok) return FA_ERR_LAUNCH;
+  constexpr int D = 256;
+  // 128-row tiles (resident operands) and 64-row blocks (streamed operands)
+  CUtensorMap tq, tdo, tk, tv, tq_s, tdo_s, tk_s, tv_s;
+  const long long zq = (long long)B * Hq, zk = (long long)B * Hkv;
+  if (!map_rows(&tq, q, D, Nq, zq, BF16) || !map_rows(&tdo, dout, D, Nq, zq, BF16) ||
+      !map_rows(&tk, k, D, Nk, zk, BF16) || !map_rows(&tv, v, D, Nk, zk, BF16) ||
+      !map_rows(&tq_s, q, D, Nq, zq, BF16, fab::kBS) ||
+      !map_rows(&tdo_s, dout, D, Nq, zq, BF16, fab::kBS) ||
+      !map_rows(&tk_s, k, D, Nk, zk, BF16, fab::kBS) || !map_rows(&tv_s, v, D, Nk, zk, BF16, fab::kBS))
+    return FA_ERR_DRIVER;
+  fab::BwdParams p;
+  const int rc = setup_bwd<D, BF16>(p, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                    wl, wr, st, ws, sms);
+  if (rc != FA_OK) return rc;
+  const unsigned kv_grid = (unsigned)(B * Hkv * p.nkt);
+  fab::bwd_kv256_kernel<BF16, false><<<kv_grid, fab::kThreads, GV::SMEM_BYTES, st>>>(
+      tq_s, tdo_s, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fab::bwd_kv256_kernel<BF16, true><<<kv_grid, fab::kThreads, GK::SMEM_BYTES, st>>>(
+      tq_s, tdo_s, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fab::bwd_dq256_kernel<BF16><<<(unsigned)(B * Hq * p.nqt), fab::kThreads, GQ::SMEM_BYTES, st>>>(
+      tq, tdo, tk_s, tv_s, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
 
 template <int D, bool BF16>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -802,37 +1422,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
       !map_rows(&tk, k, D, Nk, (long long)B * Hkv, BF16) ||
       !map_rows(&tv, v, D, Nk, (long long)B * Hkv, BF16))
     return FA_ERR_DRIVER;
-  fab::BwdParams p;
-  p.dq = dq;
-  p.dk = dk;
-  p.dv = dv;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.Nq = Nq;
-  p.Nk = Nk;
-  p.Nq_pad = nq_pad(Nq);
-  p.group = Hq / Hkv;
-  p.causal = causal ? 1 : 0;
-  p.wl = wl;
-  p.wr = causal ? 0 : wr;
-  p.scale = scale;
-  p.c = scale * fab::kLog2e;
-  p.nqt = p.Nq_pad / 128;
-  p.nkt = (Nk + 127) / 128;
-  float* lse2 = static_cast<float*>(ws);
-  float* delta = lse2 + (size_t)B * Hq * p.Nq_pad;
-  p.lse2 = lse2;
-  p.delta = delta;
   // 1. Delta and LSE * log2(e), padded
-  const long long rows = (long long)B * Hq * p.Nq_pad;
-  const long long warps_needed = (rows * (D / 8) + 31) / 32;
-  long long blocks = (warps_needed + 7) / 8;
-  if (blocks > 16LL * sms) blocks = 16LL * sms;
-  fab::bwd_prep_kernel<D, BF16><<<(unsigned)blocks, 256, 0, st>>>(
-      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, lse2, delta,
-      B * Hq, Nq, p.Nq_pad);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fab::BwdParams p;
+  const int rc = setup_bwd<D, BF16>(p, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                    wl, wr, st, ws, sms);
+  if (rc != FA_OK) return rc;
   // 2. dK, dV: one CTA per (b, kv head, key block)
   fab::bwd_dkdv_kernel<D, BF16><<<(unsigned)(B * Hkv * p.nkt), fab::kThreads, GK::SMEM_BYTES, st>>>(
       tq, tdo, tk, tv, p);
@@ -858,7 +1452,7 @@ int fa_bwd_window(const void* q, const void* k, const void* v, const void* o, co
                   void* stream, int dtype, void* workspace, size_t workspace_bytes) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
   if (window_left < -1 || window_right < -1 || (causal && window_right > 0)) return FA_ERR_BAD_WINDOW;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+  if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_BAD_SHAPE;
   if (Hq % Hkv != 0) return FA_ERR_BAD_GROUPING;
   if ((long long)B * Hq * nq_pad(Nq) >= (1ll << 31) || (long long)B * Hkv * Nk >= (1ll << 31))
@@ -895,6 +1489,7 @@ int fa_bwd_window(const void* q, const void* k, const void* v, const void* o, co
 #define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, \
                     window_right, st, workspace, sms
   if (D == 64) return bf ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
+  if (D == 256) return bf ? launch_bwd256<true>(FA_BWD_ARGS) : launch_bwd256<false>(FA_BWD_ARGS);
   return bf ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
 #undef FA_BWD_ARGS
 }

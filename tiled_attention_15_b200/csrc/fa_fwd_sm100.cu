@@ -1087,7 +1087,13 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
           // scaled score + bias * log2(e); the tile holds this row's 128 bias
           // values as 16 swizzled 16-byte units (one row for every query when
           // broadcast over queries)
-          if (p.causal) lim = min(lim, row - kbase + 1);
+          // keys of the block before lim are visible (one query tile: the key
+          // window's right bound; its left bound is applied after the bias)
+          if constexpr (kWin) {
+            if (p.wr >= 0) lim = min(lim, row + p.wr - kbase + 1);
+          } else if (p.causal) {
+            lim = min(lim, row - kbase + 1);
+          }
           const int bs = NQ == 2 ? q : static_cast<int>(b_cnt % G::NBS);
           ok = wait_bar(B(G::B_BFULL + bs), (b_phase >> bs) & 1u, cx.abort_flag);
           if (!__all_sync(0xffffffffu, ok)) return;
@@ -1124,6 +1130,14 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
                 sr[i] = __float_as_uint(i < lim ? x.x : -INFINITY);
                 sr[i + 1] = __float_as_uint(i + 1 < lim ? x.y : -INFINITY);
               }
+            }
+          }
+          if constexpr (kWin) {  // left bound of a key window: keys before lo
+            const int lo = p.wl >= 0 ? row - p.wl - kbase : 0;
+            if (__any_sync(0xffffffffu, lo > 0)) {
+#pragma unroll
+              for (int i = 0; i < kBN; ++i)
+                if (i < lo) sr[i] = __float_as_uint(-INFINITY);
             }
           }
           __syncwarp();
@@ -1746,13 +1760,15 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   // A work tile of at most 128 rows (short queries, or a packed GQA group) runs
   // the one-query-tile kernel: its two S buffers let the softmax of key block j
   // overlap the S MMA of block j + 1, and its K/V staging is deeper.
-  if (bias != nullptr) {  // score bias: the one-query-tile kernels with bias staging
-#define FA_BARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, -1, -1, st, dev, nullptr, 0, \
+  if (bias != nullptr) {  // score bias: the kernels with bias staging
+#define FA_BARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, wl, wr, st, dev, nullptr, 0, \
                  Scratch::kCaller, bias
-    // more than 128 query rows (D <= 128): the two-query-tile kernel
-    if (D == 64 && Nq > fa::kBM)
+    // more than 128 query rows (D <= 128) and no key window: the two-query-tile
+    // kernel; key windows: the one-query-tile kernels, which take them per tile
+    const bool win = wl >= 0 || wr >= 0;
+    if (D == 64 && Nq > fa::kBM && !win)
       return bf ? launch<64, 2, true, true>(FA_BARGS) : launch<64, 2, false, true>(FA_BARGS);
-    if (D == 128 && Nq > fa::kBM)
+    if (D == 128 && Nq > fa::kBM && !win)
       return bf ? launch<128, 2, true, true>(FA_BARGS) : launch<128, 2, false, true>(FA_BARGS);
     switch (D) {
       case 64: return bf ? launch<64, 1, true, true>(FA_BARGS) : launch<64, 1, false, true>(FA_BARGS);
@@ -1809,10 +1825,11 @@ int fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* l
                   window_left, window_right);
 }
 
-int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                int Hkv, int Nq, int Nk, int D, float scale, int causal, const void* bias,
-                long long bias_stride_b, long long bias_stride_h, long long bias_stride_q,
-                void* stream, int dtype) {
+int fa_fwd_bias_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
+                       const void* bias, long long bias_stride_b, long long bias_stride_h,
+                       long long bias_stride_q, int window_left, int window_right, void* stream,
+                       int dtype) {
   if (bias == nullptr) return FA_ERR_NULL_POINTER;
   if (bias_stride_b < 0 || bias_stride_h < 0 || bias_stride_q < 0) return FA_ERR_BAD_SHAPE;
   if ((reinterpret_cast<uintptr_t>(bias) & 15u) || (bias_stride_b & 7) || (bias_stride_h & 7) ||
@@ -1827,7 +1844,15 @@ int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse
   }
   const BiasArg a{bias, bias_stride_b, bias_stride_h, bias_stride_q};
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, nullptr, 0,
-                  Scratch::kCaller, -1, -1, &a);
+                  Scratch::kCaller, window_left, window_right, &a);
+}
+
+int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, const void* bias,
+                long long bias_stride_b, long long bias_stride_h, long long bias_stride_q,
+                void* stream, int dtype) {
+  return fa_fwd_bias_window(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, bias,
+                            bias_stride_b, bias_stride_h, bias_stride_q, -1, -1, stream, dtype);
 }
 
 size_t fa_fwd_workspace_size(int D) {
