@@ -59,7 +59,8 @@ def _load():
             ctypes.c_int64, ctypes.c_int]
         lib.oracle_attention_bwd_ex.restype = ctypes.c_int
         lib.oracle_attention_bwd_ex.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64] * 6 + [
-            ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
+            ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
         lib.oracle_attention_bwd.restype = ctypes.c_int
         lib.oracle_attention_bwd.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64] * 6 + [
             ctypes.c_double, ctypes.c_int, ctypes.c_int]
@@ -115,18 +116,7 @@ def attention(q, k, v, scale: float, causal: bool, rows: Optional[np.ndarray] = 
         pos_ptr = None
     o = np.empty((B, Hq, R, D), dtype=np.float64)
     lse = np.empty((B, Hq, R), dtype=np.float64)
-    bias_ptr, sb, sh, sq = None, 0, 0, 0
-    if bias is not None:
-        bf = _as_f32(bias)
-        while bf.ndim < 4:
-            bf = bf[None]
-        if bf.ndim != 4 or bf.shape[3] != Nk or any(
-                n not in (1, full) for n, full in zip(bf.shape[:3], (B, Hq, Nq))):
-            raise ValueError("bias must broadcast to [B, Hq, Nq, Nk] with its last dim Nk")
-        bf = np.ascontiguousarray(bf)
-        # element strides; a broadcast dim gets stride 0
-        st = [0 if bf.shape[d] == 1 else int(np.prod(bf.shape[d + 1:])) for d in range(3)]
-        bias_ptr, (sb, sh, sq) = bf.ctypes.data, st
+    bf, bias_ptr, sb, sh, sq = _bias_args(bias, B, Hq, Nq, Nk)
     wl, wr = (int(x) for x in window)
     rc = lib.oracle_attention_ex(qf.ctypes.data, pos_ptr, R, kf.ctypes.data, vf.ctypes.data,
                                  o.ctypes.data, lse.ctypes.data, B, Hq, Hkv, Nq, Nk, D,
@@ -137,13 +127,32 @@ def attention(q, k, v, scale: float, causal: bool, rows: Optional[np.ndarray] = 
     return o, lse
 
 
+def _bias_args(bias, B, Hq, Nq, Nk):
+    """(array kept alive, pointer, stride_b, stride_h, stride_q) of a bias that
+    broadcasts to [B, Hq, Nq, Nk]; all None / 0 without a bias."""
+    if bias is None:
+        return None, None, 0, 0, 0
+    bf = _as_f32(bias)
+    while bf.ndim < 4:
+        bf = bf[None]
+    if bf.ndim != 4 or bf.shape[3] != Nk or any(
+            n not in (1, full) for n, full in zip(bf.shape[:3], (B, Hq, Nq))):
+        raise ValueError("bias must broadcast to [B, Hq, Nq, Nk] with its last dim Nk")
+    bf = np.ascontiguousarray(bf)
+    # element strides; a broadcast dim gets stride 0
+    st = [0 if bf.shape[d] == 1 else int(np.prod(bf.shape[d + 1:])) for d in range(3)]
+    return bf, bf.ctypes.data, st[0], st[1], st[2]
+
+
 def attention_bwd(q, k, v, dout, scale: float, causal: bool, nthreads: int = 0,
-                  window: Tuple[int, int] = (-1, -1)):
+                  window: Tuple[int, int] = (-1, -1), bias=None):
     """Gradients of attention in float64 for the upstream gradient dout.
 
     q, dout: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] (torch tensors or numpy arrays).
     window: (left, right) key window as in attention(); rows with no visible
     key contribute nothing.
+    bias: optional additive score bias as in attention() (a given input: the
+    gradients are those of Q, K and V).
     Returns (dQ [B, Hq, Nq, D], dK [B, Hkv, Nk, D], dV [B, Hkv, Nk, D],
     Delta [B, Hq, Nq]) as float64 numpy arrays; Delta_i = dO_i . O_i.
     """
@@ -158,10 +167,12 @@ def attention_bwd(q, k, v, dout, scale: float, causal: bool, nthreads: int = 0,
     dv = np.empty((B, Hkv, Nk, D), dtype=np.float64)
     delta = np.empty((B, Hq, Nq), dtype=np.float64)
     wl, wr = (int(x) for x in window)
+    bf, bias_ptr, sb, sh, sq = _bias_args(bias, B, Hq, Nq, Nk)
     rc = lib.oracle_attention_bwd_ex(qf.ctypes.data, kf.ctypes.data, vf.ctypes.data,
                                      gf.ctypes.data, dq.ctypes.data, dk.ctypes.data,
                                      dv.ctypes.data, delta.ctypes.data, B, Hq, Hkv, Nq, Nk, D,
-                                     float(scale), int(bool(causal)), wl, wr, int(nthreads))
+                                     float(scale), int(bool(causal)), wl, wr, bias_ptr, sb, sh,
+                                     sq, int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_attention_bwd rejected its arguments (code {rc})")
     return dq, dk, dv, delta

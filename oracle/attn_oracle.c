@@ -182,6 +182,13 @@ int oracle_attention(const float *q, const int64_t *q_pos, int64_t R, const floa
  * Key windows (oracle_attention_bwd_ex; same reading as the forward pass):
  * the sums run over the keys i - window_left .. i + window_right only; a row
  * with no such key has O = 0, so it contributes nothing (dQ_i = 0, Delta_i = 0).
+ * An additive score bias (oracle_attention_bwd_ex; the forward pass's float
+ * attn_mask reading): the forward softmax is of scale * q_i . k_j + bias_ij,
+ * so P above includes the bias and nothing else changes (the bias is a given
+ * input: no gradient is formed for it); a key whose bias is -inf has P = 0,
+ * and a row whose every visible key has a bias of -inf is a row with no key.
+ * bias may be NULL; element (b, hq, i, j) at b * bias_sb + hq * bias_sh +
+ * i * bias_sq + j, a zero stride broadcasting that dimension.
  * All arrays are float32 inputs (rounded values) and float64 outputs:
  * q, dout [B, Hq, Nq, D]; k, v [B, Hkv, Nk, D]; dq [B, Hq, Nq, D];
  * dk, dv [B, Hkv, Nk, D]; delta [B, Hq, Nq] (may be NULL).
@@ -191,10 +198,12 @@ int oracle_attention_bwd_ex(const float *q, const float *k, const float *v, cons
                             double *dq, double *dk, double *dv, double *delta, int64_t B,
                             int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
                             double scale, int causal, int64_t window_left,
-                            int64_t window_right, int nthreads) {
+                            int64_t window_right, const float *bias, int64_t bias_sb,
+                            int64_t bias_sh, int64_t bias_sq, int nthreads) {
     if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
     if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || D < 1) return -2;
     if (Hq % Hkv != 0) return -3;
+    if (bias && (bias_sb < 0 || bias_sh < 0 || bias_sq < 0)) return -7;
     const int64_t group = Hq / Hkv;
     int err = 0;
 #ifdef _OPENMP
@@ -232,18 +241,21 @@ int oracle_attention_bwd_ex(const float *q, const float *k, const float *v, cons
                     if (window_right >= 0 && i + window_right < j1) j1 = i + window_right;
                     if (window_left >= 0 && i - window_left > j0) j0 = i - window_left;
                     double *dqi0 = dq + (bh * Nq + i) * D;
-                    if (j1 < j0) { /* no visible key: O = 0, nothing to propagate */
-                        for (int64_t d = 0; d < D; ++d) dqi0[d] = 0.0;
-                        if (delta) delta[bh * Nq + i] = 0.0;
-                        continue;
-                    }
+                    const float *brow =
+                        bias ? bias + b * bias_sb + hq * bias_sh + i * bias_sq : NULL;
                     /* forward softmax of the row */
                     double M = -INFINITY;
                     for (int64_t j = j0; j <= j1; ++j) {
                         double acc = 0.0;
                         for (int64_t d = 0; d < D; ++d) acc += (double)qi[d] * (double)kb[j * D + d];
                         p[j] = scale * acc;
+                        if (brow) p[j] += (double)brow[j];
                         if (p[j] > M) M = p[j];
+                    }
+                    if (M == -INFINITY) { /* no visible key: O = 0, nothing to propagate */
+                        for (int64_t d = 0; d < D; ++d) dqi0[d] = 0.0;
+                        if (delta) delta[bh * Nq + i] = 0.0;
+                        continue;
                     }
                     double Z = 0.0;
                     for (int64_t j = j0; j <= j1; ++j) {
@@ -285,7 +297,7 @@ int oracle_attention_bwd(const float *q, const float *k, const float *v, const f
                          int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
                          double scale, int causal, int nthreads) {
     return oracle_attention_bwd_ex(q, k, v, dout, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk, D, scale,
-                                   causal, -1, -1, nthreads);
+                                   causal, -1, -1, NULL, 0, 0, 0, nthreads);
 }
 
 int oracle_max_threads(void) {

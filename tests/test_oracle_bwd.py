@@ -218,3 +218,102 @@ def test_window_special_cases():
     np.testing.assert_array_equal(dq, 0.0)
     np.testing.assert_array_equal(dk, 0.0)
     np.testing.assert_array_equal(dv, g.astype(np.float64))
+
+
+# ---- additive score bias (float attn_mask): P includes the bias
+
+def _forward64_bias(q, k, v, scale, causal, bias):
+    """softmax(scale q k^T + bias) v in float64; rows with no finite score -> 0."""
+    g = q.shape[1] // k.shape[1]
+    kr, vr = np.repeat(k, g, axis=1), np.repeat(v, g, axis=1)
+    s = scale * np.einsum("bhid,bhjd->bhij", q, kr) + bias
+    if causal:
+        i, j = np.meshgrid(np.arange(q.shape[2]), np.arange(k.shape[2]), indexing="ij")
+        s = np.where(j <= i, s, -np.inf)
+    m = s.max(axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    p = np.exp(s - m)
+    z = p.sum(axis=-1, keepdims=True)
+    p = np.divide(p, z, out=np.zeros_like(p), where=z > 0)
+    return np.einsum("bhij,bhjd->bhid", p, vr)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bias_finite_differences(causal):
+    q, k, v = _rand((1, 2, 5, 3), 60), _rand((1, 1, 6, 3), 61), _rand((1, 1, 6, 3), 62)
+    g = _rand((1, 2, 5, 3), 63)
+    bias = _rand((1, 2, 5, 6), 64, 1.5).astype(np.float64)
+    bias[0, 1, 2, 0] = -np.inf  # one removed key
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.7, causal, bias=bias.astype(np.float32))
+    x = [q.astype(np.float64), k.astype(np.float64), v.astype(np.float64)]
+    bias32 = bias.astype(np.float32).astype(np.float64)
+    o_or, _ = oracle.attention(q, k, v, 0.7, causal, bias=bias.astype(np.float32))
+    np.testing.assert_allclose(_forward64_bias(*x, 0.7, causal, bias32), o_or, rtol=1e-12, atol=1e-13)
+    h = 1e-5
+
+    def loss(xs):
+        return float(np.sum(g.astype(np.float64) * _forward64_bias(*xs, 0.7, causal, bias32)))
+
+    for which, grad in enumerate((dq, dk, dv)):
+        fd = np.zeros_like(grad)
+        for idx in np.ndindex(*grad.shape):
+            xp = [a.copy() for a in x]
+            xm = [a.copy() for a in x]
+            xp[which][idx] += h
+            xm[which][idx] -= h
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * h)
+        np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal,shape", [(False, (2, 4, 30, 36)), (True, (1, 1, 30, 36)),
+                                          (False, (2, 1, 1, 36))])
+def test_bias_against_torch_autograd(causal, shape):
+    # full, shared [N, N] and key-padding shaped biases, with some -inf entries
+    q, k, v = _rand((2, 4, 30, 8), 65), _rand((2, 2, 36, 8), 66), _rand((2, 2, 36, 8), 67)
+    g = _rand((2, 4, 30, 8), 68)
+    bias = _rand(shape, 69, 2.0)
+    bias[np.random.default_rng(70).random(shape) < 0.15] = -np.inf
+    bias[..., 0] = 0.0  # key 0 stays, so every row keeps a key
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.45, causal, bias=bias)
+    qt, kt, vt = (torch.from_numpy(a).double().requires_grad_() for a in (q, k, v))
+    mask = torch.from_numpy(bias).double().expand(2, 4, 30, 36)
+    if causal:
+        mask = mask.masked_fill(~torch.ones(30, 36, dtype=torch.bool).tril(), float("-inf"))
+    o = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt.repeat_interleave(2, dim=1), vt.repeat_interleave(2, dim=1), attn_mask=mask,
+        scale=0.45)
+    o.backward(torch.from_numpy(g).double())
+    np.testing.assert_allclose(dq, qt.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_bias_special_cases():
+    q, k, v = _rand((1, 2, 10, 4), 71), _rand((1, 2, 12, 4), 72), _rand((1, 2, 12, 4), 73)
+    g = _rand((1, 2, 10, 4), 74)
+    # a bias that is constant along each row changes no probability: same gradients
+    shift = _rand((1, 2, 10, 1), 75, 3.0) * np.ones((1, 1, 1, 12), dtype=np.float32)
+    a = oracle.attention_bwd(q, k, v, g, 0.5, False, bias=shift)
+    b = oracle.attention_bwd(q, k, v, g, 0.5, False)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, rtol=1e-11, atol=1e-12)
+    # -inf everywhere but key j = i: O_i = v_i, so dV = dO and dQ = dK = 0
+    eye = np.full((1, 1, 10, 12), -np.inf, dtype=np.float32)
+    eye[0, 0, np.arange(10), np.arange(10)] = 0.0
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, 0.5, False, bias=eye)
+    np.testing.assert_array_equal(dq, 0.0)
+    np.testing.assert_array_equal(dk, 0.0)
+    want = np.zeros_like(dv)
+    want[:, :, :10] = g.astype(np.float64)
+    np.testing.assert_array_equal(dv, want)
+    # a row whose keys are all removed contributes nothing
+    cut = np.zeros((1, 1, 10, 12), dtype=np.float32)
+    cut[0, 0, 3] = -np.inf
+    dq, dk, dv, delta = oracle.attention_bwd(q, k, v, g, 0.5, False, bias=cut)
+    np.testing.assert_array_equal(dq[:, :, 3], 0.0)
+    np.testing.assert_array_equal(delta[:, :, 3], 0.0)
+    g2 = g.copy()
+    g2[:, :, 3] = 0.0
+    _, dk2, dv2, _ = oracle.attention_bwd(q, k, v, g2, 0.5, False, bias=cut)
+    np.testing.assert_allclose(dk, dk2, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dv, dv2, rtol=1e-12, atol=1e-14)
