@@ -289,21 +289,24 @@ def device_qkv(w, dev, seed):
 
 
 def time_launches(fn, flush, stream, n=10, warm=3):
-    """Median CUDA-event time (ms) of fn() over n launches, L2 flushed before each."""
+    """Median CUDA-event time (ms) of fn() over n launches, L2 flushed before each.
+
+    All n launches are enqueued before the host waits, so the host-side cost of
+    a call overlaps the GPU's previous work instead of opening a gap between an
+    event and the kernel it brackets."""
     import torch
     for _ in range(warm):
         flush.zero_()
         fn()
-    ts = []
-    for _ in range(n):
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for a, b in evs:
         flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
         b.record(stream)
-        b.synchronize()
-        ts.append(a.elapsed_time(b))
-    return statistics.median(ts)
+    evs[-1][1].synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
 
 
 def workload_line(w, ms, peak, hbm, flops=None):

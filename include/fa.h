@@ -231,6 +231,24 @@ int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, co
                   int Nk, int D, float scale, int causal, int window_left, int window_right,
                   void *stream, int dtype, void *workspace, size_t workspace_bytes);
 
+/*
+ * fa_bwd with an additive score bias (the gradient of fa_fwd_bias's operation
+ * with respect to q, k and v; the bias is a given input and gets no gradient):
+ * P = exp(scale Q K^T + bias - LSE) in every formula of fa_bwd, with lse from
+ * fa_fwd_bias on the same bias.  Bias layout, strides and their errors as
+ * fa_fwd_bias; causal as fa_bwd.  A row whose keys the bias removed entirely
+ * (its lse is -inf) contributes nothing: its dQ row is 0.  Both kernels stage
+ * each block pair's 128 x 128 bias tile through shared memory by TMA.  D must
+ * be 64 or 128 (else FA_ERR_UNSUPPORTED_HEAD_DIM: at 256 the tile does not fit
+ * beside the operands).  The outputs and the workspace may not overlap the
+ * bias (FA_ERR_OVERLAP).  Other arguments and errors as fa_bwd.
+ */
+int fa_bwd_bias(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq,
+                int Nk, int D, float scale, int causal, const void *bias, long long bias_stride_b,
+                long long bias_stride_h, long long bias_stride_q, void *stream, int dtype,
+                void *workspace, size_t workspace_bytes);
+
 /* Workspace bytes fa_bwd needs: 8 * B * Hq * (Nq rounded up to 128); 0 for bad sizes. */
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq);
 

@@ -186,6 +186,25 @@ def test_bias_window_entry_point_host_checks(lib):
             assert call(wl, wr, causal) == 8  # valid: reaches the device check
 
 
+def test_bwd_bias_host_checks(lib):
+    import torch
+    a = dict(GOOD)
+
+    def call(D=128, bias=13 * A, sq=64, ws=12 * A, dq=9 * A):
+        return lib.fa_bwd_bias(a["q"], a["k"], a["v"], 6 * A, 7 * A, 8 * A, dq, 10 * A, 11 * A,
+                               a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], D,
+                               ctypes.c_float(a["scale"]), 0, bias, 0, 0, sq, None, a["dtype"], ws,
+                               1 << 20)
+    assert call(bias=None) == 1
+    assert call(sq=-8) == 3
+    assert call(bias=13 * A + 8) == 2 and call(sq=60) == 2
+    assert call(D=256) == 5                # no bias tile room at head_dim 256
+    assert call(bias=9 * A) == 12          # dq overlaps the bias
+    assert call(bias=12 * A + 1024) == 12  # the workspace overlaps the bias
+    if not torch.cuda.is_available():
+        assert call() == 8 and call(D=64) == 8
+
+
 def test_bwd_window_host_checks(lib):
     a = dict(GOOD)
 

@@ -34,13 +34,14 @@ def _dout(w):
     return torch.from_numpy(g).to(torch.float16 if w.dtype == "fp16" else torch.bfloat16)
 
 
-def _run(w, dev, window=(-1, -1)):
+def _run(w, dev, window=(-1, -1), bias=None):
     q, k, v = make_qkv(w)
     g = _dout(w)
     qd, kd, vd, gd = (x.to(dev) for x in (q, k, v, g))
-    o, lse = fa.fa_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal, window=window)
+    bd = bias.to(dev) if bias is not None else None
+    o, lse = fa.fa_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal, window=window, bias=bd)
     dq, dk, dv = fa.fa_bwd(qd, kd, vd, o, lse, gd, scale=w.softmax_scale, causal=w.causal,
-                           window=window)
+                           window=window, bias=bd)
     torch.cuda.synchronize()
     assert fa.device_status(reset=True) == 0
     return (q, k, v, g), (dq, dk, dv)
@@ -136,3 +137,63 @@ def test_bwd_window_parity(cuda_dev, w, window):
     (q, k, v, g), got = _run(w, cuda_dev, window)
     dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, w.softmax_scale, w.causal, window=window)
     _check(w, got, (dq, dk, dv), (q, k, v, g), f" window {window}")
+
+
+# ---- additive score bias (fa_bwd_bias): P includes the bias
+
+def _bias(w, shape, seed, scale=2.0, neg_inf_frac=0.0):
+    rng = np.random.default_rng(seed)
+    b = (scale * rng.standard_normal(shape)).astype(np.float32)
+    if neg_inf_frac > 0:
+        b[rng.random(shape) < neg_inf_frac] = -np.inf
+    return torch.from_numpy(b).to(torch.float16 if w.dtype == "fp16" else torch.bfloat16)
+
+
+BIAS_CASES = [
+    (Workload("bwd bias full D128 fp16 ragged GQA", 1, 4, 2, 300, 333, 128, "fp16", False, seed=151),
+     (1, 4, 300, 333), 0.0),
+    (Workload("bwd bias shared [N,N] D128 bf16 causal", 2, 2, 2, 640, 640, 128, "bf16", True, seed=152),
+     (1, 1, 640, 640), 0.0),
+    (Workload("bwd bias key padding D64 fp16", 2, 4, 4, 500, 520, 64, "fp16", False, seed=153),
+     (2, 1, 1, 520), 0.2),
+    (Workload("bwd bias per head D64 bf16 causal GQA 4", 1, 8, 2, 384, 384, 64, "bf16", True, seed=154),
+     (1, 8, 384, 384), 0.05),
+]
+
+
+@pytest.mark.parametrize("w,shape,ninf", BIAS_CASES, ids=lambda c: c.name if hasattr(c, "name") else str(c))
+def test_bwd_bias_parity(cuda_dev, w, shape, ninf):
+    bias = _bias(w, shape, w.seed + 7, neg_inf_frac=ninf)
+    inputs, got = _run(w, cuda_dev, bias=bias)
+    q, k, v, g = inputs
+    ref = oracle.attention_bwd(q, k, v, g, w.softmax_scale, w.causal, bias=bias.float())[:3]
+    _check(w, got, ref, inputs, tag=" bias")
+
+
+def test_bwd_bias_rows_without_keys(cuda_dev):
+    # rows whose keys the bias removes entirely: lse = -inf, their dQ rows are 0
+    w = Workload("bwd bias empty rows D128 fp16", 1, 2, 2, 260, 200, 128, "fp16", False, seed=155)
+    b = np.zeros((1, 2, 260, 200), dtype=np.float32)
+    b[:, :, 100:140] = -np.inf
+    bias = torch.from_numpy(b).half()
+    inputs, got = _run(w, cuda_dev, bias=bias)
+    q, k, v, g = inputs
+    ref = oracle.attention_bwd(q, k, v, g, w.softmax_scale, w.causal, bias=bias.float())[:3]
+    _check(w, got, ref, inputs, tag=" bias")
+    assert (got[0][:, :, 100:140] == 0).all()
+
+
+def test_bwd_zero_bias_equals_no_bias(cuda_dev):
+    # the same forward outputs: a zero bias leaves every backward operation unchanged
+    w = Workload("bwd zero bias D64 fp16", 1, 2, 2, 256, 256, 64, "fp16", True, seed=156)
+    q, k, v = (x.to(cuda_dev) for x in make_qkv(w))
+    g = _dout(w).to(cuda_dev)
+    o, lse = fa.fa_fwd(q, k, v, scale=w.softmax_scale, causal=True)
+    plain = fa.fa_bwd(q, k, v, o, lse, g, scale=w.softmax_scale, causal=True)
+    for shape in ((1, 1, 256, 256), (1, 1, 1, 256)):
+        zero = fa.fa_bwd(q, k, v, o, lse, g, scale=w.softmax_scale, causal=True,
+                         bias=torch.zeros(shape, dtype=torch.float16, device=cuda_dev))
+        torch.cuda.synchronize()
+        assert fa.device_status(reset=True) == 0
+        for a, b in zip(plain, zero):
+            assert torch.equal(a, b)

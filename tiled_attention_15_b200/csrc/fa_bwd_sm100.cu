@@ -52,6 +52,10 @@ constexpr int kBN = 128;  // keys per block
 constexpr int kThreads = 384;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr float kLog2e = 1.4426950408889634f;
+// score bias broadcast (bias_mode bits): one row for every query; per query
+// head; per batch entry (a dimension without its bit has stride 0)
+constexpr int kBiasRowBcast = 1, kBiasPerHead = 2, kBiasPerBatch = 4;
+constexpr int kBiasTileBytes = 128 * 128 * 2;  // [2 boxes][128 rows][64 keys], 16-bit
 
 __device__ unsigned int g_bwd_status = 0;
 __device__ unsigned long long g_bwd_site = 0;
@@ -98,6 +102,13 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, bool bf16) {
   }
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// one 16-bit value (fp16 or bf16) from shared memory, as float
+__device__ __forceinline__ float bias_at(uint32_t saddr, bool bf16) {
+  unsigned short h;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(saddr));
+  return bf16 ? __uint_as_float(static_cast<uint32_t>(h) << 16) : __half2float(__ushort_as_half(h));
 }
 
 __device__ __forceinline__ float2 unpack2(uint32_t w, bool bf16) {
@@ -199,7 +210,7 @@ __device__ __forceinline__ void mma_tn(uint32_t d, uint32_t a, uint64_t b0, uint
 }
 
 // ================================================================== dK, dV
-template <int D>
+template <int D, bool BIAS = false>
 struct GeoKV {
   static constexpr int DCH = D / 64;
   static constexpr int T_BYTES = 128 * D * 2;  // one 128-row tile
@@ -207,14 +218,16 @@ struct GeoKV {
   // Q and dO tiles stream through a ring of single-tile slots in the order
   // Q0 dO0 Q1 dO1 ...; a slot holding Q_n also holds that block's lse2 and
   // delta (1 KB side buffer).  dO_n is freed after dV(n), Q_n after dK(n).
-  static constexpr int NSLOT = D == 64 ? 8 : 4;
+  // (a score bias takes one slot's room at head_dim 128 for its tile)
+  static constexpr int NSLOT = D == 64 ? 8 : (BIAS ? 3 : 4);
   static constexpr int SLOT_BYTES = T_BYTES + 1024;
   static constexpr int OFF_K = 0, OFF_V = T_BYTES, OFF_SL = 2 * T_BYTES;
-  static constexpr int OFF_BAR = OFF_SL + NSLOT * SLOT_BYTES;
+  static constexpr int OFF_BIAS = OFF_SL + NSLOT * SLOT_BYTES;  // the block pair's bias tile
+  static constexpr int OFF_BAR = OFF_BIAS + (BIAS ? kBiasTileBytes : 0);
   // barriers
   static constexpr int B_KV = 0, B_SLF = 1, B_SLE = 1 + NSLOT, B_SF = 1 + 2 * NSLOT,
                        B_DPF = B_SF + 1, B_PF = B_SF + 2, B_DSF = B_SF + 3, B_ACC = B_SF + 4,
-                       NBAR = B_SF + 5;
+                       B_BF = B_SF + 5, B_BE = B_SF + 6, NBAR = B_SF + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // TMEM columns: S^T 0..127 (P^T over it), dP^T 128..255 (dS^T over it), dV, dK
@@ -253,12 +266,12 @@ __device__ __forceinline__ KVTile kv_tile(const BwdParams& p, int bq = kBM) {
   return T;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool BIAS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const BwdParams p) {
-  using G = GeoKV<D>;
+                    const BwdParams p, const __grid_constant__ CUtensorMap tm_b, const int bias_mode) {
+  using G = GeoKV<D, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -282,6 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(B(G::B_PF), 8);
     mbar_init(B(G::B_DSF), 8);
     mbar_init(B(G::B_ACC), 1);
+    mbar_init(B(G::B_BF), 1);
+    mbar_init(B(G::B_BE), 8);
     misc[1] = 0u;
     fence_mbar_init();
   }
@@ -327,6 +342,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(sb + G::T_BYTES, p.lse2 + row, 512, B(G::B_SLF + sl));
         bulk_load(sb + G::T_BYTES + 512, p.delta + row, 512, B(G::B_SLF + sl));
       }
+    }
+  } else if (BIAS && warp == 10 && lane == 0 && T.nb > 0) {
+    // ---- TMA: the bias tile of each (query block, key tile) pair: rows = the
+    // block's queries (one row if broadcast over queries), columns = the tile's keys
+    const uint64_t pol = policy_evict_last();
+    const int rows = (bias_mode & kBiasRowBcast) ? 1 : kBM;
+    const int b = T.bkv / p.Hkv;
+    for (int n = 0; n < T.nb; ++n) {
+      if (n > 0 && !wait_bar(B(G::B_BE), (n - 1) & 1u, cx.abort_flag)) break;
+      const int hq = (T.bkv % p.Hkv) * p.group + n / T.nqb, i = T.i0 + n % T.nqb;
+      mbar_arrive_expect_tx(B(G::B_BF), 2 * rows * 128);
+#pragma unroll
+      for (int box = 0; box < 2; ++box)
+        tma_load_4d(sbase + G::OFF_BIAS + box * (kBiasTileBytes / 2), &tm_b, B(G::B_BF),
+                    kv_row0 + box * 64, (bias_mode & kBiasRowBcast) ? 0 : i * kBM,
+                    (bias_mode & kBiasPerHead) ? hq : 0, (bias_mode & kBiasPerBatch) ? b : 0, pol);
     }
   } else if (warp == 8 && lane == 0 && T.nb > 0) {
     // ---- MMA: S(0) dP(0) | dV(n) S(n+1) dK(n) dP(n+1) | ...
@@ -406,6 +437,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int lo_c = p.wr >= 0 ? dqk - p.wr : -kBM;
       const int hi_c = p.wl >= 0 ? dqk + p.wl : 2 * kBM;
       const uint32_t span = static_cast<uint32_t>(max(hi_c - lo_c + 1, 0));
+      // score bias of (query h*64 + x, key r): the tile's row h*64 + x (row 0 if
+      // broadcast over queries), 16-bit unit (r % 64) / 8 of box r / 64, rotated
+      // by the row (128-byte swizzle)
+      const bool rowb = (bias_mode & kBiasRowBcast) != 0;
+      if (BIAS) {
+        ok = wait_bar(B(G::B_BF), n & 1u, cx.abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      const uint32_t bkey = sbase + G::OFF_BIAS + (r >> 6) * (kBiasTileBytes / 2) + (r & 7) * 2;
+      const uint32_t bu = static_cast<uint32_t>(r >> 3) & 7u;
+      float b_row0 = 0.f;
+      if (BIAS && rowb) b_row0 = bias_at(bkey + ((bu ^ 0u) << 4), BF16) * kLog2e;
       float pv[64];
 #pragma unroll
       for (int x = 0; x < 64; x += 4) {
@@ -413,9 +456,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float e2 = ex2(fmaf(__uint_as_float(sr[x + e]), c, -lv[e]));
+          float bv = 0.f;
+          if (BIAS) {
+            const uint32_t row = static_cast<uint32_t>(h * 64 + x + e);
+            bv = rowb ? b_row0
+                      : bias_at(bkey + row * 128u + ((bu ^ static_cast<uint32_t>((x + e) & 7)) << 4), BF16) *
+                            kLog2e;
+          }
+          const float e2 = ex2(fmaf(__uint_as_float(sr[x + e]), c, bv - lv[e]));
           pv[x + e] = (msk && static_cast<uint32_t>(h * 64 + x + e - lo_c) >= span) ? 0.f : e2;
         }
+      }
+      if (BIAS) {  // this warp has read the bias tile
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B(G::B_BE));
       }
       uint32_t pk[32];
 #pragma unroll
@@ -491,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ================================================================== dQ
-template <int D>
+template <int D, bool BIAS = false>
 struct GeoQ {
   static constexpr int DCH = D / 64;
   static constexpr int T_BYTES = 128 * D * 2;
@@ -500,17 +554,19 @@ struct GeoQ {
   // K0 V0 K1 V1 ...: NKS slots take K_j in turn, NVS slots V_j.  V_j is freed
   // after dP(j), early; K_j only after dQ(j), late -- separate slot sets let
   // V_{j+2} reuse V_j's slot instead of waiting for K_j's.
-  static constexpr int NSLOT = D == 64 ? 10 : 5;
+  // (a score bias takes one K slot's room at head_dim 128 for its tile)
+  static constexpr int NSLOT = D == 64 ? 10 : (BIAS ? 4 : 5);
   static constexpr int NVS = D == 64 ? 4 : 2, NKS = NSLOT - NVS;
   // item m (K_{m/2} for even m, V_{m/2} for odd m): its slot, and how many
   // items used that slot before it
   __device__ static int slot(int m) { return (m & 1) ? NKS + (m >> 1) % NVS : (m >> 1) % NKS; }
   __device__ static int use(int m) { return (m & 1) ? (m >> 1) / NVS : (m >> 1) / NKS; }
   static constexpr int OFF_Q = 0, OFF_DO = T_BYTES, OFF_SL = 2 * T_BYTES;
-  static constexpr int OFF_BAR = OFF_SL + NSLOT * T_BYTES;
+  static constexpr int OFF_BIAS = OFF_SL + NSLOT * T_BYTES;  // the block pair's bias tile
+  static constexpr int OFF_BAR = OFF_BIAS + (BIAS ? kBiasTileBytes : 0);
   static constexpr int B_QF = 0, B_SLF = 1, B_SLE = 1 + NSLOT, B_SDP = 1 + 2 * NSLOT,
                        B_SFREE = B_SDP + 1, B_DSF = B_SDP + 2, B_DSE = B_SDP + 3, B_DQF = B_SDP + 4,
-                       NBAR = B_SDP + 5;
+                       B_BF = B_SDP + 5, B_BE = B_SDP + 6, NBAR = B_SDP + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // TMEM columns: S 0..127, dP 128..255, dS (packed) 256..319, dQ 320..320+D-1
@@ -519,12 +575,12 @@ struct GeoQ {
   static_assert(320 + D <= 512, "tensor memory budget");
 };
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool BIAS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const BwdParams p) {
-  using G = GeoQ<D>;
+                  const BwdParams p, const __grid_constant__ CUtensorMap tm_b, const int bias_mode) {
+  using G = GeoQ<D, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -566,6 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(B(G::B_DSF), 8);
     mbar_init(B(G::B_DSE), 1);
     mbar_init(B(G::B_DQF), 1);
+    mbar_init(B(G::B_BF), 1);
+    mbar_init(B(G::B_BE), 8);
     misc[1] = 0u;
     fence_mbar_init();
   }
@@ -598,6 +656,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < G::DCH; ++c)
         tma_load_3d(sbase + G::OFF_SL + sl * G::T_BYTES + c * G::CHUNK, (m & 1) ? &tm_v : &tm_k,
                     B(G::B_SLF + sl), c * 64, (jb0 + (m >> 1)) * kBN, kvz, pol_last);
+    }
+  } else if (BIAS && warp == 10 && lane == 0 && nb > 0) {
+    // ---- TMA: the bias tile of each key block: rows = this tile's queries (one
+    // row if broadcast over queries), columns = the block's keys
+    const uint64_t pol = policy_evict_last();
+    const int rows = (bias_mode & kBiasRowBcast) ? 1 : kBM;
+    for (int j = 0; j < nb; ++j) {
+      if (j > 0 && !wait_bar(B(G::B_BE), (j - 1) & 1u, cx.abort_flag)) break;
+      mbar_arrive_expect_tx(B(G::B_BF), 2 * rows * 128);
+#pragma unroll
+      for (int box = 0; box < 2; ++box)
+        tma_load_4d(sbase + G::OFF_BIAS + box * (kBiasTileBytes / 2), &tm_b, B(G::B_BF),
+                    (jb0 + j) * kBN + box * 64, (bias_mode & kBiasRowBcast) ? 0 : q0,
+                    (bias_mode & kBiasPerHead) ? bh % p.Hq : 0,
+                    (bias_mode & kBiasPerBatch) ? bh / p.Hq : 0, pol);
     }
   } else if (warp == 8 && lane == 0 && nb > 0) {
     // ---- MMA: S(0) dP(0) | S(j+1) dP(j+1) dQ(j) | ...
@@ -668,14 +741,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.wr >= 0) lim = min(lim, qpos + p.wr - kbase + 1);
       const int lo = p.wl >= 0 ? qpos - p.wl - kbase : 0;
       const uint32_t span = static_cast<uint32_t>(max(lim - lo, 0));
+      // score bias of this row, keys h*64 .. +63: box h of the tile, row r (row 0
+      // if broadcast over queries), 16-byte units rotated by the row
+      uint32_t bw[32];
+      if (BIAS) {
+        ok = wait_bar(B(G::B_BF), j & 1u, cx.abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const uint32_t brow = (bias_mode & kBiasRowBcast) ? 0u : static_cast<uint32_t>(r);
+        const uint32_t bb = sbase + G::OFF_BIAS + h * (kBiasTileBytes / 2) + brow * 128u;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(bw[4 * u]), "=r"(bw[4 * u + 1]), "=r"(bw[4 * u + 2]), "=r"(bw[4 * u + 3])
+                       : "r"(bb + ((static_cast<uint32_t>(u) ^ (brow & 7u)) << 4)));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B(G::B_BE));
+      }
       uint32_t pk[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
+        float2 b2 = make_float2(0.f, 0.f);
+        if (BIAS) b2 = unpack2(bw[x], BF16);
         float v2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int i = 2 * x + e;
-          const float pe = ex2(fmaf(__uint_as_float(sr[i]), c, -lse2));
+          const float bv = BIAS ? (e ? b2.y : b2.x) * kLog2e : 0.f;
+          const float pe = ex2(fmaf(__uint_as_float(sr[i]), c, bv - lse2));
           v2[e] = static_cast<uint32_t>(i - lo) < span ? pe * (__uint_as_float(dr[i]) - dlt) : 0.f;
         }
         pk[x] = pack2(v2[0], v2[1], BF16);
@@ -1305,6 +1397,33 @@ bool map_rows(CUtensorMap* m, const void* ptr, int D, long long rows, long long 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A score bias: element (b, hq, i, j) at ptr + b * sb + hq * sh + i * sq + j
+// (elements; a zero stride broadcasts that dimension).
+struct BiasArgB {
+  const void* ptr;
+  long long sb, sh, sq;
+};
+
+// [B][H][Nq][Nk] view of the bias with broadcast dimensions of extent 1; boxes
+// of 64 keys x 128 rows (1 row when broadcast over queries), 128-byte swizzle.
+bool map_bias(CUtensorMap* m, const BiasArgB& a, int B, int H, int Nq, int Nk, bool bf16) {
+  EncodeTiledFnB enc = encode_fn_b();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)Nk, (cuuint64_t)(a.sq ? Nq : 1), (cuuint64_t)(a.sh ? H : 1),
+                              (cuuint64_t)(a.sb ? B : 1)};
+  // strides of extent-1 dimensions are never used; keep them valid and increasing
+  const cuuint64_t s1 = a.sq ? (cuuint64_t)a.sq * 2 : (cuuint64_t)((Nk * 2 + 15) / 16 * 16);
+  const cuuint64_t s2 = a.sh ? (cuuint64_t)a.sh * 2 : s1 * dims[1];
+  const cuuint64_t s3 = a.sb ? (cuuint64_t)a.sb * 2 : s2 * dims[2];
+  const cuuint64_t strides[3] = {s1, s2, s3};
+  const cuuint32_t box[4] = {64u, a.sq ? 128u : 1u, 1u, 1u};
+  const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+             const_cast<void*>(a.ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool overlaps_b(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
@@ -1398,20 +1517,20 @@ int launch_bwd256(const void* q, const void* k, const void* v, const void* o, co
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool BIAS = false>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
                int Nk, float scale, int causal, int wl, int wr, cudaStream_t st, void* ws,
-               int sms) {
-  using GK = fab::GeoKV<D>;
-  using GQ = fab::GeoQ<D>;
+               int sms, const BiasArgB* bias = nullptr) {
+  using GK = fab::GeoKV<D, BIAS>;
+  using GQ = fab::GeoQ<D, BIAS>;
   static std::once_flag once;
   static bool attr_ok = false;
   std::call_once(once, [] {
-    attr_ok = cudaFuncSetAttribute(fab::bwd_dkdv_kernel<D, BF16>,
+    attr_ok = cudaFuncSetAttribute(fab::bwd_dkdv_kernel<D, BF16, BIAS>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    GK::SMEM_BYTES) == cudaSuccess &&
-              cudaFuncSetAttribute(fab::bwd_dq_kernel<D, BF16>,
+              cudaFuncSetAttribute(fab::bwd_dq_kernel<D, BF16, BIAS>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    GQ::SMEM_BYTES) == cudaSuccess;
   });
@@ -1422,18 +1541,25 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
       !map_rows(&tk, k, D, Nk, (long long)B * Hkv, BF16) ||
       !map_rows(&tv, v, D, Nk, (long long)B * Hkv, BF16))
     return FA_ERR_DRIVER;
+  CUtensorMap tb = tk;  // (unused without a bias)
+  int bias_mode = 0;
+  if (BIAS) {
+    if (!map_bias(&tb, *bias, B, Hq, Nq, Nk, BF16)) return FA_ERR_DRIVER;
+    bias_mode = (bias->sq ? 0 : fab::kBiasRowBcast) | (bias->sh ? fab::kBiasPerHead : 0) |
+                (bias->sb ? fab::kBiasPerBatch : 0);
+  }
   // 1. Delta and LSE * log2(e), padded
   fab::BwdParams p;
   const int rc = setup_bwd<D, BF16>(p, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal,
                                     wl, wr, st, ws, sms);
   if (rc != FA_OK) return rc;
   // 2. dK, dV: one CTA per (b, kv head, key block)
-  fab::bwd_dkdv_kernel<D, BF16><<<(unsigned)(B * Hkv * p.nkt), fab::kThreads, GK::SMEM_BYTES, st>>>(
-      tq, tdo, tk, tv, p);
+  fab::bwd_dkdv_kernel<D, BF16, BIAS><<<(unsigned)(B * Hkv * p.nkt), fab::kThreads, GK::SMEM_BYTES, st>>>(
+      tq, tdo, tk, tv, p, tb, bias_mode);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   // 3. dQ: one CTA per (b, query head, query block)
-  fab::bwd_dq_kernel<D, BF16><<<(unsigned)(B * Hq * p.nqt), fab::kThreads, GQ::SMEM_BYTES, st>>>(
-      tq, tdo, tk, tv, p);
+  fab::bwd_dq_kernel<D, BF16, BIAS><<<(unsigned)(B * Hq * p.nqt), fab::kThreads, GQ::SMEM_BYTES, st>>>(
+      tq, tdo, tk, tv, p, tb, bias_mode);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -1446,13 +1572,18 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Nq) {
   return 2ull * (size_t)B * Hq * nq_pad(Nq) * sizeof(float);
 }
 
-int fa_bwd_window(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                  const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
-                  int Nk, int D, float scale, int causal, int window_left, int window_right,
-                  void* stream, int dtype, void* workspace, size_t workspace_bytes) {
+}  // extern "C"
+
+namespace {
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+             int D, float scale, int causal, int window_left, int window_right, void* stream,
+             int dtype, void* workspace, size_t workspace_bytes, const BiasArgB* bias) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_BAD_DTYPE;
   if (window_left < -1 || window_right < -1 || (causal && window_right > 0)) return FA_ERR_BAD_WINDOW;
   if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+  if (bias && D == 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;  // no room for a bias tile
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_BAD_SHAPE;
   if (Hq % Hkv != 0) return FA_ERR_BAD_GROUPING;
   if ((long long)B * Hq * nq_pad(Nq) >= (1ll << 31) || (long long)B * Hkv * Nk >= (1ll << 31))
@@ -1478,6 +1609,12 @@ int fa_bwd_window(const void* q, const void* k, const void* v, const void* o, co
     for (int b = a + 1; b < 4; ++b)
       if (overlaps_b(outs[a], out_b[a], outs[b], out_b[b])) return FA_ERR_OVERLAP;
   }
+  if (bias) {  // the outputs and the workspace must not overlap the bias either
+    const size_t extent = 2 * static_cast<size_t>((B - 1) * bias->sb + (Hq - 1) * bias->sh +
+                                                  (Nq - 1) * bias->sq + Nk);
+    for (int a = 0; a < 4; ++a)
+      if (overlaps_b(outs[a], out_b[a], bias->ptr, extent)) return FA_ERR_OVERLAP;
+  }
   int dev = -1, major = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
@@ -1488,10 +1625,42 @@ int fa_bwd_window(const void* q, const void* k, const void* v, const void* o, co
   const bool bf = dtype == FA_BF16;
 #define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, \
                     window_right, st, workspace, sms
+  if (bias) {
+    if (D == 64)
+      return bf ? launch_bwd<64, true, true>(FA_BWD_ARGS, bias) : launch_bwd<64, false, true>(FA_BWD_ARGS, bias);
+    return bf ? launch_bwd<128, true, true>(FA_BWD_ARGS, bias) : launch_bwd<128, false, true>(FA_BWD_ARGS, bias);
+  }
   if (D == 64) return bf ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
   if (D == 256) return bf ? launch_bwd256<true>(FA_BWD_ARGS) : launch_bwd256<false>(FA_BWD_ARGS);
   return bf ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
 #undef FA_BWD_ARGS
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd_window(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                  int Nk, int D, float scale, int causal, int window_left, int window_right,
+                  void* stream, int dtype, void* workspace, size_t workspace_bytes) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                  window_left, window_right, stream, dtype, workspace, workspace_bytes, nullptr);
+}
+
+int fa_bwd_bias(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                int Nk, int D, float scale, int causal, const void* bias, long long bias_stride_b,
+                long long bias_stride_h, long long bias_stride_q, void* stream, int dtype,
+                void* workspace, size_t workspace_bytes) {
+  if (bias == nullptr) return FA_ERR_NULL_POINTER;
+  if (bias_stride_b < 0 || bias_stride_h < 0 || bias_stride_q < 0) return FA_ERR_BAD_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(bias) & 15u) || (bias_stride_b & 7) || (bias_stride_h & 7) ||
+      (bias_stride_q & 7))
+    return FA_ERR_MISALIGNED;
+  const BiasArgB a{bias, bias_stride_b, bias_stride_h, bias_stride_q};
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, D, scale, causal, -1, -1,
+                  stream, dtype, workspace, workspace_bytes, &a);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
