@@ -1,12 +1,13 @@
 """Run one attention workload a few times on synthetic inputs (for profilers).
 
     python -m tiled_attention_15_b200.run --B 1 --Hq 32 --N 4096 --D 128 [--causal]
-        [--Hkv 8] [--dtype bf16] [--iters 3] [--path fused|unfused|bwd]
+        [--Hkv 8] [--dtype bf16] [--iters 3] [--path fused|unfused|bwd] [--bias]
 
 Inputs are seeded N(0, 1) draws made on the device and rounded to the dtype;
 an L2 flush (256 MiB write) precedes every launch, so a profiler that
-captures launch k sees the same cold-L2 state the benchmark times.  Prints
-the CUDA-event time of each launch.
+captures launch k sees the same cold-L2 state the benchmark times.  --bias
+adds one [Nq, Nk] score bias shared by all heads (fused forward and
+backward).  Prints the CUDA-event time of each launch.
 """
 from __future__ import annotations
 
@@ -30,6 +31,7 @@ def main():
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--path", default="fused", choices=["fused", "unfused", "bwd"])
+    ap.add_argument("--bias", action="store_true")
     a = ap.parse_args()
     dev = torch.device("cuda:0")
     dt = torch.bfloat16 if a.dtype == "bf16" else torch.float16
@@ -43,21 +45,23 @@ def main():
     lse = torch.empty((a.B, a.Hq, a.N), dtype=torch.float32, device=dev)
     flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
     scale = 1.0 / math.sqrt(a.D)
+    bias = torch.randn((1, 1, a.N, nk), device=dev, generator=g).to(dt) if a.bias else None
     if a.path == "bwd":
-        fa.fa_fwd(q, k, v, o=o, lse=lse, scale=scale, causal=a.causal)
+        fa.fa_fwd(q, k, v, o=o, lse=lse, scale=scale, causal=a.causal, bias=bias)
         dout = torch.randn(q.shape, device=dev, generator=g).to(dt)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         ws = torch.empty(int(fa.load_library().fa_bwd_workspace_size(a.B, a.Hq, a.N)),
                          dtype=torch.uint8, device=dev)
         call = lambda: fa.fa_bwd(q, k, v, o, lse, dout, scale=scale, causal=a.causal,  # noqa: E731
-                                 dq=dq, dk=dk, dv=dv, workspace=ws)
+                                 dq=dq, dk=dk, dv=dv, workspace=ws, bias=bias)
     elif a.path == "unfused":
         ws = torch.empty(int(fa.load_library().fa_fwd_unfused_workspace_size(a.B, a.Hq, a.N, nk)),
                          dtype=torch.uint8, device=dev)
         call = lambda: fa.fa_fwd_unfused(q, k, v, o=o, lse=lse, scale=scale,  # noqa: E731
                                          causal=a.causal, workspace=ws)
     else:
-        call = lambda: fa.fa_fwd(q, k, v, o=o, lse=lse, scale=scale, causal=a.causal)  # noqa: E731
+        call = lambda: fa.fa_fwd(q, k, v, o=o, lse=lse, scale=scale, causal=a.causal,  # noqa: E731
+                                 bias=bias)
     for i in range(a.iters):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
