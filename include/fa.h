@@ -188,6 +188,22 @@ int fa_fwd_bias_window(const void *q, const void *k, const void *v, void *o, flo
                        int dtype);
 
 /*
+ * fa_fwd_bias_window with a caller workspace (as fa_fwd_ws: at least
+ * fa_fwd_workspace_size(D) bytes, 256-byte aligned, zero-filled before first
+ * use and left zeroed; NULL = fa_fwd_bias_window).  With it, bias launches
+ * take work units from the dynamic schedule, and those with more than 128
+ * query rows and no key window split the last round of tiles over two CTAs
+ * (merged in a fixed order; a part in which the bias removed every key of a
+ * row carries no weight).  The workspace may not overlap the bias
+ * (FA_ERR_OVERLAP).  Other arguments and errors as fa_fwd_bias_window.
+ */
+int fa_fwd_bias_ws(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int D, float scale, int causal, const void *bias,
+                   long long bias_stride_b, long long bias_stride_h, long long bias_stride_q,
+                   int window_left, int window_right, void *stream, int dtype, void *workspace,
+                   size_t workspace_bytes);
+
+/*
  * Backward pass: the gradients of the attention above for an upstream gradient
  * dout (the pages mention only that training keeps gradients -- hwcomputing.
  * csdn.net page, section on standard attention; the operation is taken as the

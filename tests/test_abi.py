@@ -205,6 +205,22 @@ def test_bwd_bias_host_checks(lib):
         assert call() == 8 and call(D=64) == 8
 
 
+def test_bias_ws_entry_point_host_checks(lib):
+    import torch
+    a = dict(GOOD)
+
+    def call(ws=14 * A, bias=9 * A, causal=0, wl=-1):
+        return lib.fa_fwd_bias_ws(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"],
+                                  a["Hkv"], a["Nq"], a["Nk"], a["D"], ctypes.c_float(a["scale"]),
+                                  causal, bias, 0, 0, 64, wl, -1, None, a["dtype"], ws, 1 << 20)
+    assert call(bias=None) == 1
+    assert call(ws=14 * A + 128) == 2          # workspace not 256-byte aligned
+    assert call(ws=9 * A - 4096) == 12         # the workspace overlaps the bias
+    assert call(wl=-2) == 14
+    if not torch.cuda.is_available():
+        assert call() == 8 and call(ws=None) == 8 and call(wl=16, causal=1) == 8
+
+
 def test_bwd_window_host_checks(lib):
     a = dict(GOOD)
 

@@ -156,3 +156,43 @@ def test_window_and_bias_d256_per_head(cuda_dev):
     w = Workload("window 96 causal + per-head bias D256 bf16", 1, 4, 1, 400, 400, 256, "bf16",
                  True, seed=124)
     _check(w, _bias(w, (1, 4, 400, 400), 12), cuda_dev, " window", window=(96, -1))
+
+
+# ---- split tail and dynamic schedule with a bias (fa_fwd_bias_ws)
+
+def test_bias_split_tail_and_removed_rows(cuda_dev):
+    # 20 tiles of 256 rows on 16 CTAs: the last 4 tiles are split over two CTAs
+    # each (8 key blocks -> two halves) and merged.  Rows 300..339 of head 0 lose
+    # every key; rows 600..639 lose exactly the first half of the keys (one part
+    # of their split tile sees no key) and rows 700..739 the second half.
+    w = Workload("split tail + removed rows D128 fp16", 1, 5, 5, 1024, 1024, 128, "fp16", False,
+                 seed=125)
+    b = 2.0 * np.random.default_rng(13).standard_normal((1, 5, 1024, 1024)).astype(np.float32)
+    b[0, 0, 300:340, :] = -np.inf
+    b[0, 4, 600:640, :512] = -np.inf
+    b[0, 4, 700:740, 512:] = -np.inf
+    bias = torch.from_numpy(b).half()
+    prev = fa.set_max_ctas(16)
+    try:
+        o, lse = _check(w, bias, cuda_dev, " split")
+        assert torch.isneginf(lse[0, 0, 300:340]).all() and (o[0, 0, 300:340] == 0).all()
+        wb = w.with_(name="split tail shared [N,N] bias D64 bf16", D=64, dtype="bf16", seed=126)
+        _check(wb, _bias(wb, (1, 1, 1024, 1024), 14), cuda_dev, " split")
+    finally:
+        fa.set_max_ctas(prev)
+
+
+def test_bias_workspace_matches_no_workspace(cuda_dev):
+    # the dynamic schedule does not change a unit's arithmetic: bit-identical
+    # to the static order (no split: 8 tiles on 8 CTAs per round)
+    w = Workload("bias ws vs none D128 bf16", 2, 4, 4, 512, 700, 128, "bf16", False, seed=127)
+    q, k, v = (x.to(cuda_dev) for x in make_qkv(w))
+    bias = _bias(w, (2, 4, 512, 700), 15).to(cuda_dev)
+    prev = fa.set_max_ctas(5)
+    try:
+        a = fa.fa_fwd(q, k, v, scale=w.softmax_scale, bias=bias)
+        b_ = fa.fa_fwd(q, k, v, scale=w.softmax_scale, bias=bias, use_workspace=False)
+    finally:
+        fa.set_max_ctas(prev)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b_[0]) and torch.equal(a[1], b_[1])

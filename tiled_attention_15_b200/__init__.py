@@ -26,7 +26,7 @@ FA_ERR_BAD_WORKSPACE = 15
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
-            "fa_fwd_window", "fa_fwd_bias", "fa_fwd_bias_window", "fa_bwd", "fa_bwd_window", "fa_bwd_bias",
+            "fa_fwd_window", "fa_fwd_bias", "fa_fwd_bias_window", "fa_fwd_bias_ws", "fa_bwd", "fa_bwd_window", "fa_bwd_bias",
             "fa_bwd_workspace_size",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
             "fa_fwd_unfused", "fa_fwd_unfused_workspace_size",
@@ -68,6 +68,9 @@ def load_library() -> ctypes.CDLL:
     lib.fa_fwd_bias.restype = i
     lib.fa_fwd_bias_window.argtypes = fwd_args[:13] + [vp, ll, ll, ll, i, i, vp, i]
     lib.fa_fwd_bias_window.restype = i
+    lib.fa_fwd_bias_ws.argtypes = fwd_args[:13] + [vp, ll, ll, ll, i, i, vp, i, vp,
+                                                    ctypes.c_size_t]
+    lib.fa_fwd_bias_ws.restype = i
     lib.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, vp, i, vp, ctypes.c_size_t]
     lib.fa_bwd.restype = i
     lib.fa_bwd_window.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, i, i, vp, i, vp, ctypes.c_size_t]
@@ -185,9 +188,9 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
     scale defaults to 1/sqrt(D).  use_workspace: call fa_fwd_ws with a cached
     per-(device, stream) workspace (load balance), else fa_fwd.  window:
     (left, right) key window, -1 = unbounded (fa_fwd_window when either is set).
-    bias: additive score bias (fa_fwd_bias), a CUDA tensor of q's dtype that
-    broadcasts to [B, Hq, Nq, Nk] (size-1 dims broadcast); with a window as
-    well, fa_fwd_bias_window.
+    bias: additive score bias (fa_fwd_bias_ws, with the workspace when
+    use_workspace), a CUDA tensor of q's dtype that broadcasts to
+    [B, Hq, Nq, Nk] (size-1 dims broadcast); a window may come with it.
     Returns (o, lse or None).
     """
     import torch
@@ -223,15 +226,12 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
     wl, wr = (int(x) for x in window)
     if bias is not None:
         bt, sb, sh, sq = _bias_view(bias, q.dtype, B, Hq, Nq, Nk)
-        if (wl, wr) != (-1, -1):
-            rc = lib.fa_fwd_bias_window(*args[:13], bt.data_ptr(), sb, sh, sq, wl, wr, args[13],
-                                        dtype)
-            if rc != FA_OK:
-                raise FaError(rc, "fa_fwd_bias_window")
-            return o, lse
-        rc = lib.fa_fwd_bias(*args[:13], bt.data_ptr(), sb, sh, sq, args[13], dtype)
+        ws = workspace(q.device, stream) if use_workspace else None
+        rc = lib.fa_fwd_bias_ws(*args[:13], bt.data_ptr(), sb, sh, sq, wl, wr, args[13], dtype,
+                                ws.data_ptr() if ws is not None else None,
+                                ws.numel() if ws is not None else 0)
         if rc != FA_OK:
-            raise FaError(rc, "fa_fwd_bias")
+            raise FaError(rc, "fa_fwd_bias_ws")
         return o, lse
     if (wl, wr) != (-1, -1):
         ws = workspace(q.device, stream) if use_workspace else None

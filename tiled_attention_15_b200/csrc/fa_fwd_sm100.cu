@@ -998,7 +998,10 @@ __device__ __forceinline__ void merge_epilogue_rows(const FwdParams& p, const Ti
       L = fmaf(a, ml.y, L);
       Lr = fmaf(a, ml.z, Lr);
     }
-    const float inv = 1.f / (BF16 ? Lr : L);
+    // a part in which a score bias removed every key of the row has m = -inf
+    // (weight 0); a row with no key in any part has no softmax: O = 0, LSE = -inf
+    const bool empty = M == -INFINITY;
+    const float inv = empty ? 0.f : 1.f / (BF16 ? Lr : L);
     uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
 #pragma unroll 1
     for (int c4 = 0; c4 < D / 4; c4 += 8) {  // 32 columns per pass
@@ -1006,7 +1009,7 @@ __device__ __forceinline__ void merge_epilogue_rows(const FwdParams& p, const Ti
 #pragma unroll
       for (int x = 0; x < 32; ++x) z[x] = 0.f;
       for (int s = 0; s < T.nparts; ++s) {
-        const float sc = ex2(__ldcg(p.ws_ml + mlx(s)).x - M) * inv;
+        const float sc = empty ? 0.f : ex2(__ldcg(p.ws_ml + mlx(s)).x - M) * inv;
         float4 u[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) u[x] = __ldcg(p.ws_o + ox(s, c4 + x));
@@ -1027,7 +1030,7 @@ __device__ __forceinline__ void merge_epilogue_rows(const FwdParams& p, const Ti
                               pack2(z[8 * x + 6], z[8 * x + 7], BF16));
       }
     }
-    if (p.lse != nullptr && ri.live) p.lse[ri.out_row] = (M + log2f(L)) * kLn2;
+    if (p.lse != nullptr && ri.live) p.lse[ri.out_row] = empty ? -INFINITY : (M + log2f(L)) * kLn2;
   }
   __syncwarp();
   if (lane == 0) *cnt = 0;
@@ -1240,7 +1243,8 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
     if (T.slot >= 0) {
       if constexpr (NQ == 2) {
-        merge_epilogue_rows<D, NQ, BF16>(p, T, q, sub, lane, ri, tm + 256 + q * D, m_sub, l, l_r);
+        merge_epilogue_rows<D, NQ, BF16>(p, T, q, sub, lane, ri, tm + 256 + q * D,
+                                         BIAS ? m_used : m_sub, l, l_r);
       } else if (!merge_epilogue<D, NQ, BF16, G>(cx, m_phase, p, T, q, sub, lane, tm + 256 + q * D,
                                                  m_sub, l, l_r)) {
         return;
@@ -1590,8 +1594,9 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.ws_rows = (p.ws_rows + 31) / 32 * 32;
   int n_split = 0, nsplit = 1;
   int sk_w = 0, sk_grid = 0;
-  if (ws != nullptr && !causal && !windowed && !BIAS) {
-    if (p.n_tiles < ctas && p.n_tiles <= kMaxSplit) {
+  // (score bias: the split tail on the two-query-tile kernel, no stream-K)
+  if (ws != nullptr && !causal && !windowed && (!BIAS || NQ == 2)) {
+    if (!BIAS && p.n_tiles < ctas && p.n_tiles <= kMaxSplit) {
       // Stream-K: fewer tiles than CTAs (decode-like shapes).  The key blocks of
       // all tiles are shared out evenly over C CTAs, each with at least
       // kMinPartBlocks of them; C shrinks until the partials fit the workspace.
@@ -1764,7 +1769,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   // the one-query-tile kernel: its two S buffers let the softmax of key block j
   // overlap the S MMA of block j + 1, and its K/V staging is deeper.
   if (bias != nullptr) {  // score bias: the kernels with bias staging
-#define FA_BARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, wl, wr, st, dev, nullptr, 0, \
+#define FA_BARGS q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, wl, wr, st, dev, ws, ws_bytes, \
                  Scratch::kCaller, bias
     // more than 128 query rows (D <= 128) and no key window: the two-query-tile
     // kernel; key windows: the one-query-tile kernels, which take them per tile
@@ -1828,12 +1833,14 @@ int fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* l
                   window_left, window_right);
 }
 
-int fa_fwd_bias_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                       int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
-                       const void* bias, long long bias_stride_b, long long bias_stride_h,
-                       long long bias_stride_q, int window_left, int window_right, void* stream,
-                       int dtype) {
+int fa_fwd_bias_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int D, float scale, int causal, const void* bias,
+                   long long bias_stride_b, long long bias_stride_h, long long bias_stride_q,
+                   int window_left, int window_right, void* stream, int dtype, void* workspace,
+                   size_t workspace_bytes) {
   if (bias == nullptr) return FA_ERR_NULL_POINTER;
+  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return FA_ERR_MISALIGNED;
   if (bias_stride_b < 0 || bias_stride_h < 0 || bias_stride_q < 0) return FA_ERR_BAD_SHAPE;
   if ((reinterpret_cast<uintptr_t>(bias) & 15u) || (bias_stride_b & 7) || (bias_stride_h & 7) ||
       (bias_stride_q & 7))
@@ -1845,9 +1852,25 @@ int fa_fwd_bias_window(const void* q, const void* k, const void* v, void* o, flo
         (lse && overlaps(lse, (size_t)B * Hq * Nq * 4, bias, extent)))
       return FA_ERR_OVERLAP;
   }
+  if (workspace != nullptr && B >= 1 && Hq >= 1 && Nq >= 1 && Nk >= 1) {  // nor the workspace
+    const size_t extent = 2 * static_cast<size_t>((B - 1) * bias_stride_b + (Hq - 1) * bias_stride_h +
+                                                  (Nq - 1) * bias_stride_q + Nk);
+    if (overlaps(workspace, workspace_bytes, bias, extent)) return FA_ERR_OVERLAP;
+  }
   const BiasArg a{bias, bias_stride_b, bias_stride_h, bias_stride_q};
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, nullptr, 0,
-                  Scratch::kCaller, window_left, window_right, &a);
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dtype, workspace,
+                  workspace != nullptr ? workspace_bytes : 0, Scratch::kCaller, window_left,
+                  window_right, &a);
+}
+
+int fa_fwd_bias_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
+                       const void* bias, long long bias_stride_b, long long bias_stride_h,
+                       long long bias_stride_q, int window_left, int window_right, void* stream,
+                       int dtype) {
+  return fa_fwd_bias_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, bias, bias_stride_b,
+                        bias_stride_h, bias_stride_q, window_left, window_right, stream, dtype,
+                        nullptr, 0);
 }
 
 int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
