@@ -1104,8 +1104,10 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
           ++b_cnt;
           const uint32_t brow = (bias_mode & kBiasRowBcast) ? 0u : static_cast<uint32_t>(sub * 32 + lane);
           const uint32_t bbase = cx.sbase + G::OFF_BIAS + bs * G::BIAS_BYTES + brow * 128u;
-          // (pairs: one packed multiply-add per two keys; the key-range test only
-          // where some lane's row ends inside the block)
+          // scale * s + bias in natural-log units, one packed multiply-add per two
+          // keys (log2 e enters with the exponent's multiply-add); the key-range
+          // test only where some lane's row ends inside the block
+          const float sc_nat = c * (1.f / kLog2e);
           const bool all_visible = __all_sync(0xffffffffu, lim >= kBN);
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
@@ -1124,8 +1126,8 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
                 const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
                 bv = f2(f.x, f.y);
               }
-              const F2 x = ffma2(f2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), f2(c, c),
-                                 fmul2(bv, f2(kLog2e, kLog2e)));
+              const F2 x = ffma2(f2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
+                                 f2(sc_nat, sc_nat), bv);
               if (all_visible) {
                 sr[i] = __float_as_uint(x.x);
                 sr[i + 1] = __float_as_uint(x.y);
@@ -1159,7 +1161,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
           for (int i = 0; i < kBN; ++i)
             sr[i] = __float_as_uint((i < lim) ? __uint_as_float(sr[i]) * c : -INFINITY);
         }
-        m_blk = row_max(sr);
+        m_blk = row_max(sr) * (BIAS ? kLog2e : 1.f);  // (a bias: natural-log units)
       } else {  // max of raw scores; the scale (of either sign) is applied to the max
         m_blk = (c >= 0.f ? row_max(sr) : row_min(sr)) * c;
       }
@@ -1174,7 +1176,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
         need = true;
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      const float cs = masked ? 1.f : c;
+      const float cs = BIAS ? kLog2e : masked ? 1.f : c;
       // bf16 only: also sum the rounded P that the PV product actually uses, and
       // normalise O by that sum -- the weights then sum to one exactly, which
       // removes the bf16 rounding error of the dominant weight(s) from O.
