@@ -512,6 +512,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait_bar(B(G::B_ACC), 0u, cx.abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
+        // Every MMA has retired, so the slot ring is idle: each warp stages its 32
+        // rows there (16-byte units rotated by the row), then writes whole lines.
+        constexpr int U = D * 2 / 16;  // 16-byte units of a row
+        const uint32_t stg = sbase + G::OFF_SL + static_cast<uint32_t>(warp) * (32u * D * 2u);
+        const uint32_t srow = stg + static_cast<uint32_t>(lane) * (D * 2u);
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t a[32];
@@ -520,11 +525,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int x = 0; x < 16; ++x)
             w[x] = pack2(__uint_as_float(a[2 * x]) * mul, __uint_as_float(a[2 * x + 1]) * mul, BF16);
-          if (key < p.Nk) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
-            for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+          for (int x = 0; x < 4; ++x) {
+            const uint32_t u = static_cast<uint32_t>(c0 / 8 + x);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             srow + ((u ^ (static_cast<uint32_t>(lane) & (U - 1))) << 4)),
+                         "r"(w[4 * x]), "r"(w[4 * x + 1]), "r"(w[4 * x + 2]), "r"(w[4 * x + 3])
+                         : "memory");
           }
+        }
+        __syncwarp();
+        const int key0 = kv_row0 + (warp & 3) * 32;
+        uint16_t* out = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
+                        static_cast<size_t>(T.bkv) * p.Nk * D;
+#pragma unroll 1
+        for (int k = 0; k < U; ++k) {
+          const int rr = k * (32 / U) + lane / U, u = lane % U;
+          uint32_t w[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                       : "r"(stg + static_cast<uint32_t>(rr) * (D * 2u) +
+                             ((static_cast<uint32_t>(u) ^ (static_cast<uint32_t>(rr) & (U - 1))) << 4))
+                       : "memory");
+          if (key0 + rr < p.Nk)
+            reinterpret_cast<uint4*>(out + static_cast<size_t>(key0 + rr) * D)[u] =
+                make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
@@ -793,22 +818,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait_bar(B(G::B_DQF), 0u, cx.abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
-        uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) +
-                        (static_cast<size_t>(bh) * p.Nq + (qpos < p.Nq ? qpos : 0)) * D;
+        // The K / V slots are idle once dQ is final: each warp stages its 32 rows'
+        // half rows there (16-byte units rotated by the row), then writes lines.
+        constexpr int U = D / 16;  // 16-byte units of a half row
+        const uint32_t stg = sbase + G::OFF_SL + static_cast<uint32_t>(warp) * (32u * D);
+        const uint32_t srow = stg + static_cast<uint32_t>(lane) * D;
 #pragma unroll 1
-        for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 32) {
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
           uint32_t a[32];
-          tmem_ld_x32(tm + G::T_DQ + c0, a);
+          tmem_ld_x32(tm + G::T_DQ + h * (D / 2) + c0, a);
           uint32_t w[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x)
             w[x] = pack2(__uint_as_float(a[2 * x]) * p.scale, __uint_as_float(a[2 * x + 1]) * p.scale,
                          BF16);
-          if (qpos < p.Nq) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
-            for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+          for (int x = 0; x < 4; ++x) {
+            const uint32_t u = static_cast<uint32_t>(c0 / 8 + x);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             srow + ((u ^ (static_cast<uint32_t>(lane) & (U - 1))) << 4)),
+                         "r"(w[4 * x]), "r"(w[4 * x + 1]), "r"(w[4 * x + 2]), "r"(w[4 * x + 3])
+                         : "memory");
           }
+        }
+        __syncwarp();
+        const int q0w = q0 + (warp & 3) * 32;
+        uint16_t* out = reinterpret_cast<uint16_t*>(p.dq) + static_cast<size_t>(bh) * p.Nq * D + h * (D / 2);
+#pragma unroll 1
+        for (int k = 0; k < U; ++k) {
+          const int rr = k * (32 / U) + lane / U, u = lane % U;
+          uint32_t w[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                       : "r"(stg + static_cast<uint32_t>(rr) * D +
+                             ((static_cast<uint32_t>(u) ^ (static_cast<uint32_t>(rr) & (U - 1))) << 4))
+                       : "memory");
+          if (q0w + rr < p.Nq)
+            reinterpret_cast<uint4*>(out + static_cast<size_t>(q0w + rr) * D)[u] =
+                make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
