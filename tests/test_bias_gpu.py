@@ -196,3 +196,22 @@ def test_bias_workspace_matches_no_workspace(cuda_dev):
         fa.set_max_ctas(prev)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b_[0]) and torch.equal(a[1], b_[1])
+
+
+def test_window_and_bias_dynamic_schedule(cuda_dev):
+    # windowed bias launches (one-query-tile bias kernel) on 4 CTAs: 20 units go
+    # through the dynamic schedule's ring, with the bias tiles loaded beside K/V;
+    # the result equals the static order bit for bit
+    w = Workload("window 150 + bias D128 fp16, 4 CTAs", 1, 4, 2, 600, 600, 128, "fp16", True,
+                 seed=128)
+    b = _bias(w, (1, 4, 600, 600), 16)
+    prev = fa.set_max_ctas(4)
+    try:
+        o, lse = _check(w, b, cuda_dev, " window dynamic", window=(150, -1))
+        q, k, v = (x.to(cuda_dev) for x in make_qkv(w))
+        o2, lse2 = fa.fa_fwd(q, k, v, scale=w.softmax_scale, causal=True, window=(150, -1),
+                             bias=b.to(cuda_dev), use_workspace=False)
+    finally:
+        fa.set_max_ctas(prev)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
