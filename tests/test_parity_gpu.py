@@ -224,6 +224,16 @@ def test_scale_values(cuda_dev, scale):
                                    atol=1e-5)
 
 
+@pytest.mark.parametrize("scale", [0.0, -0.0883883])
+def test_scale_values_two_tile_kernel(cuda_dev, scale):
+    # enough 256-row tiles for the two-query-tile kernel, whose causal diagonal
+    # blocks keep fp16 scores unscaled with -inf * sign(scale) at masked keys
+    # (scale 0 takes the scaled form)
+    w = Workload("scale two-tile", 2, 40, 40, 600, 600, 128, "fp16", True, seed=6, scale=scale)
+    assert 2 * fa.num_tiles(w.B, w.Hq, w.Nq, w.D) >= 148
+    compare(w, cuda_dev)
+
+
 def test_deterministic_and_lse_optional(cuda_dev):
     w = Workload("det", 1, 4, 2, 777, 777, 128, "bf16", True, seed=5)
     (q, k, v), o1, l1 = run_cuda(w, cuda_dev)

@@ -1084,6 +1084,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
                               (p.wl >= 0 && kbase < rfirst + kBM - 1 - p.wl)
                         : (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst));
       float m_blk;
+      bool raw = false;  // masked scores left unscaled (the scale enters with the exponent)
       if (masked) {  // scaled scores, -inf where the key is outside the window or past Nk
         int lim = p.Nk - kbase;  // keys [lo, lim) of the block are visible to this row
         if constexpr (BIAS) {
@@ -1157,11 +1158,21 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
                                                                           : -INFINITY);
         } else {
           if (p.causal) lim = min(lim, row - kbase + 1);
+          // fp16: raw scores, -inf * sign(c) past the row (c enters with the
+          // exponent; bf16 keeps the scaled form, which its register budget fits)
+          if (!BF16 && c != 0.f) {
+            raw = true;
+            const uint32_t off = __float_as_uint(c > 0.f ? -INFINITY : INFINITY);
 #pragma unroll
-          for (int i = 0; i < kBN; ++i)
-            sr[i] = __float_as_uint((i < lim) ? __uint_as_float(sr[i]) * c : -INFINITY);
+            for (int i = 0; i < kBN; ++i) sr[i] = (i < lim) ? sr[i] : off;
+          } else {
+#pragma unroll
+            for (int i = 0; i < kBN; ++i)
+              sr[i] = __float_as_uint((i < lim) ? __uint_as_float(sr[i]) * c : -INFINITY);
+          }
         }
-        m_blk = row_max(sr) * (BIAS ? kLog2e : 1.f);  // (a bias: natural-log units)
+        if (raw) m_blk = (c > 0.f ? row_max(sr) : row_min(sr)) * c;
+        else m_blk = row_max(sr) * (BIAS ? kLog2e : 1.f);  // (a bias: natural-log units)
       } else {  // max of raw scores; the scale (of either sign) is applied to the max
         m_blk = (c >= 0.f ? row_max(sr) : row_min(sr)) * c;
       }
@@ -1176,7 +1187,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
         need = true;
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      const float cs = BIAS ? kLog2e : masked ? 1.f : c;
+      const float cs = BIAS ? kLog2e : (masked && !raw) ? 1.f : c;
       // bf16 only: also sum the rounded P that the PV product actually uses, and
       // normalise O by that sum -- the weights then sum to one exactly, which
       // removes the bf16 rounding error of the dominant weight(s) from O.
