@@ -482,8 +482,38 @@ def main():
             backward["causal" if w.causal else "noncausal"] = {
                 "ms": round(ms, 4), "tflops": round(bflops / (ms * 1e-3) / 1e12, 1),
                 "frac_of_peak": round(bflops / (ms * 1e-3) / 1e12 / peak, 3)}
-        backward["flops"] = "2.5 x the forward pass's (five GEMMs); three launches per call"
-        del bdo, bws, bdq, bdk, bdv
+        # the same non-causal pass with one [N, N] score bias shared by all heads
+        w = ws[0]
+        g1 = torch.Generator(device=dev).manual_seed(2)
+        bb = torch.randn((1, 1, w.Nq, w.Nk), device=dev, dtype=q.dtype, generator=g1)
+        bo, bl = fa.fa_fwd(q, k, v, scale=w.softmax_scale, bias=bb, stream=sptr)
+        ms = time_launches(lambda: fa.fa_bwd(q, k, v, bo, bl, bdo, scale=w.softmax_scale, dq=bdq,
+                                             dk=bdk, dv=bdv, stream=sptr, workspace=bws, bias=bb),
+                           flush, stream)
+        bflops = 2.5 * w.flops()
+        backward["noncausal_shared_bias"] = {
+            "ms": round(ms, 4), "tflops": round(bflops / (ms * 1e-3) / 1e12, 1),
+            "frac_of_peak": round(bflops / (ms * 1e-3) / 1e12 / peak, 3)}
+        del bdo, bws, bdq, bdk, bdv, bb
+        # head_dim 256: the GQA configuration's D = 256 variant (B4 Hq32 Hkv8 N8192 bf16 causal)
+        from fa_inputs import gqa
+        w = gqa(8, 256)
+        gq, gk, gv = (x.to(dev) for x in make_qkv(w))
+        gdo = torch.randn(gq.shape, device=dev, dtype=gq.dtype, generator=g0)
+        gws = torch.empty(fa.load_library().fa_bwd_workspace_size(*gq.shape[:3]), dtype=torch.uint8,
+                          device=dev)
+        go, gl = fa.fa_fwd(gq, gk, gv, scale=w.softmax_scale, causal=True, stream=sptr)
+        gdq, gdk, gdv = torch.empty_like(gq), torch.empty_like(gk), torch.empty_like(gv)
+        ms = time_launches(lambda: fa.fa_bwd(gq, gk, gv, go, gl, gdo, scale=w.softmax_scale,
+                                             causal=True, dq=gdq, dk=gdk, dv=gdv, stream=sptr,
+                                             workspace=gws), flush, stream, n=5, warm=2)
+        bflops = 2.5 * w.flops()
+        backward["gqa_d256_causal"] = {
+            "workload": w.name, "ms": round(ms, 4), "tflops": round(bflops / (ms * 1e-3) / 1e12, 1),
+            "frac_of_peak": round(bflops / (ms * 1e-3) / 1e12 / peak, 3)}
+        backward["flops"] = ("2.5 x the forward pass's (five GEMMs); three launches per call "
+                             "(four at head_dim 256)")
+        del gq, gk, gv, gdo, gws, go, gl, gdq, gdk, gdv
         assert fa.device_status(reset=True) == 0
 
     clk.section("bias")

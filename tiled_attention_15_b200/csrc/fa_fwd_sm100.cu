@@ -1085,12 +1085,11 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
                         : (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > rfirst));
       float m_blk;
       bool raw = false;  // masked scores left unscaled (the scale enters with the exponent)
-      if (masked) {  // scaled scores, -inf where the key is outside the window or past Nk
+      if (masked) {  // -inf where the key is outside the window or past Nk (see each branch)
         int lim = p.Nk - kbase;  // keys [lo, lim) of the block are visible to this row
         if constexpr (BIAS) {
-          // scaled score + bias * log2(e); the tile holds this row's 128 bias
-          // values as 16 swizzled 16-byte units (one row for every query when
-          // broadcast over queries)
+          // the tile holds this row's 128 bias values as 16 swizzled 16-byte
+          // units (one row for every query when broadcast over queries)
           // keys of the block before lim are visible (one query tile: the key
           // window's right bound; its left bound is applied after the bias)
           if constexpr (kWin) {
