@@ -265,6 +265,22 @@ int fa_bwd_bias(const void *q, const void *k, const void *v, const void *o, cons
                 long long bias_stride_h, long long bias_stride_q, void *stream, int dtype,
                 void *workspace, size_t workspace_bytes);
 
+/*
+ * fa_bwd_bias with a key window as well (the gradient of fa_fwd_bias_window's
+ * operation): query i sees keys i - window_left .. i + window_right (-1: no
+ * bound; causal = 1 is window_right = 0) and the bias enters P as in
+ * fa_bwd_bias; query and key blocks wholly outside the windows are skipped.
+ * A row with no visible key contributes nothing.  Arguments and errors as
+ * fa_bwd_bias and fa_bwd_window; window_left = window_right = -1 is
+ * fa_bwd_bias.
+ */
+int fa_bwd_bias_window(const void *q, const void *k, const void *v, const void *o,
+                       const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                       int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
+                       const void *bias, long long bias_stride_b, long long bias_stride_h,
+                       long long bias_stride_q, int window_left, int window_right, void *stream,
+                       int dtype, void *workspace, size_t workspace_bytes);
+
 /* Workspace bytes fa_bwd needs: 8 * B * Hq * (Nq rounded up to 128); 0 for bad sizes. */
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq);
 

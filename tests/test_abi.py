@@ -221,6 +221,21 @@ def test_bias_ws_entry_point_host_checks(lib):
         assert call() == 8 and call(ws=None) == 8 and call(wl=16, causal=1) == 8
 
 
+def test_bwd_bias_window_host_checks(lib):
+    import torch
+    a = dict(GOOD)
+
+    def call(wl=-1, wr=-1, causal=0, D=128):
+        return lib.fa_bwd_bias_window(a["q"], a["k"], a["v"], 6 * A, 7 * A, 8 * A, 9 * A, 10 * A,
+                                      11 * A, a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], D,
+                                      ctypes.c_float(a["scale"]), causal, 13 * A, 0, 0, 64, wl, wr,
+                                      None, a["dtype"], 12 * A, 1 << 20)
+    assert call(wl=-2) == 14 and call(wr=3, causal=1) == 14
+    assert call(D=256) == 5
+    if not torch.cuda.is_available():
+        assert call() == 8 and call(wl=32, causal=1) == 8 and call(wl=5, wr=7) == 8
+
+
 def test_bwd_window_host_checks(lib):
     a = dict(GOOD)
 

@@ -197,3 +197,20 @@ def test_bwd_zero_bias_equals_no_bias(cuda_dev):
         assert fa.device_status(reset=True) == 0
         for a, b in zip(plain, zero):
             assert torch.equal(a, b)
+
+
+# ---- a key window and a score bias together (fa_bwd_bias_window)
+
+@pytest.mark.parametrize("w,window,shape", [
+    (Workload("bwd window 200 causal + full bias D128 fp16", 1, 4, 2, 600, 600, 128, "fp16", True,
+              seed=161), (200, -1), (1, 4, 600, 600)),
+    (Workload("bwd window 40/20 + padding mask D64 bf16", 2, 2, 2, 333, 350, 64, "bf16", False,
+              seed=162), (40, 20), (2, 1, 1, 350)),
+], ids=lambda c: c.name if hasattr(c, "name") else str(c))
+def test_bwd_window_and_bias_parity(cuda_dev, w, window, shape):
+    bias = _bias(w, shape, w.seed + 7, neg_inf_frac=0.1)
+    inputs, got = _run(w, cuda_dev, window=window, bias=bias)
+    q, k, v, g = inputs
+    ref = oracle.attention_bwd(q, k, v, g, w.softmax_scale, w.causal, window=window,
+                               bias=bias.float())[:3]
+    _check(w, got, ref, inputs, tag=" window bias")

@@ -26,7 +26,7 @@ FA_ERR_BAD_WORKSPACE = 15
 
 # Every symbol include/fa.h declares (checked by the tests).
 EXPORTED = ("fa_fwd", "fa_fwd_fp16", "fa_fwd_bf16", "fa_fwd_ws", "fa_fwd_workspace_size",
-            "fa_fwd_window", "fa_fwd_bias", "fa_fwd_bias_window", "fa_fwd_bias_ws", "fa_bwd", "fa_bwd_window", "fa_bwd_bias",
+            "fa_fwd_window", "fa_fwd_bias", "fa_fwd_bias_window", "fa_fwd_bias_ws", "fa_bwd", "fa_bwd_window", "fa_bwd_bias", "fa_bwd_bias_window",
             "fa_bwd_workspace_size",
             "fa_fwd_noalloc", "fa_fwd_noalloc_scratch_bytes", "fa_set_max_ctas",
             "fa_fwd_unfused", "fa_fwd_unfused_workspace_size",
@@ -78,6 +78,9 @@ def load_library() -> ctypes.CDLL:
     lib.fa_bwd_bias.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, vp, ll, ll, ll, vp, i, vp,
                                            ctypes.c_size_t]
     lib.fa_bwd_bias.restype = i
+    lib.fa_bwd_bias_window.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, i, vp, ll, ll, ll, i, i, vp,
+                                                  i, vp, ctypes.c_size_t]
+    lib.fa_bwd_bias_window.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i]
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_fwd_noalloc.argtypes = fwd_args + [i]
@@ -296,7 +299,7 @@ def fa_bwd(q, k, v, o, lse, dout, scale: Optional[float] = None, causal: bool = 
     workspace: a uint8 CUDA tensor of at least fa_bwd_workspace_size bytes
     (allocated here when None).  window: (left, right) key window of the
     forward pass (fa_bwd_window), -1 = unbounded.  bias: the forward pass's
-    additive score bias (fa_bwd_bias; as in fa_fwd, not with a window).
+    additive score bias (fa_bwd_bias_window, with or without a window).
     Returns (dq, dk, dv).
     """
     import torch
@@ -334,14 +337,12 @@ def fa_bwd(q, k, v, o, lse, dout, scale: Optional[float] = None, causal: bool = 
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
             lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
     if bias is not None:
-        if (wl, wr) != (-1, -1):
-            raise ValueError("the backward pass takes a bias or a key window, not both")
         bt, sb, sh, sq = _bias_view(bias, q.dtype, B, Hq, Nq, Nk)
-        rc = lib.fa_bwd_bias(*ptrs, B, Hq, Hkv, Nq, Nk, D, ctypes.c_float(scale),
-                             1 if causal else 0, bt.data_ptr(), sb, sh, sq, stream or None, dtype,
-                             workspace.data_ptr(), workspace.numel())
+        rc = lib.fa_bwd_bias_window(*ptrs, B, Hq, Hkv, Nq, Nk, D, ctypes.c_float(scale),
+                                    1 if causal else 0, bt.data_ptr(), sb, sh, sq, wl, wr,
+                                    stream or None, dtype, workspace.data_ptr(), workspace.numel())
         if rc != FA_OK:
-            raise FaError(rc, "fa_bwd_bias")
+            raise FaError(rc, "fa_bwd_bias_window")
         return dq, dk, dv
     rc = lib.fa_bwd_window(*ptrs, B, Hq, Hkv, Nq, Nk, D, ctypes.c_float(scale), 1 if causal else 0,
                            wl, wr, stream or None, dtype, workspace.data_ptr(), workspace.numel())

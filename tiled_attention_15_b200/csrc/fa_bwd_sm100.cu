@@ -1695,19 +1695,30 @@ int fa_bwd_window(const void* q, const void* k, const void* v, const void* o, co
                   window_left, window_right, stream, dtype, workspace, workspace_bytes, nullptr);
 }
 
-int fa_bwd_bias(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
-                int Nk, int D, float scale, int causal, const void* bias, long long bias_stride_b,
-                long long bias_stride_h, long long bias_stride_q, void* stream, int dtype,
-                void* workspace, size_t workspace_bytes) {
+int fa_bwd_bias_window(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
+                       const void* bias, long long bias_stride_b, long long bias_stride_h,
+                       long long bias_stride_q, int window_left, int window_right, void* stream,
+                       int dtype, void* workspace, size_t workspace_bytes) {
   if (bias == nullptr) return FA_ERR_NULL_POINTER;
   if (bias_stride_b < 0 || bias_stride_h < 0 || bias_stride_q < 0) return FA_ERR_BAD_SHAPE;
   if ((reinterpret_cast<uintptr_t>(bias) & 15u) || (bias_stride_b & 7) || (bias_stride_h & 7) ||
       (bias_stride_q & 7))
     return FA_ERR_MISALIGNED;
   const BiasArgB a{bias, bias_stride_b, bias_stride_h, bias_stride_q};
-  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, D, scale, causal, -1, -1,
-                  stream, dtype, workspace, workspace_bytes, &a);
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                  window_left, window_right, stream, dtype, workspace, workspace_bytes, &a);
+}
+
+int fa_bwd_bias(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                int Nk, int D, float scale, int causal, const void* bias, long long bias_stride_b,
+                long long bias_stride_h, long long bias_stride_q, void* stream, int dtype,
+                void* workspace, size_t workspace_bytes) {
+  return fa_bwd_bias_window(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                            bias, bias_stride_b, bias_stride_h, bias_stride_q, -1, -1, stream,
+                            dtype, workspace, workspace_bytes);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
