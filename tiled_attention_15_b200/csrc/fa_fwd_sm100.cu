@@ -95,8 +95,15 @@ struct Geometry {
   // ... then this CTA's stream-K unit range (2 x s32), then per query tile the
   // split-merge verdict (2 x s32: 1 = this CTA merges the tile)
   static constexpr int SMEM_BYTES = OFF_MISC + 8 + 4 * kTileRing + 8 + 8 + 1024;  // + alignment slack
+  // The staged epilogue (two query tiles, no score bias; an instantiation of its
+  // own) adds per softmax warp a 4 KB area, 32 rows x 64 columns of 16-bit output,
+  // after everything else.  (Not in every kernel: with it a CTA takes the largest
+  // shared-memory carveout, which leaves the L1 cache half the room.)
+  static constexpr int OFF_STAGE = (OFF_MISC + 8 + 4 * kTileRing + 8 + 8 + 1023) & ~1023;
+  static constexpr int SMEM_BYTES_STAGED = OFF_STAGE + 8 * 4096 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(NQ == 1 || BIAS || SMEM_BYTES_STAGED <= 232448, "shared memory budget (staged)");
   static_assert(NQ == 2 ? (256 + 2 * D <= 512) : (256 + D <= 512), "tensor memory budget");
 };
 
@@ -1037,7 +1044,7 @@ __device__ __forceinline__ void merge_epilogue_rows(const FwdParams& p, const Ti
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
-template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false>
+template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false, bool STG = false>
 __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, int wg, int sub,
                                              int lane, int bias_mode) {
   using G = Geometry<D, NQ, BIAS>;
@@ -1059,9 +1066,9 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     int nblk, rfirst, jb;
     {
       const Tile T0 = get_tile<NQ, WIN>(p, t);
-      nblk = T0.nblk[q];
+      nblk = q ? T0.nblk[1] : T0.nblk[0];  // (selects keep the tile off the stack)
       rfirst = T0.row0 + q * kBM;
-      jb = WIN ? T0.jb + T0.j0[q] : T0.jb;
+      jb = WIN ? T0.jb + (q ? T0.j0[1] : T0.j0[0]) : T0.jb;
     }
     if (nblk == 0) continue;
     // query position of this thread's row (causal mask; packing is non-causal only)
@@ -1069,9 +1076,11 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
     float m_used = -INFINITY, l = 0.f, l_r = 0.f;  // l: exact sum (LSE); l_r: rounded-P sum
     for (int j = 0; j < nblk; ++j) {
       const int sb = (NQ == 2) ? q : (j & 1);
-      bool ok = wait_bar(B(G::B_SFULL + sb), s_phase[sb], cx.abort_flag);
+      // (selects, not s_phase[sb]: a runtime index would put the array on the stack)
+      bool ok = wait_bar(B(G::B_SFULL + sb), sb ? s_phase[1] : s_phase[0], cx.abort_flag);
       if (!__all_sync(0xffffffffu, ok)) return;
-      s_phase[sb] ^= 1u;
+      if (sb) s_phase[1] ^= 1u;
+      else s_phase[0] ^= 1u;
       tc_fence_after();
       uint32_t sr[kBN];
       tmem_ld_x128(tm + sb * 128, sr);
@@ -1266,6 +1275,51 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
       // softmax: O = 0, LSE = -inf
       const bool empty = (kWin || BIAS) && m_used == -INFINITY;
       const float inv_l = empty ? 0.f : 1.f / (BF16 ? l_r : l);
+      if constexpr (STG) {
+        // Each 64-column half goes through the warp's staging area: the thread's
+        // own row in (16-byte units rotated by row, so neither direction has bank
+        // conflicts), then each store instruction writes four whole 128-byte row
+        // segments instead of 32 scattered 16-byte pieces.  (The staging address
+        // is an opaque copy: hoisted out of the unit loop it would hold a
+        // register through the key loop.)
+        uint32_t stg;
+        asm volatile("mov.b32 %0, %1;"
+                     : "=r"(stg)
+                     : "r"(cx.sbase + G::OFF_STAGE + static_cast<uint32_t>(wg * 4 + sub) * 4096u));
+        const unsigned orow = live ? static_cast<unsigned>(ri.out_row) : 0xffffffffu;
+        const uint32_t cu = static_cast<uint32_t>(lane & 7);
+#pragma unroll 1
+        for (int h = 0; h < D / 64; ++h) {
+#pragma unroll 1
+          for (int u0 = 0; u0 < 8; u0 += 4) {
+            uint32_t orr[32];
+            tmem_ld_x32(tm + 256 + q * D + h * 64 + u0 * 8, orr);
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
+              const uint32_t u = static_cast<uint32_t>(u0 + uu);
+              uint32_t w[4];
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                w[x] = pack2(__uint_as_float(orr[8 * uu + 2 * x]) * inv_l,
+                             __uint_as_float(orr[8 * uu + 2 * x + 1]) * inv_l, BF16);
+              st_shared_v4(stg + static_cast<uint32_t>(lane) * 128u + ((u ^ (lane & 7u)) << 4), w);
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t r = static_cast<uint32_t>(4 * k + (lane >> 3));
+            uint32_t w[4];
+            ld_shared_v4(stg + r * 128u + ((cu ^ (r & 7u)) << 4), w);
+            const unsigned dst_row = __shfl_sync(0xffffffffu, orow, static_cast<int>(r));
+            if (dst_row != 0xffffffffu)
+              reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
+                                       static_cast<size_t>(dst_row) * D + h * 64)[cu] =
+                  make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          __syncwarp();
+        }
+      } else {
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ri.out_row * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -1283,6 +1337,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
             dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
         }
       }
+      }
       if (p.lse != nullptr && live)
         p.lse[ri.out_row] = empty ? -INFINITY : (m_sub + log2f(l)) * kLn2;
     }
@@ -1292,7 +1347,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& cx, const FwdParams& p, 
   }
 }
 
-template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false>
+template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false, bool STG = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q4,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -1372,7 +1427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   else setmaxnreg_dec<kOtherRegs>();
   if (warp < 8) {
     if (NQ == 2 || warp < 4)
-      role_softmax<D, NQ, BF16, BIAS, WIN>(cx, p, warp >> 2, warp & 3, lane, bias_mode);
+      role_softmax<D, NQ, BF16, BIAS, WIN, STG>(cx, p, warp >> 2, warp & 3, lane, bias_mode);
   } else if (warp == 8) {
     if (lane == 0) role_mma<D, NQ, BF16, BIAS, WIN>(cx, p);
   } else if (warp == 9) {
@@ -1458,6 +1513,10 @@ EncodeTiledFn encode_fn() {
 }
 
 constexpr int kMaxDevices = 64;
+// Longest key range that takes the staged epilogue (32 key blocks): past it the
+// epilogue is a small share of a tile and the larger shared-memory footprint
+// costs more than the whole-line stores save.
+constexpr int kStagedMaxKeys = 32 * fa::kBN;
 struct DeviceState {
   std::once_flag once;
   int sms = 0;
@@ -1548,19 +1607,20 @@ bool make_bias_map(CUtensorMap* m, const BiasArg& a, int B, int H, int Nq, int N
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false>
+template <int D, int NQ, bool BF16, bool BIAS = false, bool WIN = false, bool STG = false>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
            int Hkv, int Nq, int Nk, float scale, int causal, int wl, int wr, cudaStream_t stream,
            int dev, void* ws, size_t ws_bytes, Scratch mode, const BiasArg* bias = nullptr) {
   using G = fa::Geometry<D, NQ, BIAS>;
+  static_assert(!STG || (NQ == 2 && !BIAS), "the staged epilogue: two query tiles, no bias");
+  constexpr int kSmem = STG ? G::SMEM_BYTES_STAGED : G::SMEM_BYTES;
   static bool attr_done[kMaxDevices] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     if (!attr_done[dev]) {
-      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, NQ, BF16, BIAS, WIN>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               G::SMEM_BYTES) != cudaSuccess)
+      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, NQ, BF16, BIAS, WIN, STG>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
         return FA_ERR_LAUNCH;
       attr_done[dev] = true;
     }
@@ -1681,7 +1741,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     bias_mode = (bias->sq ? 0 : fa::kBiasRowBcast) | (bias->sh ? fa::kBiasPerHead : 0) |
                 (bias->sb ? fa::kBiasPerBatch : 0);
   }
-  fa::fa_fwd_kernel<D, NQ, BF16, BIAS, WIN><<<grid, fa::kThreads, G::SMEM_BYTES, stream>>>(
+  fa::fa_fwd_kernel<D, NQ, BF16, BIAS, WIN, STG><<<grid, fa::kThreads, kSmem, stream>>>(
       tq, tq4, tk, tv, p, tb, bias_mode);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
@@ -1822,6 +1882,10 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
       return bf ? launch<64, 2, true>(FA_ARGS) : launch<64, 2, false>(FA_ARGS);
     case 128:
       if (one_tile) return bf ? launch<128, 1, true>(FA_ARGS) : launch<128, 1, false>(FA_ARGS);
+      // fp16 without a mask, rows of at most kStagedMaxKeys keys: the staged
+      // epilogue (output written as whole lines; the epilogue is a larger share
+      // of such a short tile)
+      if (!bf && !causal && Nk <= kStagedMaxKeys) return launch<128, 2, false, false, false, true>(FA_ARGS);
       return bf ? launch<128, 2, true>(FA_ARGS) : launch<128, 2, false>(FA_ARGS);
     default:
       return bf ? launch<256, 1, true>(FA_ARGS) : launch<256, 1, false>(FA_ARGS);
