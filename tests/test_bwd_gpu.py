@@ -214,3 +214,34 @@ def test_bwd_window_and_bias_parity(cuda_dev, w, window, shape):
     ref = oracle.attention_bwd(q, k, v, g, w.softmax_scale, w.causal, window=window,
                                bias=bias.float())[:3]
     _check(w, got, ref, inputs, tag=" window bias")
+
+
+# ---- the persistent kernels: more tiles than SMs, so a CTA takes several
+
+MANY = [
+    # causal over 256 keys: tiles of one and two query blocks (a short tile's
+    # staging gate is still pending when the next tile's items are issued)
+    (Workload("bwd many tiles D128 fp16 causal", 4, 40, 40, 256, 256, 128, "fp16", True, seed=171),
+     (-1, -1), None),
+    # causal with Nk > Nq: key tiles no query sees (zeros) between the others
+    (Workload("bwd many tiles D128 bf16 causal Nk>Nq GQA", 4, 40, 20, 256, 512, 128, "bf16", True,
+              seed=172), (-1, -1), None),
+    (Workload("bwd many tiles D64 fp16", 3, 40, 40, 384, 384, 64, "fp16", False, seed=173), (-1, -1), None),
+    (Workload("bwd many tiles D128 fp16 window", 2, 40, 20, 640, 640, 128, "fp16", False, seed=174),
+     (100, 50), None),
+    (Workload("bwd many tiles D128 fp16 bias", 2, 40, 40, 256, 300, 128, "fp16", False, seed=175),
+     (-1, -1), (1, 1, 256, 300)),
+]
+
+
+@pytest.mark.parametrize("w,window,shape", MANY, ids=lambda c: c.name if hasattr(c, "name") else str(c))
+def test_bwd_many_tiles_per_cta(cuda_dev, w, window, shape):
+    kv_tiles = w.B * w.Hkv * -(-w.Nk // 128)
+    q_tiles = w.B * w.Hq * -(-w.Nq // 128)
+    assert min(kv_tiles, q_tiles) > 148
+    bias = _bias(w, shape, w.seed + 7, neg_inf_frac=0.05) if shape is not None else None
+    inputs, got = _run(w, cuda_dev, window=window, bias=bias)
+    q, k, v, g = inputs
+    ref = oracle.attention_bwd(q, k, v, g, w.softmax_scale, w.causal, window=window,
+                               bias=None if bias is None else bias.float())[:3]
+    _check(w, got, ref, inputs, tag=" many tiles")

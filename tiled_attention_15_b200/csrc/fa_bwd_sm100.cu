@@ -16,12 +16,14 @@
 //   * bwd_prep_kernel: Delta = rowsum(dO * O) and LSE * log2(e), into two planes
 //     padded to whole 128-row blocks (+inf / 0 in the padding, which zeroes P
 //     there without a mask);
-//   * bwd_dkdv_kernel: one 128-key tile per CTA; loops over the query blocks of
+//   * bwd_dkdv_kernel: per 128-key tile, a loop over the query blocks of
 //     every query head of its GQA group: S^T = K Q^T, dP^T = V dO^T,
 //     P^T and dS^T (16-bit, written back over S^T and dP^T), dV += P^T dO,
 //     dK += dS^T Q;
-//   * bwd_dq_kernel: one 128-query tile per CTA; loops over the key blocks:
+//   * bwd_dq_kernel: per 128-query tile, a loop over the key blocks:
 //     S = Q K^T, dP = dO V^T, dS, dQ += dS K.
+// Both are persistent (one CTA per SM, tiles in a snake order): a tile's
+// loads and first MMAs overlap the previous tile's epilogue.
 // dQ is computed in its own pass (S and dP recomputed: two extra MMAs per block
 // pair) instead of being accumulated across key tiles with atomics: no atomic
 // traffic, and the result does not depend on the order CTAs finish in.
@@ -224,10 +226,13 @@ struct GeoKV {
   static constexpr int OFF_K = 0, OFF_V = T_BYTES, OFF_SL = 2 * T_BYTES;
   static constexpr int OFF_BIAS = OFF_SL + NSLOT * SLOT_BYTES;  // the block pair's bias tile
   static constexpr int OFF_BAR = OFF_BIAS + (BIAS ? kBiasTileBytes : 0);
-  // barriers
+  // barriers (the kernel is persistent: B_KVE = the tile's K and V no longer
+  // read, B_ACCE = its dV and dK read out of tensor memory, B_STG = its
+  // epilogue done with the staging slots)
   static constexpr int B_KV = 0, B_SLF = 1, B_SLE = 1 + NSLOT, B_SF = 1 + 2 * NSLOT,
                        B_DPF = B_SF + 1, B_PF = B_SF + 2, B_DSF = B_SF + 3, B_ACC = B_SF + 4,
-                       B_BF = B_SF + 5, B_BE = B_SF + 6, NBAR = B_SF + 7;
+                       B_BF = B_SF + 5, B_BE = B_SF + 6, B_KVE = B_SF + 7, B_ACCE = B_SF + 8,
+                       B_STG = B_SF + 9, NBAR = B_SF + 10;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // TMEM columns: S^T 0..127 (P^T over it), dP^T 128..255 (dS^T over it), dV, dK
@@ -244,11 +249,16 @@ struct KVTile {
   int nb;   // blocks: group heads x query blocks
 };
 
-// bq: rows of a query block (128, or 64 at head_dim 256)
-__device__ __forceinline__ KVTile kv_tile(const BwdParams& p, int bq = kBM) {
+// The tile a persistent CTA takes in round r (snake order over the grid).
+__device__ __forceinline__ int snake_tile(int r) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return r * G + ((r & 1) ? G - 1 - c : c);
+}
+
+// tile t; bq: rows of a query block (128, or 64 at head_dim 256)
+__device__ __forceinline__ KVTile kv_tile(const BwdParams& p, int t, int bq = kBM) {
   KVTile T;
   const int BK = p.B * p.Hkv;
-  const int t = blockIdx.x;
   if (p.causal) {  // small key blocks see the most query blocks: run them first
     T.kt = t / BK;
     T.bkv = t % BK;
@@ -266,6 +276,18 @@ __device__ __forceinline__ KVTile kv_tile(const BwdParams& p, int bq = kBM) {
   return T;
 }
 
+// Persistent: in round r CTA c takes tile r G + c (r even) or r G + G - 1 - c
+// (r odd), G = gridDim.x -- the tiles come heaviest first (causal), so the
+// snake order evens out each CTA's sum.  Ring items, block
+// indices and tile indices run on across tiles (the barrier phases follow
+// them), so the next tile's K, V and first Q / dO blocks load, and its first
+// S^T and dP^T run, while the compute warps write the previous tile's dK, dV.
+// The epilogue stages its rows in the two slots the next tile's ring items
+// reach last (items M + NSLOT - 2 and M + NSLOT - 1, M = the first item after
+// the tile): they held the tile's own last Q and dO, so they are idle once its
+// accumulators are final, and the TMA thread loads into them only after
+// B_STG.  Tiles no query sees (key windows) write zeros and take no part in
+// the barriers.
 template <int D, bool BF16, bool BIAS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -282,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   cx.sbase = sbase;
   cx.abort_flag = misc + 1;
   auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
-  const KVTile T = kv_tile(p);
+  const int n_tiles = p.B * p.Hkv * p.nkt;
 
   if (threadIdx.x == 0) {
     mbar_init(B(G::B_KV), 1);
@@ -297,6 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(B(G::B_ACC), 1);
     mbar_init(B(G::B_BF), 1);
     mbar_init(B(G::B_BE), 8);
+    mbar_init(B(G::B_KVE), 1);
+    mbar_init(B(G::B_ACCE), 8);
+    mbar_init(B(G::B_STG), 8);
     misc[1] = 0u;
     fence_mbar_init();
   }
@@ -311,102 +336,152 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Registers: 208 for the two compute warpgroups, 88 for the rest (2 x 128 x
   // 208 + 128 x 88 = 384 x 168); each role branch sets its own limit.
-  const int kv_row0 = T.kt * kBN;
   if (warp >= 8) setmaxnreg_dec<88>();
-  if (warp == 9 && lane == 0 && T.nb > 0) {
-    // ---- TMA: K and V tiles once, then (Q, dO, lse2, delta) per query block
+  if (warp == 9 && lane == 0) {
+    // ---- TMA: per tile K and V, then (Q, dO, lse2, delta) per query block
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_do);
     const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
-    mbar_arrive_expect_tx(B(G::B_KV), 2 * G::T_BYTES);
+    uint32_t m0 = 0;                    // ring items issued before this tile
+    uint32_t gate = 0xffffffffu;        // first item that must wait for an epilogue's staging
+    uint32_t gate_par = 0;              // ... and that epilogue's B_STG phase
+    int it = 0;                         // tiles with blocks before this one
+    bool ok = true;
+    for (int rd = 0; ok && rd * static_cast<int>(gridDim.x) < n_tiles; ++rd) {
+      const int t = snake_tile(rd);
+      if (t >= n_tiles) continue;
+      const KVTile T = kv_tile(p, t);
+      if (T.nb == 0) continue;
+      if (it > 0 && !wait_bar(B(G::B_KVE), (it - 1) & 1u, cx.abort_flag)) break;
+      const int kv_row0 = T.kt * kBN;
+      mbar_arrive_expect_tx(B(G::B_KV), 2 * G::T_BYTES);
 #pragma unroll
-    for (int c = 0; c < G::DCH; ++c) {
-      tma_load_3d(sbase + G::OFF_K + c * G::CHUNK, &tm_k, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
-      tma_load_3d(sbase + G::OFF_V + c * G::CHUNK, &tm_v, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
-    }
-    const int nqb = T.nqb;
-    for (int m = 0; m < 2 * T.nb; ++m) {  // item m: Q (even, + lse2, delta) or dO (odd) of block m / 2
-      const int sl = m % G::NSLOT, n = m >> 1;
-      if (m >= G::NSLOT && !wait_bar(B(G::B_SLE + sl), ((m / G::NSLOT) - 1) & 1u, cx.abort_flag))
-        break;
-      const int h = n / nqb, i = T.i0 + n % nqb;
-      const int bh = (T.bkv / p.Hkv) * p.Hq + (T.bkv % p.Hkv) * p.group + h;
-      const uint32_t sb = sbase + G::OFF_SL + sl * G::SLOT_BYTES;
-      mbar_arrive_expect_tx(B(G::B_SLF + sl), G::T_BYTES + ((m & 1) ? 0 : 1024));
-#pragma unroll
-      for (int c = 0; c < G::DCH; ++c)
-        tma_load_3d(sb + c * G::CHUNK, (m & 1) ? &tm_do : &tm_q, B(G::B_SLF + sl), c * 64, i * kBM,
-                    bh, pol_last);
-      if ((m & 1) == 0) {
-        const size_t row = static_cast<size_t>(bh) * p.Nq_pad + static_cast<size_t>(i) * kBM;
-        bulk_load(sb + G::T_BYTES, p.lse2 + row, 512, B(G::B_SLF + sl));
-        bulk_load(sb + G::T_BYTES + 512, p.delta + row, 512, B(G::B_SLF + sl));
+      for (int c = 0; c < G::DCH; ++c) {
+        tma_load_3d(sbase + G::OFF_K + c * G::CHUNK, &tm_k, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
+        tma_load_3d(sbase + G::OFF_V + c * G::CHUNK, &tm_v, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
       }
+      const int nqb = T.nqb;
+      for (int mm = 0; mm < 2 * T.nb; ++mm) {  // item mm: Q (even, + lse2, delta) or dO (odd) of block mm / 2
+        const uint32_t m = m0 + static_cast<uint32_t>(mm);
+        if (m == gate && !wait_bar(B(G::B_STG), gate_par, cx.abort_flag)) { ok = false; break; }
+        const int sl = static_cast<int>(m % G::NSLOT), n = mm >> 1;
+        if (m >= (uint32_t)G::NSLOT &&
+            !wait_bar(B(G::B_SLE + sl), ((m / G::NSLOT) - 1) & 1u, cx.abort_flag)) { ok = false; break; }
+        const int h = n / nqb, i = T.i0 + n % nqb;
+        const int bh = (T.bkv / p.Hkv) * p.Hq + (T.bkv % p.Hkv) * p.group + h;
+        const uint32_t sb = sbase + G::OFF_SL + sl * G::SLOT_BYTES;
+        mbar_arrive_expect_tx(B(G::B_SLF + sl), G::T_BYTES + ((mm & 1) ? 0 : 1024));
+#pragma unroll
+        for (int c = 0; c < G::DCH; ++c)
+          tma_load_3d(sb + c * G::CHUNK, (mm & 1) ? &tm_do : &tm_q, B(G::B_SLF + sl), c * 64, i * kBM,
+                      bh, pol_last);
+        if ((mm & 1) == 0) {
+          const size_t row = static_cast<size_t>(bh) * p.Nq_pad + static_cast<size_t>(i) * kBM;
+          bulk_load(sb + G::T_BYTES, p.lse2 + row, 512, B(G::B_SLF + sl));
+          bulk_load(sb + G::T_BYTES + 512, p.delta + row, 512, B(G::B_SLF + sl));
+        }
+      }
+      if (!ok) break;
+      m0 += 2u * static_cast<uint32_t>(T.nb);
+      // a previous epilogue's gate not reached by this tile's items (short
+      // tiles): wait for it here, before this tile's gate replaces it
+      if (gate != 0xffffffffu && gate >= m0 && !wait_bar(B(G::B_STG), gate_par, cx.abort_flag)) break;
+      gate = m0 + G::NSLOT - 2;
+      gate_par = static_cast<uint32_t>(it) & 1u;
+      ++it;
     }
-  } else if (BIAS && warp == 10 && lane == 0 && T.nb > 0) {
+  } else if (BIAS && warp == 10 && lane == 0) {
     // ---- TMA: the bias tile of each (query block, key tile) pair: rows = the
     // block's queries (one row if broadcast over queries), columns = the tile's keys
     const uint64_t pol = policy_evict_last();
     const int rows = (bias_mode & kBiasRowBcast) ? 1 : kBM;
-    const int b = T.bkv / p.Hkv;
-    for (int n = 0; n < T.nb; ++n) {
-      if (n > 0 && !wait_bar(B(G::B_BE), (n - 1) & 1u, cx.abort_flag)) break;
-      const int hq = (T.bkv % p.Hkv) * p.group + n / T.nqb, i = T.i0 + n % T.nqb;
-      mbar_arrive_expect_tx(B(G::B_BF), 2 * rows * 128);
+    uint32_t g0 = 0;  // blocks before this tile
+    bool ok = true;
+    for (int rd = 0; ok && rd * static_cast<int>(gridDim.x) < n_tiles; ++rd) {
+      const int t = snake_tile(rd);
+      if (t >= n_tiles) continue;
+      const KVTile T = kv_tile(p, t);
+      if (T.nb == 0) continue;
+      const int b = T.bkv / p.Hkv, kv_row0 = T.kt * kBN;
+      for (int n = 0; n < T.nb; ++n) {
+        const uint32_t g = g0 + static_cast<uint32_t>(n);
+        if (g > 0 && !wait_bar(B(G::B_BE), (g - 1) & 1u, cx.abort_flag)) { ok = false; break; }
+        const int hq = (T.bkv % p.Hkv) * p.group + n / T.nqb, i = T.i0 + n % T.nqb;
+        mbar_arrive_expect_tx(B(G::B_BF), 2 * rows * 128);
 #pragma unroll
-      for (int box = 0; box < 2; ++box)
-        tma_load_4d(sbase + G::OFF_BIAS + box * (kBiasTileBytes / 2), &tm_b, B(G::B_BF),
-                    kv_row0 + box * 64, (bias_mode & kBiasRowBcast) ? 0 : i * kBM,
-                    (bias_mode & kBiasPerHead) ? hq : 0, (bias_mode & kBiasPerBatch) ? b : 0, pol);
+        for (int box = 0; box < 2; ++box)
+          tma_load_4d(sbase + G::OFF_BIAS + box * (kBiasTileBytes / 2), &tm_b, B(G::B_BF),
+                      kv_row0 + box * 64, (bias_mode & kBiasRowBcast) ? 0 : i * kBM,
+                      (bias_mode & kBiasPerHead) ? hq : 0, (bias_mode & kBiasPerBatch) ? b : 0, pol);
+      }
+      g0 += static_cast<uint32_t>(T.nb);
     }
-  } else if (warp == 8 && lane == 0 && T.nb > 0) {
-    // ---- MMA: S(0) dP(0) | dV(n) S(n+1) dK(n) dP(n+1) | ...
+  } else if (warp == 8 && lane == 0) {
+    // ---- MMA, per tile: S(0) dP(0) | dV(n) S(n+1) dK(n) dP(n+1) | ...
     constexpr uint32_t kIdNT = idesc_f16(128, 128, BF16, false);
     constexpr uint32_t kIdTN = idesc_f16(128, D, BF16, true);
     const uint32_t tm = cx.tmem;
     const uint64_t dk0 = sdesc_sw128(sbase + G::OFF_K, 16, 1024);
     const uint64_t dv0 = sdesc_sw128(sbase + G::OFF_V, 16, 1024);
-    auto st_desc = [&](int m, bool mn) {  // ring item m: Q_{m/2} (even) or dO_{m/2} (odd)
+    auto st_desc = [&](uint32_t m, bool mn) {  // ring item m: a Q (even) or dO (odd) block
       const uint32_t a = sbase + G::OFF_SL + (m % G::NSLOT) * G::SLOT_BYTES;
       return mn ? sdesc_sw128(a, G::CHUNK, 1024) : sdesc_sw128(a, 16, 1024);
     };
-    auto wait_item = [&](int m) {
+    auto wait_item = [&](uint32_t m) {
       return wait_bar(B(G::B_SLF + m % G::NSLOT), (m / G::NSLOT) & 1u, cx.abort_flag);
     };
     // P^T / dS^T of query column q: warpgroup q / 64 packed its half at its own
     // first 32 columns -> K step kk (16 queries) at (kk / 4) * 64 + (kk % 4) * 8
     auto acol = [](int kk) { return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8); };
-    bool ok = wait_bar(B(G::B_KV), 0u, cx.abort_flag) && wait_item(0) && wait_item(1);
-    if (ok) {
+    uint32_t m0 = 0, g0 = 0;
+    int it = 0;
+    bool ok = true;
+    for (int rd = 0; ok && rd * static_cast<int>(gridDim.x) < n_tiles; ++rd) {
+      const int t = snake_tile(rd);
+      if (t >= n_tiles) continue;
+      const KVTile T = kv_tile(p, t);
+      if (T.nb == 0) continue;
+      ok = wait_bar(B(G::B_KV), static_cast<uint32_t>(it) & 1u, cx.abort_flag) && wait_item(m0) &&
+           wait_item(m0 + 1);
+      if (!ok) break;
       tc_fence_after();
-      mma_nt<D>(tm + G::T_S, dk0, st_desc(0, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_nt<D>(tm + G::T_S, dk0, st_desc(m0, false), kIdNT, G::CHUNK, G::CHUNK);
       mma_commit(B(G::B_SF));
-      mma_nt<D>(tm + G::T_DP, dv0, st_desc(1, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_nt<D>(tm + G::T_DP, dv0, st_desc(m0 + 1, false), kIdNT, G::CHUNK, G::CHUNK);
       mma_commit(B(G::B_DPF));
-    }
-    for (int n = 0; ok && n < T.nb; ++n) {
-      if (!wait_bar(B(G::B_PF), n & 1u, cx.abort_flag)) break;
-      tc_fence_after();
-      mma_tn<D>(tm + G::T_DV, tm + G::T_S, st_desc(2 * n + 1, true), kIdTN, n > 0, acol);
-      mma_commit(B(G::B_SLE + (2 * n + 1) % G::NSLOT));  // dO_n's slot
-      if (n + 1 < T.nb) {
-        if (!wait_item(2 * n + 2)) break;
+      if (T.nb == 1) mma_commit(B(G::B_KVE));
+      for (int n = 0; n < T.nb; ++n) {
+        const uint32_t g = g0 + static_cast<uint32_t>(n), m = m0 + 2u * static_cast<uint32_t>(n);
+        if (!wait_bar(B(G::B_PF), g & 1u, cx.abort_flag)) { ok = false; break; }
+        // the first dV of a tile overwrites the accumulators: the previous
+        // tile's epilogue must have read them out
+        if (n == 0 && it > 0 && !wait_bar(B(G::B_ACCE), (it - 1) & 1u, cx.abort_flag)) { ok = false; break; }
         tc_fence_after();
-        mma_nt<D>(tm + G::T_S, dk0, st_desc(2 * n + 2, false), kIdNT, G::CHUNK, G::CHUNK);
-        mma_commit(B(G::B_SF));
-      }
-      if (!wait_bar(B(G::B_DSF), n & 1u, cx.abort_flag)) break;
-      tc_fence_after();
-      mma_tn<D>(tm + G::T_DK, tm + G::T_DP, st_desc(2 * n, true), kIdTN, n > 0, acol);
-      mma_commit(B(G::B_SLE + (2 * n) % G::NSLOT));  // Q_n's slot (and its lse2, delta)
-      if (n + 1 < T.nb) {
-        if (!wait_item(2 * n + 3)) break;
+        mma_tn<D>(tm + G::T_DV, tm + G::T_S, st_desc(m + 1, true), kIdTN, n > 0, acol);
+        mma_commit(B(G::B_SLE + (m + 1) % G::NSLOT));  // dO_n's slot
+        if (n + 1 < T.nb) {
+          if (!wait_item(m + 2)) { ok = false; break; }
+          tc_fence_after();
+          mma_nt<D>(tm + G::T_S, dk0, st_desc(m + 2, false), kIdNT, G::CHUNK, G::CHUNK);
+          mma_commit(B(G::B_SF));
+        }
+        if (!wait_bar(B(G::B_DSF), g & 1u, cx.abort_flag)) { ok = false; break; }
         tc_fence_after();
-        mma_nt<D>(tm + G::T_DP, dv0, st_desc(2 * n + 3, false), kIdNT, G::CHUNK, G::CHUNK);
-        mma_commit(B(G::B_DPF));
-      } else {
-        mma_commit(B(G::B_ACC));
+        mma_tn<D>(tm + G::T_DK, tm + G::T_DP, st_desc(m, true), kIdTN, n > 0, acol);
+        mma_commit(B(G::B_SLE + m % G::NSLOT));  // Q_n's slot (and its lse2, delta)
+        if (n + 1 < T.nb) {
+          if (!wait_item(m + 3)) { ok = false; break; }
+          tc_fence_after();
+          mma_nt<D>(tm + G::T_DP, dv0, st_desc(m + 3, false), kIdNT, G::CHUNK, G::CHUNK);
+          mma_commit(B(G::B_DPF));
+          if (n + 2 == T.nb) mma_commit(B(G::B_KVE));  // the tile's last read of K and V
+        } else {
+          mma_commit(B(G::B_ACC));
+        }
       }
+      m0 += 2u * static_cast<uint32_t>(T.nb);
+      g0 += static_cast<uint32_t>(T.nb);
+      ++it;
     }
   } else if (warp < 8) {
     // ---- compute: thread = key row r of the tile, warpgroup h = query columns h*64 .. +63
@@ -414,144 +489,164 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2, r = (warp & 3) * 32 + lane;
     const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.c;
-    const int nqb = T.nqb;
+    uint32_t m0 = 0, g0 = 0;
+    int it = 0;
     bool ok = true;
-    for (int n = 0; ok && n < T.nb; ++n) {
-      const int sl = (2 * n) % G::NSLOT;  // the slot of Q_n, with lse2 and delta
-      const int i = T.i0 + n % nqb;
-      // lse2 / delta of this block were written by the TMA unit: observe its barrier
-      ok = wait_bar(B(G::B_SLF + sl), ((2 * n) / G::NSLOT) & 1u, cx.abort_flag) &&
-           wait_bar(B(G::B_SF), n & 1u, cx.abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      const float* l2 = reinterpret_cast<const float*>(gbase + G::OFF_SL + sl * G::SLOT_BYTES +
-                                                       G::T_BYTES) + h * 64;
-      const float* dl = l2 + 128;
-      uint32_t sr[64];
-      tmem_ld_x64(tm + G::T_S + h * 64, sr);
-      // visible query columns of this key row: [lo_c, lo_c + span) -- key k0 + r
-      // is seen by query q0 + col iff k0 + r <= q0 + col + wr and k0 + r >= q0 + col - wl
-      const int dqk = kv_row0 + r - i * kBM;  // key minus query offset of column 0
-      const bool msk = (p.wr >= 0 && kv_row0 + kBN - 1 - p.wr > i * kBM) ||
-                       (p.wl >= 0 && kv_row0 + p.wl < i * kBM + kBM - 1);
-      const int lo_c = p.wr >= 0 ? dqk - p.wr : -kBM;
-      const int hi_c = p.wl >= 0 ? dqk + p.wl : 2 * kBM;
-      const uint32_t span = static_cast<uint32_t>(max(hi_c - lo_c + 1, 0));
-      // score bias of (query h*64 + x, key r): the tile's row h*64 + x (row 0 if
-      // broadcast over queries), 16-bit unit (r % 64) / 8 of box r / 64, rotated
-      // by the row (128-byte swizzle)
-      const bool rowb = (bias_mode & kBiasRowBcast) != 0;
-      if (BIAS) {
-        ok = wait_bar(B(G::B_BF), n & 1u, cx.abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      const uint32_t bkey = sbase + G::OFF_BIAS + (r >> 6) * (kBiasTileBytes / 2) + (r & 7) * 2;
-      const uint32_t bu = static_cast<uint32_t>(r >> 3) & 7u;
-      float b_row0 = 0.f;
-      if (BIAS && rowb) b_row0 = bias_at(bkey + ((bu ^ 0u) << 4), BF16) * kLog2e;
-      float pv[64];
-#pragma unroll
-      for (int x = 0; x < 64; x += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(l2 + x);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float bv = 0.f;
-          if (BIAS) {
-            const uint32_t row = static_cast<uint32_t>(h * 64 + x + e);
-            bv = rowb ? b_row0
-                      : bias_at(bkey + row * 128u + ((bu ^ static_cast<uint32_t>((x + e) & 7)) << 4), BF16) *
-                            kLog2e;
-          }
-          const float e2 = ex2(fmaf(__uint_as_float(sr[x + e]), c, bv - lv[e]));
-          pv[x + e] = (msk && static_cast<uint32_t>(h * 64 + x + e - lo_c) >= span) ? 0.f : e2;
+    for (int rd = 0; ok && rd * static_cast<int>(gridDim.x) < n_tiles; ++rd) {
+      const int t = snake_tile(rd);
+      if (t >= n_tiles) continue;
+      const KVTile T = kv_tile(p, t);
+      const int kv_row0 = T.kt * kBN;
+      const int key = kv_row0 + r;
+      if (T.nb == 0) {  // no query sees these keys: zero gradients
+        if (key < p.Nk) {
+          uint16_t* dst = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
+                          (static_cast<size_t>(T.bkv) * p.Nk + key) * D;
+          for (int c0 = 0; c0 < D; c0 += 8) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(0, 0, 0, 0);
         }
+        continue;
       }
-      if (BIAS) {  // this warp has read the bias tile
-        __syncwarp();
-        if (lane == 0) mbar_arrive(B(G::B_BE));
-      }
-      uint32_t pk[32];
-#pragma unroll
-      for (int x = 0; x < 32; ++x) pk[x] = pack2(pv[2 * x], pv[2 * x + 1], BF16);
-      tmem_st_x32(tm + G::T_S + h * 64, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(B(G::B_PF));
-
-      ok = wait_bar(B(G::B_DPF), n & 1u, cx.abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      uint32_t dr[64];
-      tmem_ld_x64(tm + G::T_DP + h * 64, dr);
-#pragma unroll
-      for (int x = 0; x < 64; x += 4) {
-        const float4 d4 = *reinterpret_cast<const float4*>(dl + x);
-        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) pv[x + e] *= __uint_as_float(dr[x + e]) - dv4[e];
-      }
-#pragma unroll
-      for (int x = 0; x < 32; ++x) pk[x] = pack2(pv[2 * x], pv[2 * x + 1], BF16);
-      tmem_st_x32(tm + G::T_DP + h * 64, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(B(G::B_DSF));
-    }
-    // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale)
-    const int key = kv_row0 + r;
-    uint16_t* dst = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
-                    (static_cast<size_t>(T.bkv) * p.Nk + (key < p.Nk ? key : 0)) * D;
-    const float mul = h == 0 ? 1.f : p.scale;
-    if (T.nb == 0) {  // no query sees these keys: zero gradients
-      if (key < p.Nk)
-        for (int c0 = 0; c0 < D; c0 += 8) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(0, 0, 0, 0);
-    } else if (ok) {
-      ok = wait_bar(B(G::B_ACC), 0u, cx.abort_flag);
-      if (__all_sync(0xffffffffu, ok)) {
+      const int nqb = T.nqb;
+      for (int n = 0; n < T.nb; ++n) {
+        const uint32_t g = g0 + static_cast<uint32_t>(n), m = m0 + 2u * static_cast<uint32_t>(n);
+        const int sl = static_cast<int>(m % G::NSLOT);  // the slot of Q_n, with lse2 and delta
+        const int i = T.i0 + n % nqb;
+        // lse2 / delta of this block were written by the TMA unit: observe its barrier
+        ok = wait_bar(B(G::B_SLF + sl), (m / G::NSLOT) & 1u, cx.abort_flag) &&
+             wait_bar(B(G::B_SF), g & 1u, cx.abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        // Every MMA has retired, so the slot ring is idle: each warp stages its 32
-        // rows there (16-byte units rotated by the row), then writes whole lines.
-        constexpr int U = D * 2 / 16;  // 16-byte units of a row
-        const uint32_t stg = sbase + G::OFF_SL + static_cast<uint32_t>(warp) * (32u * D * 2u);
-        const uint32_t srow = stg + static_cast<uint32_t>(lane) * (D * 2u);
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t a[32];
-          tmem_ld_x32(tm + (h == 0 ? G::T_DV : G::T_DK) + c0, a);
-          uint32_t w[16];
+        const float* l2 = reinterpret_cast<const float*>(gbase + G::OFF_SL + sl * G::SLOT_BYTES +
+                                                         G::T_BYTES) + h * 64;
+        const float* dl = l2 + 128;
+        uint32_t sr[64];
+        tmem_ld_x64(tm + G::T_S + h * 64, sr);
+        // visible query columns of this key row: [lo_c, lo_c + span) -- key k0 + r
+        // is seen by query q0 + col iff k0 + r <= q0 + col + wr and k0 + r >= q0 + col - wl
+        const int dqk = kv_row0 + r - i * kBM;  // key minus query offset of column 0
+        const bool msk = (p.wr >= 0 && kv_row0 + kBN - 1 - p.wr > i * kBM) ||
+                         (p.wl >= 0 && kv_row0 + p.wl < i * kBM + kBM - 1);
+        const int lo_c = p.wr >= 0 ? dqk - p.wr : -kBM;
+        const int hi_c = p.wl >= 0 ? dqk + p.wl : 2 * kBM;
+        const uint32_t span = static_cast<uint32_t>(max(hi_c - lo_c + 1, 0));
+        // score bias of (query h*64 + x, key r): the tile's row h*64 + x (row 0 if
+        // broadcast over queries), 16-bit unit (r % 64) / 8 of box r / 64, rotated
+        // by the row (128-byte swizzle)
+        const bool rowb = (bias_mode & kBiasRowBcast) != 0;
+        if (BIAS) {
+          ok = wait_bar(B(G::B_BF), g & 1u, cx.abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        }
+        const uint32_t bkey = sbase + G::OFF_BIAS + (r >> 6) * (kBiasTileBytes / 2) + (r & 7) * 2;
+        const uint32_t bu = static_cast<uint32_t>(r >> 3) & 7u;
+        float b_row0 = 0.f;
+        if (BIAS && rowb) b_row0 = bias_at(bkey + ((bu ^ 0u) << 4), BF16) * kLog2e;
+        float pv[64];
 #pragma unroll
-          for (int x = 0; x < 16; ++x)
-            w[x] = pack2(__uint_as_float(a[2 * x]) * mul, __uint_as_float(a[2 * x + 1]) * mul, BF16);
+        for (int x = 0; x < 64; x += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(l2 + x);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const uint32_t u = static_cast<uint32_t>(c0 / 8 + x);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             srow + ((u ^ (static_cast<uint32_t>(lane) & (U - 1))) << 4)),
-                         "r"(w[4 * x]), "r"(w[4 * x + 1]), "r"(w[4 * x + 2]), "r"(w[4 * x + 3])
-                         : "memory");
+          for (int e = 0; e < 4; ++e) {
+            float bv = 0.f;
+            if (BIAS) {
+              const uint32_t row = static_cast<uint32_t>(h * 64 + x + e);
+              bv = rowb ? b_row0
+                        : bias_at(bkey + row * 128u + ((bu ^ static_cast<uint32_t>((x + e) & 7)) << 4), BF16) *
+                              kLog2e;
+            }
+            const float e2 = ex2(fmaf(__uint_as_float(sr[x + e]), c, bv - lv[e]));
+            pv[x + e] = (msk && static_cast<uint32_t>(h * 64 + x + e - lo_c) >= span) ? 0.f : e2;
           }
         }
+        if (BIAS) {  // this warp has read the bias tile
+          __syncwarp();
+          if (lane == 0) mbar_arrive(B(G::B_BE));
+        }
+        uint32_t pk[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) pk[x] = pack2(pv[2 * x], pv[2 * x + 1], BF16);
+        tmem_st_x32(tm + G::T_S + h * 64, pk);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        const int key0 = kv_row0 + (warp & 3) * 32;
-        uint16_t* out = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
-                        static_cast<size_t>(T.bkv) * p.Nk * D;
+        if (lane == 0) mbar_arrive(B(G::B_PF));
+
+        ok = wait_bar(B(G::B_DPF), g & 1u, cx.abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t dr[64];
+        tmem_ld_x64(tm + G::T_DP + h * 64, dr);
+#pragma unroll
+        for (int x = 0; x < 64; x += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(dl + x);
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pv[x + e] *= __uint_as_float(dr[x + e]) - dv4[e];
+        }
+#pragma unroll
+        for (int x = 0; x < 32; ++x) pk[x] = pack2(pv[2 * x], pv[2 * x + 1], BF16);
+        tmem_st_x32(tm + G::T_DP + h * 64, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B(G::B_DSF));
+      }
+      if (!ok) break;
+      // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale)
+      ok = wait_bar(B(G::B_ACC), static_cast<uint32_t>(it) & 1u, cx.abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t m_next = m0 + 2u * static_cast<uint32_t>(T.nb);
+      const float mul = h == 0 ? 1.f : p.scale;
+      // staging: warpgroup h's four warps in slot (m_next + NSLOT - 2 + h) % NSLOT,
+      // 32 rows of D 16-bit values each (16-byte units rotated by the row)
+      constexpr int U = D * 2 / 16;  // 16-byte units of a row
+      const uint32_t stg = sbase + G::OFF_SL +
+                           ((m_next + G::NSLOT - 2 + static_cast<uint32_t>(h)) % G::NSLOT) * G::SLOT_BYTES +
+                           static_cast<uint32_t>(warp & 3) * (32u * D * 2u);
+      const uint32_t srow = stg + static_cast<uint32_t>(lane) * (D * 2u);
 #pragma unroll 1
-        for (int k = 0; k < U; ++k) {
-          const int rr = k * (32 / U) + lane / U, u = lane % U;
-          uint32_t w[4];
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                       : "r"(stg + static_cast<uint32_t>(rr) * (D * 2u) +
-                             ((static_cast<uint32_t>(u) ^ (static_cast<uint32_t>(rr) & (U - 1))) << 4))
-                       : "memory");
-          if (key0 + rr < p.Nk)
-            reinterpret_cast<uint4*>(out + static_cast<size_t>(key0 + rr) * D)[u] =
-                make_uint4(w[0], w[1], w[2], w[3]);
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t a[32];
+        tmem_ld_x32(tm + (h == 0 ? G::T_DV : G::T_DK) + c0, a);
+        uint32_t w[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          w[x] = pack2(__uint_as_float(a[2 * x]) * mul, __uint_as_float(a[2 * x + 1]) * mul, BF16);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const uint32_t u = static_cast<uint32_t>(c0 / 8 + x);
+          st_shared_v4(srow + ((u ^ (static_cast<uint32_t>(lane) & (U - 1))) << 4), w + 4 * x);
         }
       }
+      // the accumulators are in registers and shared memory: the next tile's
+      // first dV and dK may overwrite them
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_ACCE));
+      const int key0 = kv_row0 + (warp & 3) * 32;
+      uint16_t* out = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
+                      static_cast<size_t>(T.bkv) * p.Nk * D;
+#pragma unroll 1
+      for (int k = 0; k < U; ++k) {
+        const int rr = k * (32 / U) + lane / U, u = lane % U;
+        uint32_t w[4];
+        ld_shared_v4(stg + static_cast<uint32_t>(rr) * (D * 2u) +
+                         ((static_cast<uint32_t>(u) ^ (static_cast<uint32_t>(rr) & (U - 1))) << 4),
+                     w);
+        if (key0 + rr < p.Nk)
+          reinterpret_cast<uint4*>(out + static_cast<size_t>(key0 + rr) * D)[u] =
+              make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      // the TMA unit loads into the staging slots next: order these shared
+      // accesses before its writes
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_STG));
+      m0 = m_next;
+      g0 += static_cast<uint32_t>(T.nb);
+      ++it;
     }
   }
   __syncwarp();
@@ -589,9 +684,12 @@ struct GeoQ {
   static constexpr int OFF_Q = 0, OFF_DO = T_BYTES, OFF_SL = 2 * T_BYTES;
   static constexpr int OFF_BIAS = OFF_SL + NSLOT * T_BYTES;  // the block pair's bias tile
   static constexpr int OFF_BAR = OFF_BIAS + (BIAS ? kBiasTileBytes : 0);
+  // (persistent: B_QE = the tile's Q and dO no longer read, B_ACCE = its dQ
+  // read out of tensor memory, B_STG = its epilogue done with the staging slot)
   static constexpr int B_QF = 0, B_SLF = 1, B_SLE = 1 + NSLOT, B_SDP = 1 + 2 * NSLOT,
                        B_SFREE = B_SDP + 1, B_DSF = B_SDP + 2, B_DSE = B_SDP + 3, B_DQF = B_SDP + 4,
-                       B_BF = B_SDP + 5, B_BE = B_SDP + 6, NBAR = B_SDP + 7;
+                       B_BF = B_SDP + 5, B_BE = B_SDP + 6, B_QE = B_SDP + 7, B_ACCE = B_SDP + 8,
+                       B_STG = B_SDP + 9, NBAR = B_SDP + 10;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // TMEM columns: S 0..127, dP 128..255, dS (packed) 256..319, dQ 320..320+D-1
@@ -600,6 +698,41 @@ struct GeoQ {
   static_assert(320 + D <= 512, "tensor memory budget");
 };
 
+// One query tile of the dQ kernel: (b, query head) row bh, first row q0, its
+// key/value head kvz, and the key blocks its rows see, [jb0, jb0 + nb).
+struct QTile {
+  int bh, q0, kvz, jb0, nb;
+};
+
+// tile t: causal launches take the last query blocks (most keys) first
+__device__ __forceinline__ QTile q_tile(const BwdParams& p, int t) {
+  QTile T;
+  const int BH = p.B * p.Hq;
+  int qt;
+  if (p.causal) {
+    qt = p.nqt - 1 - t / BH;
+    T.bh = t % BH;
+  } else {
+    T.bh = t / p.nqt;
+    qt = t % p.nqt;
+  }
+  T.q0 = qt * kBM;
+  T.kvz = (T.bh / p.Hq) * p.Hkv + (T.bh % p.Hq) / p.group;
+  const int nkb = (p.Nk + kBN - 1) / kBN;
+  // key blocks this tile's rows see: keys q - wl .. q + wr (causal: wr = 0)
+  const int qlast = min(T.q0 + kBM, p.Nq) - 1;
+  T.jb0 = p.wl >= 0 ? min(max(0, T.q0 - p.wl) / kBN, nkb) : 0;
+  const int jb1 = p.wr >= 0 ? min(nkb - 1, (qlast + p.wr) / kBN) : nkb - 1;
+  T.nb = jb1 >= T.jb0 ? jb1 - T.jb0 + 1 : 0;
+  return T;
+}
+
+// Persistent like the dK/dV kernel (snake order over the tiles; ring items,
+// blocks and tiles counted across tiles): the next tile's Q, dO and first K/V
+// blocks load, and its first S and dP run, while the compute warps write the
+// previous tile's dQ.  The epilogue stages in the K slot of the next tile's
+// NKS-th K block (item M + 2 (NKS - 1), M = the first item after the tile),
+// which held the tile's own last K; the TMA thread loads it only after B_STG.
 template <int D, bool BF16, bool BIAS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -616,25 +749,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   cx.sbase = sbase;
   cx.abort_flag = misc + 1;
   auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
-
-  // tile: (b, hq, query block); causal: the last query blocks (most keys) first
-  const int BH = p.B * p.Hq, t = blockIdx.x;
-  int bh, qt;
-  if (p.causal) {
-    qt = p.nqt - 1 - t / BH;
-    bh = t % BH;
-  } else {
-    bh = t / p.nqt;
-    qt = t % p.nqt;
-  }
-  const int q0 = qt * kBM;
-  const int kvz = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
-  const int nkb = (p.Nk + kBN - 1) / kBN;
-  // key blocks this tile's rows see: keys q - wl .. q + wr (causal: wr = 0)
-  const int qlast = min(q0 + kBM, p.Nq) - 1;
-  const int jb0 = p.wl >= 0 ? min(max(0, q0 - p.wl) / kBN, nkb) : 0;
-  const int jb1 = p.wr >= 0 ? min(nkb - 1, (qlast + p.wr) / kBN) : nkb - 1;
-  const int nb = jb1 >= jb0 ? jb1 - jb0 + 1 : 0;
+  const int n_tiles = p.B * p.Hq * p.nqt;
+  constexpr int kGateOff = 2 * (G::NKS - 1);  // staging item, from the first item after a tile
 
   if (threadIdx.x == 0) {
     mbar_init(B(G::B_QF), 1);
@@ -649,6 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(B(G::B_DQF), 1);
     mbar_init(B(G::B_BF), 1);
     mbar_init(B(G::B_BE), 8);
+    mbar_init(B(G::B_QE), 1);
+    mbar_init(B(G::B_ACCE), 8);
+    mbar_init(B(G::B_STG), 8);
     misc[1] = 0u;
     fence_mbar_init();
   }
@@ -662,49 +781,81 @@ __global__ void __launch_bounds__(kThreads, 1)
   cx.tmem = misc[0];
 
   if (warp >= 8) setmaxnreg_dec<88>();
-  if (warp == 9 && lane == 0 && nb > 0) {
-    // ---- TMA: Q and dO once, then (K_j, V_j) per key block
+  if (warp == 9 && lane == 0) {
+    // ---- TMA: per tile Q and dO, then (K_j, V_j) per key block
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
-    mbar_arrive_expect_tx(B(G::B_QF), 2 * G::T_BYTES);
+    int m0 = 0;              // ring items issued before this tile
+    int gate = -1;           // item that must wait for an epilogue's staging (-1: none)
+    uint32_t gate_par = 0;   // ... and that epilogue's B_STG phase
+    int it = 0;              // tiles with blocks before this one
+    bool ok = true;
+    for (int rd = 0; ok && rd * static_cast<int>(gridDim.x) < n_tiles; ++rd) {
+      const int t = snake_tile(rd);
+      if (t >= n_tiles) continue;
+      const QTile T = q_tile(p, t);
+      if (T.nb == 0) continue;
+      if (it > 0 && !wait_bar(B(G::B_QE), (it - 1) & 1u, cx.abort_flag)) break;
+      mbar_arrive_expect_tx(B(G::B_QF), 2 * G::T_BYTES);
 #pragma unroll
-    for (int c = 0; c < G::DCH; ++c) {
-      tma_load_3d(sbase + G::OFF_Q + c * G::CHUNK, &tm_q, B(G::B_QF), c * 64, q0, bh, pol_first);
-      tma_load_3d(sbase + G::OFF_DO + c * G::CHUNK, &tm_do, B(G::B_QF), c * 64, q0, bh, pol_first);
-    }
-    for (int m = 0; m < 2 * nb; ++m) {  // item m: K (even) or V (odd) of block m / 2
-      const int sl = G::slot(m), u = G::use(m);
-      if (u > 0 && !wait_bar(B(G::B_SLE + sl), (u - 1) & 1u, cx.abort_flag)) break;
-      mbar_arrive_expect_tx(B(G::B_SLF + sl), G::T_BYTES);
+      for (int c = 0; c < G::DCH; ++c) {
+        tma_load_3d(sbase + G::OFF_Q + c * G::CHUNK, &tm_q, B(G::B_QF), c * 64, T.q0, T.bh, pol_first);
+        tma_load_3d(sbase + G::OFF_DO + c * G::CHUNK, &tm_do, B(G::B_QF), c * 64, T.q0, T.bh, pol_first);
+      }
+      for (int mm = 0; mm < 2 * T.nb; ++mm) {  // item mm: K (even) or V (odd) of block mm / 2
+        const int m = m0 + mm;
+        if (m == gate && !wait_bar(B(G::B_STG), gate_par, cx.abort_flag)) { ok = false; break; }
+        const int sl = G::slot(m), u = G::use(m);
+        if (u > 0 && !wait_bar(B(G::B_SLE + sl), (u - 1) & 1u, cx.abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(B(G::B_SLF + sl), G::T_BYTES);
 #pragma unroll
-      for (int c = 0; c < G::DCH; ++c)
-        tma_load_3d(sbase + G::OFF_SL + sl * G::T_BYTES + c * G::CHUNK, (m & 1) ? &tm_v : &tm_k,
-                    B(G::B_SLF + sl), c * 64, (jb0 + (m >> 1)) * kBN, kvz, pol_last);
+        for (int c = 0; c < G::DCH; ++c)
+          tma_load_3d(sbase + G::OFF_SL + sl * G::T_BYTES + c * G::CHUNK, (mm & 1) ? &tm_v : &tm_k,
+                      B(G::B_SLF + sl), c * 64, (T.jb0 + (mm >> 1)) * kBN, T.kvz, pol_last);
+      }
+      if (!ok) break;
+      m0 += 2 * T.nb;
+      // a previous epilogue's gate not reached by this tile's items (short
+      // tiles): wait for it here, before this tile's gate replaces it
+      if (gate >= m0 && !wait_bar(B(G::B_STG), gate_par, cx.abort_flag)) break;
+      gate = m0 + kGateOff;
+      gate_par = static_cast<uint32_t>(it) & 1u;
+      ++it;
     }
-  } else if (BIAS && warp == 10 && lane == 0 && nb > 0) {
+  } else if (BIAS && warp == 10 && lane == 0) {
     // ---- TMA: the bias tile of each key block: rows = this tile's queries (one
     // row if broadcast over queries), columns = the block's keys
     const uint64_t pol = policy_evict_last();
     const int rows = (bias_mode & kBiasRowBcast) ? 1 : kBM;
-    for (int j = 0; j < nb; ++j) {
-      if (j > 0 && !wait_bar(B(G::B_BE), (j - 1) & 1u, cx.abort_flag)) break;
-      mbar_arrive_expect_tx(B(G::B_BF), 2 * rows * 128);
+    int g0 = 0;  // blocks before this tile
+    bool ok = true;
+    for (int rd = 0; ok && rd * static_cast<int>(gridDim.x) < n_tiles; ++rd) {
+      const int t = snake_tile(rd);
+      if (t >= n_tiles) continue;
+      const QTile T = q_tile(p, t);
+      if (T.nb == 0) continue;
+      for (int j = 0; j < T.nb; ++j) {
+        const int g = g0 + j;
+        if (g > 0 && !wait_bar(B(G::B_BE), (g - 1) & 1u, cx.abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(B(G::B_BF), 2 * rows * 128);
 #pragma unroll
-      for (int box = 0; box < 2; ++box)
-        tma_load_4d(sbase + G::OFF_BIAS + box * (kBiasTileBytes / 2), &tm_b, B(G::B_BF),
-                    (jb0 + j) * kBN + box * 64, (bias_mode & kBiasRowBcast) ? 0 : q0,
-                    (bias_mode & kBiasPerHead) ? bh % p.Hq : 0,
-                    (bias_mode & kBiasPerBatch) ? bh / p.Hq : 0, pol);
+        for (int box = 0; box < 2; ++box)
+          tma_load_4d(sbase + G::OFF_BIAS + box * (kBiasTileBytes / 2), &tm_b, B(G::B_BF),
+                      (T.jb0 + j) * kBN + box * 64, (bias_mode & kBiasRowBcast) ? 0 : T.q0,
+                      (bias_mode & kBiasPerHead) ? T.bh % p.Hq : 0,
+                      (bias_mode & kBiasPerBatch) ? T.bh / p.Hq : 0, pol);
+      }
+      g0 += T.nb;
     }
-  } else if (warp == 8 && lane == 0 && nb > 0) {
-    // ---- MMA: S(0) dP(0) | S(j+1) dP(j+1) dQ(j) | ...
+  } else if (warp == 8 && lane == 0) {
+    // ---- MMA, per tile: S(0) dP(0) | S(j+1) dP(j+1) dQ(j) | ...
     constexpr uint32_t kIdNT = idesc_f16(128, 128, BF16, false);
     constexpr uint32_t kIdTN = idesc_f16(128, D, BF16, true);
     const uint32_t tm = cx.tmem;
     const uint64_t dq0 = sdesc_sw128(sbase + G::OFF_Q, 16, 1024);
     const uint64_t ddo0 = sdesc_sw128(sbase + G::OFF_DO, 16, 1024);
-    // ring item m (K_{m/2} or V_{m/2}): its slot, and the parity of its fill
+    // ring item m (a K or V block): its slot, and the parity of its fill
     auto kv_desc = [&](int m, bool mn) {
       const uint32_t a = sbase + G::OFF_SL + G::slot(m) * G::T_BYTES;
       return mn ? sdesc_sw128(a, G::CHUNK, 1024) : sdesc_sw128(a, 16, 1024);
@@ -712,33 +863,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto wait_item = [&](int m) {
       return wait_bar(B(G::B_SLF + G::slot(m)), G::use(m) & 1u, cx.abort_flag);
     };
-    // S(j) and dP(j); V_j's slot is free once dP(j) completes
-    auto issue_sdp = [&](int j) {
-      mma_nt<D>(tm + G::T_S, dq0, kv_desc(2 * j, false), kIdNT, G::CHUNK, G::CHUNK);
-      mma_nt<D>(tm + G::T_DP, ddo0, kv_desc(2 * j + 1, false), kIdNT, G::CHUNK, G::CHUNK);
+    // S and dP of the block whose K is item m; its V's slot is free once dP completes
+    auto issue_sdp = [&](int m) {
+      mma_nt<D>(tm + G::T_S, dq0, kv_desc(m, false), kIdNT, G::CHUNK, G::CHUNK);
+      mma_nt<D>(tm + G::T_DP, ddo0, kv_desc(m + 1, false), kIdNT, G::CHUNK, G::CHUNK);
       mma_commit(B(G::B_SDP));
-      mma_commit(B(G::B_SLE + G::slot(2 * j + 1)));
+      mma_commit(B(G::B_SLE + G::slot(m + 1)));
     };
     // dS of key column k: warpgroup k / 64 packed its half at columns (k / 64) * 32 ..
     auto acol = [](int kk) { return static_cast<uint32_t>(kk * 8); };
-    bool ok = wait_bar(B(G::B_QF), 0u, cx.abort_flag) && wait_item(0) && wait_item(1);
-    if (ok) {
+    int m0 = 0, g0 = 0, it = 0;
+    bool ok = true;
+    for (int rd = 0; ok && rd * static_cast<int>(gridDim.x) < n_tiles; ++rd) {
+      const int t = snake_tile(rd);
+      if (t >= n_tiles) continue;
+      const QTile T = q_tile(p, t);
+      if (T.nb == 0) continue;
+      // S(0) and dP(0) overwrite S and dP: the compute warps must have read the
+      // previous tile's last block
+      ok = (g0 == 0 || wait_bar(B(G::B_SFREE), (g0 - 1) & 1u, cx.abort_flag)) &&
+           wait_bar(B(G::B_QF), static_cast<uint32_t>(it) & 1u, cx.abort_flag) && wait_item(m0) &&
+           wait_item(m0 + 1);
+      if (!ok) break;
       tc_fence_after();
-      issue_sdp(0);
-    }
-    for (int j = 0; ok && j < nb; ++j) {
-      if (j + 1 < nb) {  // next S and dP once the compute warps have read this block's
-        if (!wait_bar(B(G::B_SFREE), j & 1u, cx.abort_flag)) break;
-        if (!wait_item(2 * j + 2) || !wait_item(2 * j + 3)) break;
+      issue_sdp(m0);
+      if (T.nb == 1) mma_commit(B(G::B_QE));
+      for (int j = 0; j < T.nb; ++j) {
+        const int g = g0 + j, m = m0 + 2 * j;
+        if (j + 1 < T.nb) {  // next S and dP once the compute warps have read this block's
+          if (!wait_bar(B(G::B_SFREE), g & 1u, cx.abort_flag)) { ok = false; break; }
+          if (!wait_item(m + 2) || !wait_item(m + 3)) { ok = false; break; }
+          tc_fence_after();
+          issue_sdp(m + 2);
+          if (j + 2 == T.nb) mma_commit(B(G::B_QE));  // the tile's last read of Q and dO
+        }
+        if (!wait_bar(B(G::B_DSF), g & 1u, cx.abort_flag)) { ok = false; break; }
+        // the first dQ of a tile overwrites the accumulator: the previous tile's
+        // epilogue must have read it out
+        if (j == 0 && it > 0 && !wait_bar(B(G::B_ACCE), (it - 1) & 1u, cx.abort_flag)) { ok = false; break; }
         tc_fence_after();
-        issue_sdp(j + 1);
+        mma_tn<D>(tm + G::T_DQ, tm + G::T_DS, kv_desc(m, true), kIdTN, j > 0, acol);
+        mma_commit(B(G::B_DSE));
+        mma_commit(B(G::B_SLE + G::slot(m)));  // K_j's slot
+        if (j + 1 == T.nb) mma_commit(B(G::B_DQF));
       }
-      if (!wait_bar(B(G::B_DSF), j & 1u, cx.abort_flag)) break;
-      tc_fence_after();
-      mma_tn<D>(tm + G::T_DQ, tm + G::T_DS, kv_desc(2 * j, true), kIdTN, j > 0, acol);
-      mma_commit(B(G::B_DSE));
-      mma_commit(B(G::B_SLE + G::slot(2 * j)));  // K_j's slot
-      if (j + 1 == nb) mma_commit(B(G::B_DQF));
+      m0 += 2 * T.nb;
+      g0 += T.nb;
+      ++it;
     }
   } else if (warp < 8) {
     // ---- compute: thread = query row r, warpgroup h = key columns h*64 .. +63
@@ -746,118 +917,133 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2, r = (warp & 3) * 32 + lane;
     const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.c;
-    const size_t srow = static_cast<size_t>(bh) * p.Nq_pad + q0 + r;
-    const float lse2 = p.lse2[srow], dlt = p.delta[srow];
-    const int qpos = q0 + r;
+    int m0 = 0, g0 = 0, it = 0;
     bool ok = true;
-    for (int j = 0; ok && j < nb; ++j) {
-      ok = wait_bar(B(G::B_SDP), j & 1u, cx.abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      uint32_t sr[64], dr[64];
-      tmem_ld_x64(tm + G::T_S + h * 64, sr);
-      tmem_ld_x64(tm + G::T_DP + h * 64, dr);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(B(G::B_SFREE));
-      // visible keys of this row in the block: [0, lim)
-      const int kbase = (jb0 + j) * kBN + h * 64;
-      int lim = p.Nk - kbase;  // keys [lo, lim) of this half block are visible to the row
-      if (p.wr >= 0) lim = min(lim, qpos + p.wr - kbase + 1);
-      const int lo = p.wl >= 0 ? qpos - p.wl - kbase : 0;
-      const uint32_t span = static_cast<uint32_t>(max(lim - lo, 0));
-      // score bias of this row, keys h*64 .. +63: box h of the tile, row r (row 0
-      // if broadcast over queries), 16-byte units rotated by the row
-      uint32_t bw[32];
-      if (BIAS) {
-        ok = wait_bar(B(G::B_BF), j & 1u, cx.abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        const uint32_t brow = (bias_mode & kBiasRowBcast) ? 0u : static_cast<uint32_t>(r);
-        const uint32_t bb = sbase + G::OFF_BIAS + h * (kBiasTileBytes / 2) + brow * 128u;
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(bw[4 * u]), "=r"(bw[4 * u + 1]), "=r"(bw[4 * u + 2]), "=r"(bw[4 * u + 3])
-                       : "r"(bb + ((static_cast<uint32_t>(u) ^ (brow & 7u)) << 4)));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(B(G::B_BE));
-      }
-      uint32_t pk[32];
-#pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        float2 b2 = make_float2(0.f, 0.f);
-        if (BIAS) b2 = unpack2(bw[x], BF16);
-        float v2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int i = 2 * x + e;
-          const float bv = BIAS ? (e ? b2.y : b2.x) * kLog2e : 0.f;
-          const float pe = ex2(fmaf(__uint_as_float(sr[i]), c, bv - lse2));
-          v2[e] = static_cast<uint32_t>(i - lo) < span ? pe * (__uint_as_float(dr[i]) - dlt) : 0.f;
+    for (int rd = 0; ok && rd * static_cast<int>(gridDim.x) < n_tiles; ++rd) {
+      const int t = snake_tile(rd);
+      if (t >= n_tiles) continue;
+      const QTile T = q_tile(p, t);
+      const int qpos = T.q0 + r;
+      if (T.nb == 0) {  // no key seen by this tile's rows (key windows): dQ = 0
+        if (qpos < p.Nq) {
+          uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) + (static_cast<size_t>(T.bh) * p.Nq + qpos) * D;
+          for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 8)
+            *reinterpret_cast<uint4*>(dst + c0) = make_uint4(0, 0, 0, 0);
         }
-        pk[x] = pack2(v2[0], v2[1], BF16);
+        continue;
       }
-      if (j > 0) {  // dQ(j-1) has read the previous dS
-        ok = wait_bar(B(G::B_DSE), (j - 1) & 1u, cx.abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) break;
+      const size_t srow = static_cast<size_t>(T.bh) * p.Nq_pad + qpos;
+      const float lse2 = p.lse2[srow], dlt = p.delta[srow];
+      for (int j = 0; j < T.nb; ++j) {
+        const int g = g0 + j;
+        ok = wait_bar(B(G::B_SDP), g & 1u, cx.abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-      }
-      tmem_st_x32(tm + G::T_DS + h * 32, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(B(G::B_DSF));
-    }
-    // ---- epilogue: dQ = scale * acc, warpgroup h writes columns h * D/2 .. +D/2
-    if (nb == 0 && qpos < p.Nq) {  // no key seen by this tile's rows (key windows): dQ = 0
-      uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) + (static_cast<size_t>(bh) * p.Nq + qpos) * D;
-      for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 8)
-        *reinterpret_cast<uint4*>(dst + c0) = make_uint4(0, 0, 0, 0);
-    }
-    if (ok && nb > 0) {
-      ok = wait_bar(B(G::B_DQF), 0u, cx.abort_flag);
-      if (__all_sync(0xffffffffu, ok)) {
-        tc_fence_after();
-        // The K / V slots are idle once dQ is final: each warp stages its 32 rows'
-        // half rows there (16-byte units rotated by the row), then writes lines.
-        constexpr int U = D / 16;  // 16-byte units of a half row
-        const uint32_t stg = sbase + G::OFF_SL + static_cast<uint32_t>(warp) * (32u * D);
-        const uint32_t srow = stg + static_cast<uint32_t>(lane) * D;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D / 2; c0 += 32) {
-          uint32_t a[32];
-          tmem_ld_x32(tm + G::T_DQ + h * (D / 2) + c0, a);
-          uint32_t w[16];
+        uint32_t sr[64], dr[64];
+        tmem_ld_x64(tm + G::T_S + h * 64, sr);
+        tmem_ld_x64(tm + G::T_DP + h * 64, dr);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B(G::B_SFREE));
+        // visible keys of this row in the block: [0, lim)
+        const int kbase = (T.jb0 + j) * kBN + h * 64;
+        int lim = p.Nk - kbase;  // keys [lo, lim) of this half block are visible to the row
+        if (p.wr >= 0) lim = min(lim, qpos + p.wr - kbase + 1);
+        const int lo = p.wl >= 0 ? qpos - p.wl - kbase : 0;
+        const uint32_t span = static_cast<uint32_t>(max(lim - lo, 0));
+        // score bias of this row, keys h*64 .. +63: box h of the tile, row r (row 0
+        // if broadcast over queries), 16-byte units rotated by the row
+        uint32_t bw[32];
+        if (BIAS) {
+          ok = wait_bar(B(G::B_BF), g & 1u, cx.abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          const uint32_t brow = (bias_mode & kBiasRowBcast) ? 0u : static_cast<uint32_t>(r);
+          const uint32_t bb = sbase + G::OFF_BIAS + h * (kBiasTileBytes / 2) + brow * 128u;
 #pragma unroll
-          for (int x = 0; x < 16; ++x)
-            w[x] = pack2(__uint_as_float(a[2 * x]) * p.scale, __uint_as_float(a[2 * x + 1]) * p.scale,
-                         BF16);
+          for (int u = 0; u < 8; ++u)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(bw[4 * u]), "=r"(bw[4 * u + 1]), "=r"(bw[4 * u + 2]), "=r"(bw[4 * u + 3])
+                         : "r"(bb + ((static_cast<uint32_t>(u) ^ (brow & 7u)) << 4)));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(B(G::B_BE));
+        }
+        uint32_t pk[32];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const uint32_t u = static_cast<uint32_t>(c0 / 8 + x);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             srow + ((u ^ (static_cast<uint32_t>(lane) & (U - 1))) << 4)),
-                         "r"(w[4 * x]), "r"(w[4 * x + 1]), "r"(w[4 * x + 2]), "r"(w[4 * x + 3])
-                         : "memory");
+        for (int x = 0; x < 32; ++x) {
+          float2 b2 = make_float2(0.f, 0.f);
+          if (BIAS) b2 = unpack2(bw[x], BF16);
+          float v2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int i = 2 * x + e;
+            const float bv = BIAS ? (e ? b2.y : b2.x) * kLog2e : 0.f;
+            const float pe = ex2(fmaf(__uint_as_float(sr[i]), c, bv - lse2));
+            v2[e] = static_cast<uint32_t>(i - lo) < span ? pe * (__uint_as_float(dr[i]) - dlt) : 0.f;
           }
+          pk[x] = pack2(v2[0], v2[1], BF16);
         }
+        if (g > 0) {  // the previous dQ MMA has read the previous dS
+          ok = wait_bar(B(G::B_DSE), (g - 1) & 1u, cx.abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
+        }
+        tmem_st_x32(tm + G::T_DS + h * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        const int q0w = q0 + (warp & 3) * 32;
-        uint16_t* out = reinterpret_cast<uint16_t*>(p.dq) + static_cast<size_t>(bh) * p.Nq * D + h * (D / 2);
+        if (lane == 0) mbar_arrive(B(G::B_DSF));
+      }
+      if (!ok) break;
+      // ---- epilogue: dQ = scale * acc, warpgroup h writes columns h * D/2 .. +D/2
+      ok = wait_bar(B(G::B_DQF), static_cast<uint32_t>(it) & 1u, cx.abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const int m_next = m0 + 2 * T.nb;
+      // staging: the slot of item m_next + kGateOff; each warp 32 half rows
+      // (16-byte units rotated by the row)
+      constexpr int U = D / 16;  // 16-byte units of a half row
+      const uint32_t stg = sbase + G::OFF_SL + G::slot(m_next + kGateOff) * G::T_BYTES +
+                           static_cast<uint32_t>(warp) * (32u * D);
+      const uint32_t srow_s = stg + static_cast<uint32_t>(lane) * D;
 #pragma unroll 1
-        for (int k = 0; k < U; ++k) {
-          const int rr = k * (32 / U) + lane / U, u = lane % U;
-          uint32_t w[4];
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                       : "r"(stg + static_cast<uint32_t>(rr) * D +
-                             ((static_cast<uint32_t>(u) ^ (static_cast<uint32_t>(rr) & (U - 1))) << 4))
-                       : "memory");
-          if (q0w + rr < p.Nq)
-            reinterpret_cast<uint4*>(out + static_cast<size_t>(q0w + rr) * D)[u] =
-                make_uint4(w[0], w[1], w[2], w[3]);
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+        uint32_t a[32];
+        tmem_ld_x32(tm + G::T_DQ + h * (D / 2) + c0, a);
+        uint32_t w[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          w[x] = pack2(__uint_as_float(a[2 * x]) * p.scale, __uint_as_float(a[2 * x + 1]) * p.scale, BF16);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const uint32_t u = static_cast<uint32_t>(c0 / 8 + x);
+          st_shared_v4(srow_s + ((u ^ (static_cast<uint32_t>(lane) & (U - 1))) << 4), w + 4 * x);
         }
       }
+      // dQ is in registers and shared memory: the next tile's first dQ may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_ACCE));
+      const int q0w = T.q0 + (warp & 3) * 32;
+      uint16_t* out = reinterpret_cast<uint16_t*>(p.dq) + static_cast<size_t>(T.bh) * p.Nq * D + h * (D / 2);
+#pragma unroll 1
+      for (int k = 0; k < U; ++k) {
+        const int rr = k * (32 / U) + lane / U, u = lane % U;
+        uint32_t w[4];
+        ld_shared_v4(stg + static_cast<uint32_t>(rr) * D +
+                         ((static_cast<uint32_t>(u) ^ (static_cast<uint32_t>(rr) & (U - 1))) << 4),
+                     w);
+        if (q0w + rr < p.Nq)
+          reinterpret_cast<uint4*>(out + static_cast<size_t>(q0w + rr) * D)[u] =
+              make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      // the TMA unit loads into the staging slot next: order these shared
+      // accesses before its writes
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(G::B_STG));
+      m0 = m_next;
+      g0 += T.nb;
+      ++it;
     }
   }
   __syncwarp();
@@ -948,7 +1134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   cx.sbase = sbase;
   cx.abort_flag = misc + 1;
   auto B = [&](int i) { return cx.bar(i, G::OFF_BAR); };
-  const KVTile T = kv_tile(p, kBS);
+  const KVTile T = kv_tile(p, blockIdx.x, kBS);
 
   if (threadIdx.x == 0) {
     mbar_init(B(G::B_KV), 1);
@@ -1600,12 +1786,16 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const int rc = setup_bwd<D, BF16>(p, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal,
                                     wl, wr, st, ws, sms);
   if (rc != FA_OK) return rc;
-  // 2. dK, dV: one CTA per (b, kv head, key block)
-  fab::bwd_dkdv_kernel<D, BF16, BIAS><<<(unsigned)(B * Hkv * p.nkt), fab::kThreads, GK::SMEM_BYTES, st>>>(
+  // 2. dK, dV: persistent, one CTA per SM over the (b, kv head, key block) tiles
+  const long long kv_tiles = (long long)B * Hkv * p.nkt;
+  const unsigned kv_grid = (unsigned)(kv_tiles < sms ? kv_tiles : sms);
+  fab::bwd_dkdv_kernel<D, BF16, BIAS><<<kv_grid, fab::kThreads, GK::SMEM_BYTES, st>>>(
       tq, tdo, tk, tv, p, tb, bias_mode);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
-  // 3. dQ: one CTA per (b, query head, query block)
-  fab::bwd_dq_kernel<D, BF16, BIAS><<<(unsigned)(B * Hq * p.nqt), fab::kThreads, GQ::SMEM_BYTES, st>>>(
+  // 3. dQ: persistent, one CTA per SM over the (b, query head, query block) tiles
+  const long long q_tiles = (long long)B * Hq * p.nqt;
+  const unsigned q_grid = (unsigned)(q_tiles < sms ? q_tiles : sms);
+  fab::bwd_dq_kernel<D, BF16, BIAS><<<q_grid, fab::kThreads, GQ::SMEM_BYTES, st>>>(
       tq, tdo, tk, tv, p, tb, bias_mode);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
