@@ -237,9 +237,9 @@ def test_scale_values_two_tile_kernel(cuda_dev, scale):
 # fp16 without a mask over at most 4096 keys runs the staged epilogue (output
 # rows through shared memory, written as whole lines); one key more runs the
 # plain one.  600 query rows: the last 256-row tile holds 88 live rows.
-@pytest.mark.parametrize("nk", [1500, 4096, 4097])
-def test_staged_epilogue(cuda_dev, nk):
-    w = Workload(f"staged nk{nk}", 2, 40, 40, 600, nk, 128, "fp16", False, seed=7)
+@pytest.mark.parametrize("nk,hkv", [(1500, 40), (4096, 40), (4097, 40), (2000, 10)])
+def test_staged_epilogue(cuda_dev, nk, hkv):
+    w = Workload(f"staged nk{nk} hkv{hkv}", 2, 40, hkv, 600, nk, 128, "fp16", False, seed=7)
     assert 2 * fa.num_tiles(w.B, w.Hq, w.Nq, w.D) >= 148
     rows = np.unique(np.concatenate([sample_rows(w.Nq, 24, w.seed), np.arange(505, 600, 6), [511, 512]]))
     compare(w, cuda_dev, rows=rows)
