@@ -42,6 +42,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "fa.h"
 #include "sm100_ptx.cuh"
@@ -135,7 +136,9 @@ struct BwdParams {
 // ------------------------------------------------------------------ Delta, LSE2
 // D / 8 threads per row, 8 elements (16 bytes) each; rows in the padding get
 // (+inf, 0).  Rows are taken warp by warp so that every lane of a warp reaches
-// the shuffles.
+// the shuffles, kPrepGroups row groups per pass with all their loads issued
+// before any is used (more bytes in flight per thread).
+constexpr int kPrepGroups = 4;
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o,
                                                        const uint16_t* __restrict__ dout,
@@ -144,36 +147,52 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
                                                        float* __restrict__ delta, int BH, int Nq,
                                                        int Nq_pad) {
   constexpr int TPR = D / 8;      // threads per row
-  constexpr int RPW = 32 / TPR;   // rows per warp
+  constexpr int RPW = 32 / TPR;   // rows per warp and group
+  constexpr int U = kPrepGroups;
+  grid_dep_launch();  // the dK/dV kernel may start its setup and K/V loads
   const long long total = static_cast<long long>(BH) * Nq_pad;
   const int lane = threadIdx.x & 31, sub = lane % TPR;
   const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long base = warp * RPW; base < total; base += n_warps * RPW) {
-    const long long row = base + lane / TPR;
-    const long long bh = row / Nq_pad;
-    const int i = static_cast<int>(row - bh * Nq_pad);
-    const bool live = row < total && i < Nq;
-    float acc = 0.f;
-    if (live) {
-      const size_t off = (static_cast<size_t>(bh) * Nq + i) * D + sub * 8;
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + off));
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + off));
-      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+  for (long long base = warp * RPW * U; base < total; base += n_warps * RPW * U) {
+    uint4 a[U], b[U];
+    float L[U];
+    bool live[U];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const float2 fa2 = unpack2(aw[x], BF16), fb2 = unpack2(bw[x], BF16);
-        acc = fmaf(fa2.x, fb2.x, acc);
-        acc = fmaf(fa2.y, fb2.y, acc);
+    for (int u = 0; u < U; ++u) {
+      const long long row = base + u * RPW + lane / TPR;
+      const long long bh = row / Nq_pad;
+      const int i = static_cast<int>(row - bh * Nq_pad);
+      live[u] = row < total && i < Nq;
+      a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
+      L[u] = -INFINITY;
+      if (live[u]) {
+        const size_t off = (static_cast<size_t>(bh) * Nq + i) * D + sub * 8;
+        a[u] = __ldg(reinterpret_cast<const uint4*>(o + off));
+        b[u] = __ldg(reinterpret_cast<const uint4*>(dout + off));
+        L[u] = __ldg(lse + bh * Nq + i);
       }
     }
 #pragma unroll
-    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (sub == 0 && row < total) {
-      delta[row] = live ? acc : 0.f;
-      // a row that saw no key (LSE = -inf, key windows) gets +inf: P = 0 there
-      const float L = live ? lse[bh * Nq + i] : -INFINITY;
-      lse2[row] = L == -INFINITY ? INFINITY : L * kLog2e;
+    for (int u = 0; u < U; ++u) {
+      const long long row = base + u * RPW + lane / TPR;
+      float acc = 0.f;
+      if (live[u]) {
+        const uint32_t aw[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, bw[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const float2 fa2 = unpack2(aw[x], BF16), fb2 = unpack2(bw[x], BF16);
+          acc = fmaf(fa2.x, fb2.x, acc);
+          acc = fmaf(fa2.y, fb2.y, acc);
+        }
+      }
+#pragma unroll
+      for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (sub == 0 && row < total) {
+        delta[row] = live[u] ? acc : 0.f;
+        // a row that saw no key (LSE = -inf, key windows) gets +inf: P = 0 there
+        lse2[row] = L[u] == -INFINITY ? INFINITY : L[u] * kLog2e;
+      }
     }
   }
 }
@@ -334,11 +353,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   cx.tmem = misc[0];
 
+  // every CTA is resident: the dQ kernel may launch (it waits for this one
+  // before it reads anything this call writes)
+  if (threadIdx.x == 0) grid_dep_launch();
   // Registers: 208 for the two compute warpgroups, 88 for the rest (2 x 128 x
   // 208 + 128 x 88 = 384 x 168); each role branch sets its own limit.
   if (warp >= 8) setmaxnreg_dec<88>();
   if (warp == 9 && lane == 0) {
-    // ---- TMA: per tile K and V, then (Q, dO, lse2, delta) per query block
+    // ---- TMA: per tile K and V, then (Q, dO, lse2, delta) per query block.
+    // lse2 and delta come from the prep kernel, which may still be running
+    // (programmatic launch): its writes are waited for before the first of them.
+    bool dep = false;
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_do);
     const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
@@ -359,6 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < G::DCH; ++c) {
         tma_load_3d(sbase + G::OFF_K + c * G::CHUNK, &tm_k, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
         tma_load_3d(sbase + G::OFF_V + c * G::CHUNK, &tm_v, B(G::B_KV), c * 64, kv_row0, T.bkv, pol_first);
+      }
+      if (!dep) {
+        grid_dep_wait();
+        dep = true;
       }
       const int nqb = T.nqb;
       for (int mm = 0; mm < 2 * T.nb; ++mm) {  // item mm: Q (even, + lse2, delta) or dO (odd) of block mm / 2
@@ -390,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       gate_par = static_cast<uint32_t>(it) & 1u;
       ++it;
     }
+    if (!dep) grid_dep_wait();  // (no tile with blocks: still no earlier exit than prep)
   } else if (BIAS && warp == 10 && lane == 0) {
     // ---- TMA: the bias tile of each (query block, key tile) pair: rows = the
     // block's queries (one row if broadcast over queries), columns = the tile's keys
@@ -914,6 +944,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 8) {
     // ---- compute: thread = query row r, warpgroup h = key columns h*64 .. +63
     setmaxnreg_inc<208>();
+    // the dK/dV kernel (and before it the prep kernel that wrote lse2 and delta)
+    // may still be running (programmatic launch); Q, K, V, dO are inputs, so only
+    // these warps wait
+    grid_dep_wait();
     const int h = warp >> 2, r = (warp & 3) * 32 + lane;
     const uint32_t tm = cx.tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.c;
@@ -933,7 +967,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const size_t srow = static_cast<size_t>(T.bh) * p.Nq_pad + qpos;
-      const float lse2 = p.lse2[srow], dlt = p.delta[srow];
+      const float lse2 = __ldcg(p.lse2 + srow), dlt = __ldcg(p.delta + srow);
       for (int j = 0; j < T.nb; ++j) {
         const int g = g0 + j;
         ok = wait_bar(B(G::B_SDP), g & 1u, cx.abort_flag);
@@ -1664,6 +1698,26 @@ bool overlaps_b(const void* a, size_t na, const void* b, size_t nb) {
 
 int nq_pad(int Nq) { return (Nq + 127) / 128 * 128; }
 
+// Launch with programmatic stream serialisation: the kernel may start while the
+// previous kernel in the stream still runs (once every CTA of that one has
+// signalled it, griddepcontrol.launch_dependents); it waits with
+// griddepcontrol.wait before it touches what that kernel writes.
+template <typename... Params, typename... Args>
+cudaError_t launch_after(void (*kern)(Params...), unsigned grid, int smem, cudaStream_t st,
+                         Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(fab::kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Parameters shared by the kernels, and the Delta / LSE * log2(e) pass.
 template <int D, bool BF16>
 int setup_bwd(fab::BwdParams& p, const void* o, const void* dout, const float* lse, void* dq,
@@ -1691,7 +1745,7 @@ int setup_bwd(fab::BwdParams& p, const void* o, const void* dout, const float* l
   p.lse2 = lse2;
   p.delta = delta;
   const long long rows = (long long)B * Hq * p.Nq_pad;
-  const long long warps_needed = (rows * (D / 8) + 31) / 32;
+  const long long warps_needed = (rows * (D / 8) + 32 * fab::kPrepGroups - 1) / (32 * fab::kPrepGroups);
   long long blocks = (warps_needed + 7) / 8;
   if (blocks > 16LL * sms) blocks = 16LL * sms;
   fab::bwd_prep_kernel<D, BF16><<<(unsigned)blocks, 256, 0, st>>>(
@@ -1789,15 +1843,16 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   // 2. dK, dV: persistent, one CTA per SM over the (b, kv head, key block) tiles
   const long long kv_tiles = (long long)B * Hkv * p.nkt;
   const unsigned kv_grid = (unsigned)(kv_tiles < sms ? kv_tiles : sms);
-  fab::bwd_dkdv_kernel<D, BF16, BIAS><<<kv_grid, fab::kThreads, GK::SMEM_BYTES, st>>>(
-      tq, tdo, tk, tv, p, tb, bias_mode);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  if (launch_after(fab::bwd_dkdv_kernel<D, BF16, BIAS>, kv_grid, GK::SMEM_BYTES, st, tq, tdo, tk, tv, p,
+                   tb, bias_mode) != cudaSuccess)
+    return FA_ERR_LAUNCH;
   // 3. dQ: persistent, one CTA per SM over the (b, query head, query block) tiles
   const long long q_tiles = (long long)B * Hq * p.nqt;
   const unsigned q_grid = (unsigned)(q_tiles < sms ? q_tiles : sms);
-  fab::bwd_dq_kernel<D, BF16, BIAS><<<q_grid, fab::kThreads, GQ::SMEM_BYTES, st>>>(
-      tq, tdo, tk, tv, p, tb, bias_mode);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  return launch_after(fab::bwd_dq_kernel<D, BF16, BIAS>, q_grid, GQ::SMEM_BYTES, st, tq, tdo, tk, tv, p,
+                      tb, bias_mode) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_LAUNCH;
 }
 
 }  // namespace
