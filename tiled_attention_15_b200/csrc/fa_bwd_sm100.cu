@@ -60,6 +60,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kBiasRowBcast = 1, kBiasPerHead = 2, kBiasPerBatch = 4;
 constexpr int kBiasTileBytes = 128 * 128 * 2;  // [2 boxes][128 rows][64 keys], 16-bit
 
+// Programmatic dependent launch: let the next kernel in the stream (launched
+// with programmatic stream serialisation) start; wait until the kernels this
+// one depends on have completed and their writes are visible.
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ unsigned int g_bwd_status = 0;
 __device__ unsigned long long g_bwd_site = 0;
 

@@ -28,13 +28,6 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t* w) {
                : "r"(addr)
                : "memory");
 }
-// Programmatic dependent launch: let the next kernel in the stream (launched
-// with programmatic stream serialisation) start; wait until the kernels this
-// one depends on have completed and their writes are visible.
-__device__ __forceinline__ void grid_dep_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
