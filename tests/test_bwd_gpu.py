@@ -108,6 +108,38 @@ def test_bwd_deterministic(cuda_dev):
         assert torch.equal(x, y)
 
 
+def test_bwd_back_to_back_calls(cuda_dev):
+    # two calls on one stream and one workspace, enqueued without a host wait: the
+    # second (other data, other shape) must see only its own Delta and LSE, and
+    # gives what the same call gives alone (the kernels of a call overlap their
+    # predecessor's tail through programmatic launch)
+    wa = Workload("bwd b2b a", 2, 40, 40, 512, 512, 128, "fp16", True, seed=101)
+    wb = Workload("bwd b2b b", 1, 40, 10, 640, 700, 128, "fp16", False, seed=102)
+    ws = torch.empty(max(fa.load_library().fa_bwd_workspace_size(w.B, w.Hq, w.Nq) for w in (wa, wb)),
+                     dtype=torch.uint8, device=cuda_dev)
+
+    def prepare(w):
+        q, k, v = (x.to(cuda_dev) for x in make_qkv(w))
+        g = _dout(w).to(cuda_dev)
+        o, lse = fa.fa_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal)
+        return q, k, v, o, lse, g
+
+    def bwd(w, t):
+        q, k, v, o, lse, g = t
+        return fa.fa_bwd(q, k, v, o, lse, g, scale=w.softmax_scale, causal=w.causal, workspace=ws)
+
+    ta, tb = prepare(wa), prepare(wb)
+    torch.cuda.synchronize()
+    alone = bwd(wb, tb)
+    torch.cuda.synchronize()
+    bwd(wa, ta)
+    after = bwd(wb, tb)  # enqueued right behind the first call
+    torch.cuda.synchronize()
+    assert fa.device_status(reset=True) == 0
+    for x, y in zip(alone, after):
+        assert torch.equal(x, y)
+
+
 def test_bwd_sum_invariants_on_device(cuda_dev):
     # the key-sum of dK vanishes and the key-sum of dV is the query-sum of dO
     w = Workload("bwd sums", 1, 2, 2, 512, 512, 64, "fp16", False, seed=101)
