@@ -24,7 +24,10 @@
 //   * causal attention skips key blocks above the diagonal and masks only the
 //     blocks that straddle it (or the key tail);
 //   * with NQ = 2 the two query tiles ping-pong: the tensor core works on one
-//     tile's S or PV while the other tile's softmax runs.
+//     tile's S or PV while the other tile's softmax runs;
+//   * the epilogue writes O row by row in 16-byte pieces, or (fp16 launches
+//     without a mask over at most 4096 keys: the STG instantiation) through a
+//     4 KB shared-memory stage per softmax warp as whole 128-byte lines.
 //
 // Tensor memory (512 columns x 128 lanes x 32 bit): S_0 at column 0, S_1 at
 // 128 (for NQ = 1 these are two S buffers of the single tile, used for
